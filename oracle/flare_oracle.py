@@ -1,0 +1,157 @@
+"""fp64 CPU oracle for the FLARE++ mixer forward -- TEST INFRASTRUCTURE ONLY.
+
+Only ``tests/``, ``__graft_entry__.smoke()`` and the CPU-baseline leg of
+``bench.py`` may import this module.  The library's CUDA path never calls it
+and shares no code with it.
+
+What it computes, per head (b, h), in float64, with scale s = 1 throughout:
+
+1. seed encode      Q_dyn = softmax_N(Q~ K^T) V       (softmax over the N tokens)
+2. routing encode   Z     = softmax_N(Q_dyn K^T) V
+3. decode           Y     = softmax_M(K Q_dyn^T) Z    (softmax over the M latents)
+
+Sources (page title, section):
+
+* "FLARE: Fast Low-rank Attention Routing Engine" (review page), section
+  "Основной механизм FLARE": the encode step Z_h = SDPA(Q_h, K_h, V_h, s=1)
+  with Q_h in R^{MxD} and K_h, V_h in R^{NxD}; the decode step
+  Y_h = SDPA(K_h, Q_h, Z_h, s=1).
+* same page, section "Матрица коммуникации низкого ранга": the weights
+  W_encode = softmax(Q K^T) (MxN, normalised over tokens),
+  W_decode = softmax(K Q^T) (NxM, normalised over latents) and
+  Y = (W_decode W_encode) V with W of rank at most M.
+* "FLARE++: Low-rank attention with dynamic attention routing", section
+  "Méthodologie : FLARE++": learned seeds Q~_h drive one extra encode call
+  whose M outputs become the routing queries Q_h(X) (dynamic query
+  synthesis), which then replace the learned queries in FLARE's encode-decode
+  pair (routing encode-decode).  The abstract states the same: one extra
+  encode call over the same N tokens.
+
+Readings taken where the pages are silent (listed with the others in the
+design notes): s = 1 in all three steps; the seed encode uses the same K and V
+as the routing encode; Q_dyn is used as-is (no normalisation) both as the
+routing queries and as the decode keys; softmax is max-subtracted, which is
+the same function.
+
+Every function here is "pinned" by tests in ``tests/test_oracle.py`` against
+things other than itself: the hand-derived worked examples in
+``tests/golden/``, a pure-Python brute force, torch's float64 SDPA, the dense
+NxN communication matrix, its rank and spectrum, and invariants of the
+definition.
+"""
+from __future__ import annotations
+
+import numpy as np
+
+__all__ = [
+    "softmax",
+    "sdpa",
+    "attention_weights",
+    "flare_encode",
+    "flare_decode",
+    "flarepp_head",
+    "flarepp_mix",
+    "flarepp_decode_rows",
+    "communication_matrix",
+    "communication_eigenvalues",
+]
+
+
+def softmax(S: np.ndarray, axis: int = -1) -> np.ndarray:
+    """Max-subtracted softmax along ``axis`` in float64."""
+    S = np.asarray(S, dtype=np.float64)
+    E = np.exp(S - S.max(axis=axis, keepdims=True))
+    return E / E.sum(axis=axis, keepdims=True)
+
+
+def attention_weights(q: np.ndarray, k: np.ndarray, scale: float = 1.0) -> np.ndarray:
+    """softmax(scale * q k^T) normalised over the rows of k (the keys)."""
+    q = np.asarray(q, dtype=np.float64)
+    k = np.asarray(k, dtype=np.float64)
+    return softmax(scale * (q @ k.T), axis=-1)
+
+
+def sdpa(q: np.ndarray, k: np.ndarray, v: np.ndarray, scale: float = 1.0) -> np.ndarray:
+    """Scaled dot-product attention softmax(scale q k^T) v, one head, float64."""
+    return attention_weights(q, k, scale) @ np.asarray(v, dtype=np.float64)
+
+
+def flare_encode(Q: np.ndarray, K: np.ndarray, V: np.ndarray) -> np.ndarray:
+    """FLARE encode of one head: the M queries gather the N tokens.
+
+    ``FLARE`` review page, "Основной механизм FLARE", encode step:
+    Z = SDPA(Q, K, V, s=1); Q is MxD, K and V are NxD, result MxD.
+    """
+    return sdpa(Q, K, V, 1.0)
+
+
+def flare_decode(K: np.ndarray, Q: np.ndarray, Z: np.ndarray) -> np.ndarray:
+    """FLARE decode of one head: each token's key queries the M latents.
+
+    ``FLARE`` review page, "Основной механизм FLARE", decode step:
+    Y = SDPA(K, Q, Z, s=1); the softmax runs over the M latents; result NxD.
+    """
+    return sdpa(K, Q, Z, 1.0)
+
+
+def flarepp_head(seeds: np.ndarray, K: np.ndarray, V: np.ndarray):
+    """The three chained steps of one FLARE++ head; returns (Q_dyn, Z, Y).
+
+    ``FLARE++`` page, "Méthodologie : FLARE++": dynamic query synthesis
+    (seeds query one extra encode over the tokens) followed by the standard
+    encode-decode pair driven by the synthesised queries.
+    """
+    Q_dyn = flare_encode(seeds, K, V)
+    Z = flare_encode(Q_dyn, K, V)
+    Y = flare_decode(K, Q_dyn, Z)
+    return Q_dyn, Z, Y
+
+
+def flarepp_decode_rows(K: np.ndarray, Q_dyn: np.ndarray, Z: np.ndarray, rows) -> np.ndarray:
+    """Decode output for the selected token rows only (each row is independent)."""
+    K = np.asarray(K, dtype=np.float64)
+    return flare_decode(K[np.asarray(rows)], Q_dyn, Z)
+
+
+def flarepp_mix(seeds: np.ndarray, K: np.ndarray, V: np.ndarray, heads=None):
+    """Whole mixer: seeds [H,M,D], K and V [B,H,N,D] -> (Q_dyn, Z, Y) float64.
+
+    ``heads`` optionally restricts the work to a list of (b, h) pairs; the
+    other entries of the outputs are left as NaN.
+    """
+    B, H, N, D = K.shape
+    M = seeds.shape[1]
+    Q_dyn = np.full((B, H, M, D), np.nan)
+    Z = np.full((B, H, M, D), np.nan)
+    Y = np.full((B, H, N, D), np.nan)
+    todo = heads if heads is not None else [(b, h) for b in range(B) for h in range(H)]
+    for b, h in todo:
+        Q_dyn[b, h], Z[b, h], Y[b, h] = flarepp_head(seeds[h], K[b, h], V[b, h])
+    return Q_dyn, Z, Y
+
+
+def communication_matrix(Q: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """The NxN global communication matrix W = W_decode W_encode of one head.
+
+    ``FLARE`` review page, "Матрица коммуникации низкого ранга": W_encode =
+    softmax(Q K^T) (MxN, over tokens), W_decode = softmax(K Q^T) (NxM, over
+    latents); the decode output equals W V and W has rank at most M.
+    """
+    W_enc = attention_weights(Q, K)  # M x N
+    W_dec = attention_weights(K, Q)  # N x M
+    return W_dec @ W_enc
+
+
+def communication_eigenvalues(Q: np.ndarray, K: np.ndarray) -> np.ndarray:
+    """Eigenvalues of W through the MxM product W_encode W_decode.
+
+    ``FLARE`` review page, "Спектральный анализ": the spectrum of the learned
+    communication matrices is obtained in O(M^3 + M^2 N) time.  The plainest
+    reading: the nonzero eigenvalues of W_dec W_enc (NxN) are those of
+    W_enc W_dec (MxM), which costs O(M^2 N) to form and O(M^3) to solve.
+    Returned sorted by decreasing modulus.
+    """
+    W_enc = attention_weights(Q, K)
+    W_dec = attention_weights(K, Q)
+    ev = np.linalg.eigvals(W_enc @ W_dec)
+    return ev[np.argsort(-np.abs(ev))]

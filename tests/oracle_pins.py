@@ -1,0 +1,253 @@
+"""Pins for the fp64 oracle: checks against things other than the oracle itself.
+
+Each ``pin_*`` function takes an oracle module ``o`` and raises AssertionError
+when ``o`` disagrees with the reference it pins against.  ``tests/test_oracle.py``
+runs every pin on the real oracle; ``tests/test_oracle_mutations.py`` plants
+plausible mistakes in copies of the oracle's source and checks that each
+mistake fails at least one pin.
+
+What pins what:
+
+* worked examples (``tests/golden/worked_examples.json``): hand-derived exact
+  fractions for the chained FLARE++ head (composition, operand roles, scale,
+  softmax axes).
+* torch float64 SDPA: each of ``flare_encode`` / ``flare_decode`` is one SDPA
+  call with scale 1 ("FLARE" review page, "Основной механизм FLARE").
+* pure-Python brute force: scalar loops with ``math.exp`` following the
+  definitions, independent of NumPy.
+* dense construction: explicit W_encode (MxN) and W_decode (NxM) from the
+  "Матрица коммуникации низкого ранга" section; the FLARE output is W V.
+* rank and spectrum: W has numerical rank <= M; its nonzero eigenvalues are
+  those of W_encode W_decode ("Спектральный анализ").
+* invariants of the definition: row sums, K = 0, M = 1, N = 1, constant V,
+  token permutation, key shift, convex hull.
+"""
+from __future__ import annotations
+
+import json
+import math
+import os
+from fractions import Fraction
+
+import numpy as np
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "worked_examples.json")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _case(seed, N, M, D, std=0.7):
+    g = _rng(seed)
+    return (g.standard_normal((M, D)) * std, g.standard_normal((N, D)) * std,
+            g.standard_normal((N, D)) * std)
+
+
+# ---------------------------------------------------------------- worked examples
+def _parse_key(s: str) -> float:
+    s = s.strip()
+    if s.startswith("ln(") and s.endswith(")"):
+        return math.log(float(Fraction(s[3:-1])))
+    return float(Fraction(s))
+
+
+def _frac(s: str) -> float:
+    return float(Fraction(s))
+
+
+def pin_worked_examples(o):
+    with open(GOLDEN) as f:
+        data = json.load(f)
+    for ex in data["examples"]:
+        seeds = np.array([[_parse_key(x) for x in r] for r in ex["seeds"]])
+        K = np.array([[_parse_key(x) for x in r] for r in ex["K"]])
+        V = np.array([[_parse_key(x) for x in r] for r in ex["V"]])
+        Qd, Z, Y = o.flarepp_head(seeds, K, V)
+        for name, got in (("Q_dyn", Qd), ("Z", Z), ("Y", Y)):
+            want = np.array([[_frac(x) for x in r] for r in ex[name]])
+            assert got.shape == want.shape, (ex["name"], name, got.shape, want.shape)
+            assert np.allclose(got, want, rtol=1e-13, atol=1e-13), (ex["name"], name, got, want)
+
+
+# ---------------------------------------------------------------- torch SDPA
+def pin_torch_sdpa(o):
+    import torch
+    import torch.nn.functional as F
+
+    for seed, (N, M, D) in enumerate([(37, 5, 3), (200, 16, 8), (129, 1, 4), (1, 3, 2), (64, 64, 16)]):
+        Q, K, V = _case(100 + seed, N, M, D)
+        tq, tk, tv = (torch.from_numpy(x) for x in (Q, K, V))
+        want_enc = F.scaled_dot_product_attention(tq[None], tk[None], tv[None], scale=1.0)[0].numpy()
+        got_enc = o.flare_encode(Q, K, V)
+        assert np.allclose(got_enc, want_enc, rtol=1e-12, atol=1e-13), ("encode", N, M, D)
+        Zl = _rng(200 + seed).standard_normal((M, D))
+        want_dec = F.scaled_dot_product_attention(tk[None], tq[None], torch.from_numpy(Zl)[None],
+                                                  scale=1.0)[0].numpy()
+        got_dec = o.flare_decode(K, Q, Zl)
+        assert np.allclose(got_dec, want_dec, rtol=1e-12, atol=1e-13), ("decode", N, M, D)
+
+
+# ---------------------------------------------------------------- brute force
+def _bf_encode(Q, K, V):
+    M, N, D = len(Q), len(K), len(V[0])
+    out = []
+    for m in range(M):
+        logits = [sum(Q[m][d] * K[n][d] for d in range(len(K[0]))) for n in range(N)]
+        top = max(logits)
+        w = [math.exp(x - top) for x in logits]
+        tot = math.fsum(w)
+        out.append([math.fsum(w[n] * V[n][d] for n in range(N)) / tot for d in range(D)])
+    return out
+
+
+def _bf_decode(K, Q, Z):
+    N, M, D = len(K), len(Q), len(Z[0])
+    out = []
+    for n in range(N):
+        logits = [sum(K[n][d] * Q[m][d] for d in range(len(K[0]))) for m in range(M)]
+        top = max(logits)
+        w = [math.exp(x - top) for x in logits]
+        tot = math.fsum(w)
+        out.append([math.fsum(w[m] * Z[m][d] for m in range(M)) / tot for d in range(D)])
+    return out
+
+
+def brute_force_head(seeds, K, V):
+    seeds, K, V = seeds.tolist(), K.tolist(), V.tolist()
+    Qd = _bf_encode(seeds, K, V)
+    Z = _bf_encode(Qd, K, V)
+    Y = _bf_decode(K, Qd, Z)
+    return np.array(Qd), np.array(Z), np.array(Y)
+
+
+def pin_brute_force(o):
+    for seed, (N, M, D) in enumerate([(1, 1, 1), (2, 1, 2), (5, 3, 2), (8, 4, 3), (7, 2, 1), (6, 4, 4)]):
+        S, K, V = _case(300 + seed, N, M, D, std=1.1)
+        want = brute_force_head(S, K, V)
+        got = o.flarepp_head(S, K, V)
+        for name, g, w in zip(("Q_dyn", "Z", "Y"), got, want):
+            assert np.allclose(g, w, rtol=1e-12, atol=1e-13), (name, N, M, D)
+
+
+# ---------------------------------------------------------------- dense NxN operator
+def _bf_weights(A, B):
+    """softmax over the rows of B of A B^T, by scalar loops."""
+    out = []
+    for a in A:
+        logits = [sum(x * y for x, y in zip(a, b)) for b in B]
+        top = max(logits)
+        w = [math.exp(x - top) for x in logits]
+        tot = math.fsum(w)
+        out.append([x / tot for x in w])
+    return np.array(out)
+
+
+def pin_dense_operator(o):
+    for seed, (N, M, D) in enumerate([(12, 3, 2), (40, 5, 4), (9, 9, 3)]):
+        Q, K, V = _case(400 + seed, N, M, D)
+        W_enc = _bf_weights(Q.tolist(), K.tolist())  # M x N
+        W_dec = _bf_weights(K.tolist(), Q.tolist())  # N x M
+        W = W_dec @ W_enc
+        assert np.allclose(o.communication_matrix(Q, K), W, rtol=1e-12, atol=1e-14)
+        Z = o.flare_encode(Q, K, V)
+        assert np.allclose(Z, W_enc @ V, rtol=1e-12, atol=1e-13)
+        Y = o.flare_decode(K, Q, Z)
+        assert np.allclose(Y, W @ V, rtol=1e-12, atol=1e-13)
+        assert np.allclose(o.attention_weights(Q, K), W_enc, rtol=1e-12, atol=1e-14)
+
+
+def pin_rank_and_spectrum(o):
+    for seed, (N, M, D) in enumerate([(64, 4, 8), (48, 7, 3)]):
+        Q, K, _ = _case(500 + seed, N, M, D, std=1.0)
+        W = o.communication_matrix(Q, K)
+        sv = np.linalg.svd(W, compute_uv=False)
+        assert sv[M] / sv[0] < 1e-12, ("rank", sv[: M + 2])
+        assert np.allclose(W.sum(axis=1), 1.0, atol=1e-13)  # row-stochastic
+        ev_small = o.communication_eigenvalues(Q, K)
+        ev_big = np.linalg.eigvals(W)
+        ev_big = ev_big[np.argsort(-np.abs(ev_big))][:M]
+        assert np.allclose(np.sort_complex(ev_small), np.sort_complex(ev_big), atol=1e-10), (ev_small, ev_big)
+        assert abs(ev_small[0] - 1.0) < 1e-10  # W 1 = 1, and W_enc W_dec is row-stochastic too
+
+
+# ---------------------------------------------------------------- invariants
+def pin_invariants(o):
+    N, M, D = 50, 6, 4
+    S, K, V = _case(600, N, M, D, std=0.9)
+
+    # every attention row sums to one, for all three steps
+    Qd, Z, Y = o.flarepp_head(S, K, V)
+    for A in (o.attention_weights(S, K), o.attention_weights(Qd, K), o.attention_weights(K, Qd)):
+        assert np.allclose(A.sum(axis=1), 1.0, atol=1e-13)
+
+    # K = 0: every encode weight is 1/N, so Q_dyn = Z = mean(V), and Y rows = mean(V)
+    mean = V.mean(axis=0)
+    Qd0, Z0, Y0 = o.flarepp_head(S, np.zeros_like(K), V)
+    assert np.allclose(Qd0, mean[None], atol=1e-13)
+    assert np.allclose(Z0, mean[None], atol=1e-13)
+    assert np.allclose(Y0, mean[None], atol=1e-13)
+
+    # M = 1: the decode softmax over one latent is 1, so every Y row equals Z
+    Qd1, Z1, Y1 = o.flarepp_head(S[:1], K, V)
+    assert np.allclose(Y1, Z1[0][None], atol=1e-13)
+
+    # N = 1: every softmax over tokens picks the single token
+    Qdn, Zn, Yn = o.flarepp_head(S, K[:1], V[:1])
+    assert np.allclose(Qdn, V[:1], atol=1e-13) and np.allclose(Zn, V[:1], atol=1e-13)
+    assert np.allclose(Yn, V[:1], atol=1e-13)
+
+    # constant V: every convex combination returns that constant
+    c = _rng(601).standard_normal(D)
+    _, _, Yc = o.flarepp_head(S, K, np.tile(c, (N, 1)))
+    assert np.allclose(Yc, c[None], atol=1e-13)
+
+    # token permutation: Q_dyn and Z unchanged, Y permuted the same way
+    p = _rng(602).permutation(N)
+    Qdp, Zp, Yp = o.flarepp_head(S, K[p], V[p])
+    assert np.allclose(Qdp, Qd, atol=1e-13) and np.allclose(Zp, Z, atol=1e-13)
+    assert np.allclose(Yp, Y[p], atol=1e-13)
+
+    # key shift K -> K + 1 u^T: each encode row's logits move by a constant
+    u = _rng(603).standard_normal(D)
+    Qds, Zs, Ys = o.flarepp_head(S, K + u[None], V)
+    assert np.allclose(Qds, Qd, atol=1e-12) and np.allclose(Zs, Z, atol=1e-12)
+    assert not np.allclose(Ys, Y, atol=1e-6)  # the decode is not shift invariant
+
+    # decode query shift Q -> Q + 1 c^T leaves the decode weights unchanged
+    cq = _rng(604).standard_normal(D)
+    assert np.allclose(o.flare_decode(K, Qd + cq[None], Z), o.flare_decode(K, Qd, Z), atol=1e-12)
+
+    # convex hull: every output lies within [min_n V, max_n V] per channel
+    lo, hi = V.min(axis=0), V.max(axis=0)
+    for X in (Qd, Z, Y):
+        assert np.all(X >= lo - 1e-13) and np.all(X <= hi + 1e-13)
+
+
+def pin_mix_layout(o):
+    """flarepp_mix applies one head's chain per (b, h) with seeds shared over the batch."""
+    B, H, N, M, D = 2, 3, 11, 4, 2
+    g = _rng(700)
+    seeds = g.standard_normal((H, M, D))
+    K = g.standard_normal((B, H, N, D))
+    V = g.standard_normal((B, H, N, D))
+    Qd, Z, Y = o.flarepp_mix(seeds, K, V)
+    for b in range(B):
+        for h in range(H):
+            want = brute_force_head(seeds[h], K[b, h], V[b, h])
+            for got, w in zip((Qd[b, h], Z[b, h], Y[b, h]), want):
+                assert np.allclose(got, w, rtol=1e-12, atol=1e-13), (b, h)
+    rows = [0, 5, 10]
+    Yr = o.flarepp_decode_rows(K[1, 2], Qd[1, 2], Z[1, 2], rows)
+    assert np.allclose(Yr, Y[1, 2][rows], atol=1e-14)
+
+
+ALL_PINS = [
+    pin_worked_examples,
+    pin_torch_sdpa,
+    pin_brute_force,
+    pin_dense_operator,
+    pin_rank_and_spectrum,
+    pin_invariants,
+    pin_mix_layout,
+]

@@ -1,0 +1,66 @@
+"""Plant plausible mistakes in copies of the oracle and check that the pins catch each.
+
+Every mutant is the oracle's own source with one textual edit, executed as a
+fresh module on the CPU.  A mutant that passes every pin would mean the pins
+cannot tell that mistake from the definition.
+"""
+import inspect
+import types
+
+import pytest
+
+import oracle.flare_oracle as base
+import oracle_pins
+
+MUTANTS = {
+    # scale 1/sqrt(D) instead of the pages' s = 1
+    "scale_rsqrt_d": ("return sdpa(Q, K, V, 1.0)", "return sdpa(Q, K, V, 1.0 / np.sqrt(Q.shape[1]))"),
+    # encode softmax normalised over the latents instead of the tokens
+    "encode_wrong_axis": ("return sdpa(Q, K, V, 1.0)",
+                          "return softmax(Q @ K.T, axis=0) @ np.asarray(V, dtype=np.float64)"),
+    # sign flip of the logits
+    "negated_logits": ("return softmax(scale * (q @ k.T), axis=-1)", "return softmax(-scale * (q @ k.T), axis=-1)"),
+    # decode keys taken from Z instead of Q_dyn
+    "decode_keys_from_Z": ("Y = flare_decode(K, Q_dyn, Z)", "Y = flare_decode(K, Z, Z)"),
+    # decode keys taken from the seeds instead of Q_dyn
+    "decode_keys_from_seeds": ("Y = flare_decode(K, Q_dyn, Z)", "Y = flare_decode(K, seeds, Z)"),
+    # routing encode driven by the seeds again (no dynamic routing)
+    "routing_uses_seeds": ("Z = flare_encode(Q_dyn, K, V)", "Z = flare_encode(seeds, K, V)"),
+    # encode values taken from K (dropped V term)
+    "encode_values_from_K": ("return sdpa(Q, K, V, 1.0)", "return sdpa(Q, K, K, 1.0)"),
+    # decode as the transpose of the encode weights
+    "decode_transposed_weights": ("return sdpa(K, Q, Z, 1.0)",
+                                  "return attention_weights(Q, K).T @ np.asarray(Z, dtype=np.float64)"),
+    # off-by-one in the token index of the values
+    "values_shifted": ("return sdpa(Q, K, V, 1.0)", "return sdpa(Q, K, np.roll(V, 1, axis=0), 1.0)"),
+    # unnormalised weights (dropped denominator)
+    "no_normalisation": ("return E / E.sum(axis=axis, keepdims=True)", "return E"),
+    # decode values taken from Q_dyn instead of Z
+    "decode_values_qdyn": ("Y = flare_decode(K, Q_dyn, Z)", "Y = flare_decode(K, Q_dyn, Q_dyn)"),
+    # the spectral tool using the NxN order of the product
+    "eig_wrong_product": ("ev = np.linalg.eigvals(W_enc @ W_dec)", "ev = np.linalg.eigvals(W_enc @ W_enc.T)"),
+    # communication matrix built from transposed factors (still NxN)
+    "comm_transposed_factors": ("return W_dec @ W_enc", "return W_enc.T @ W_dec.T"),
+}
+
+
+def _mutant(find, repl):
+    src = inspect.getsource(base)
+    assert src.count(find) == 1, f"mutation anchor not unique/absent: {find!r}"
+    mod = types.ModuleType("oracle_mutant")
+    exec(compile(src.replace(find, repl), "<oracle_mutant>", "exec"), mod.__dict__)
+    return mod
+
+
+@pytest.mark.parametrize("name", sorted(MUTANTS))
+def test_mutant_is_caught(name):
+    mod = _mutant(*MUTANTS[name])
+    caught = []
+    for pin in oracle_pins.ALL_PINS:
+        try:
+            pin(mod)
+        except AssertionError:
+            caught.append(pin.__name__)
+        except Exception as e:  # a crash on a pin input also exposes the mutant
+            caught.append(f"{pin.__name__}:{type(e).__name__}")
+    assert caught, f"mutant {name} passed every pin"
