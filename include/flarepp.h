@@ -1,0 +1,150 @@
+/*
+ * flarepp.h -- C ABI of the FLARE++ token-mixer forward pass for NVIDIA B200
+ * (sm_100a).  Implemented by libflarepp.so (rank_latent_attention_b200/).
+ *
+ * The mixer routes N tokens through M << N latents, per head (b, h), in three
+ * chained attention steps with scale s = 1:
+ *
+ *   seed encode     Q_dyn = softmax_N(Q~ K^T) V      Q~ = learned seeds of head h
+ *   routing encode  Z     = softmax_N(Q_dyn K^T) V
+ *   decode          Y     = softmax_M(K Q_dyn^T) Z
+ *
+ * Sources: the FLARE encode Z_h = SDPA(Q_h, K_h, V_h, s=1) and decode
+ * Y_h = SDPA(K_h, Q_h, Z_h, s=1) ("FLARE: Fast Low-rank Attention Routing
+ * Engine", review page, section "Основной механизм FLARE"); FLARE++ replaces
+ * the learned queries by Q_dyn, produced by one extra encode driven by the
+ * seeds ("FLARE++: Low-rank attention with dynamic attention routing",
+ * section "Méthodologie : FLARE++", items "Synthèse de Requêtes Dynamiques"
+ * and "Routage Encode-Décode"; abstract).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are dense, row-major, contiguous, in DEVICE memory owned by the
+ *   caller, and 16-byte aligned:
+ *     seeds / fixed queries  [H][M][D]      (shared by the batch)
+ *     batched queries        [B][H][M][D]
+ *     K, V, Y                [B][H][N][D]
+ *     Q_dyn, Z               [B][H][M][D]
+ * - dtype is FLARE_BF16 (bf16 storage, fp32 accumulation and fp32 softmax on
+ *   the tensor cores; intermediates Q_dyn and Z are stored as bf16, rounded to
+ *   nearest) or FLARE_F32 (fp32 everywhere, CUDA-core path).  Every tensor of
+ *   a call has that dtype.
+ * - Supported sizes: B >= 1, H >= 1, B*H <= 65535, 1 <= N < 2^31 - 256,
+ *   D in {16, 32, 64, 128}, 1 <= M <= 256; for FLARE_BF16 additionally
+ *   M % 16 == 0.  N needs no alignment: the last tile of each head is masked.
+ * - stream is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *   Work is enqueued asynchronously; nothing synchronises the host.
+ * - Return value: a flare_status_t.  Invalid arguments (null or unaligned
+ *   pointers, host pointers, unsupported sizes, a workspace that is too
+ *   small) return an error before any work is enqueued.  FLARE_ERR_CUDA means
+ *   a launch failed; the CUDA error is left for cudaGetLastError.  The kernels
+ *   never trap: a wait inside a kernel that exceeds the wait limit records
+ *   FLARE_ERR_TIMEOUT in a per-device status word that flare_check_status
+ *   reports.
+ * - Workspace: device scratch of at least the size returned by the matching
+ *   *_workspace_size function, owned by the caller, 256-byte aligned.  If
+ *   workspace is NULL the library allocates it with cudaMallocAsync on the
+ *   stream and frees it with cudaFreeAsync after the last kernel.
+ */
+#ifndef FLAREPP_H
+#define FLAREPP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { FLARE_F32 = 0, FLARE_BF16 = 1 } flare_dtype_t;
+
+typedef enum {
+  FLARE_OK = 0,
+  FLARE_ERR_INVALID_ARG = 1,  /* null/unaligned/host pointer, bad enum, workspace too small */
+  FLARE_ERR_UNSUPPORTED = 2,  /* sizes outside the supported set */
+  FLARE_ERR_CUDA = 3,         /* a CUDA call or kernel launch failed */
+  FLARE_ERR_TIMEOUT = 4       /* a kernel gave up waiting (reported by flare_check_status) */
+} flare_status_t;
+
+/* Bytes of workspace flare_encode needs for these sizes (0 for invalid sizes). */
+size_t flare_encode_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+
+/* Bytes of workspace flarepp_mix / flarepp_mix_debug need (0 for invalid sizes). */
+size_t flarepp_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+
+/*
+ * FLARE encode: Z[b,h] = softmax_N(Q K[b,h]^T) V[b,h], softmax over the N tokens.
+ * ("FLARE" review page, "Основной механизм FLARE", encode step.)
+ *   Q          [H][M][D] if q_batched == 0 (learned queries, shared by the batch)
+ *              [B][H][M][D] if q_batched == 1
+ *   K, V       [B][H][N][D]
+ *   Z          [B][H][M][D] output
+ * The token axis is split across CTAs; the per-split softmax statistics are
+ * merged exactly (log-sum-exp) in a second kernel.
+ */
+int flare_encode(const void* Q, int q_batched, const void* K, const void* V, void* Z, int B, int H, int64_t N,
+                 int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * FLARE decode: Y[b,h][n] = softmax_M(K[b,h][n] . Q^T) Z[b,h], softmax over the
+ * M latents, one row per token.  ("FLARE" review page, "Основной механизм
+ * FLARE", decode step Y = SDPA(K, Q, Z, s=1).)
+ *   K          [B][H][N][D]
+ *   Q          latent keys: [H][M][D] if q_batched == 0, [B][H][M][D] if 1
+ *   Z          [B][H][M][D]
+ *   Y          [B][H][N][D] output
+ * Needs no workspace.
+ */
+int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N,
+                 int M, int D, int dtype, void* stream);
+
+/*
+ * FLARE++ mixer forward: seed encode -> routing encode -> decode (see top).
+ *   seeds      [H][M][D]
+ *   K, V       [B][H][N][D]
+ *   Y          [B][H][N][D] output
+ * K and V are streamed from memory three times in all (K, V; K, V; K) and Y
+ * written once; Q_dyn and Z live in the workspace.
+ */
+int flarepp_mix(const void* seeds, const void* K, const void* V, void* Y, int B, int H, int64_t N, int M, int D,
+                int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Same as flarepp_mix, and also returns the intermediates: Q_dyn and Z
+ * ([B][H][M][D], dtype) are written to the caller's buffers, which the later
+ * steps then read, so the returned values are exactly the ones used.
+ */
+int flarepp_mix_debug(const void* seeds, const void* K, const void* V, void* Y, void* Q_dyn, void* Z, int B, int H,
+                      int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
+ * Synchronises `stream`, then reads and clears the current device's status
+ * word.  Returns FLARE_OK or the first error a kernel recorded since the last
+ * check (FLARE_ERR_TIMEOUT); *site (if not NULL) receives the kernel role
+ * that recorded it (1-3 encode producer/MMA/softmax, 4-6 decode).  Returns
+ * FLARE_ERR_CUDA if the synchronisation itself fails.
+ */
+int flare_check_status(void* stream, int* site);
+
+/* Static, human-readable name of a status code. */
+const char* flare_status_string(int status);
+
+/* Number of kernels the last successful call on this host thread enqueued. */
+int flare_last_launch_count(void);
+
+/*
+ * Tuning / test hooks (process-wide, not thread-safe against concurrent calls):
+ *   flare_set_split_override(s): use s CTAs per head along the tokens (clamped
+ *     to the number of 128-token tiles); 0 restores the built-in choice.
+ *   flare_set_wait_limit_ms(ms): how long a tensor-core kernel waits on one
+ *     barrier before recording FLARE_ERR_TIMEOUT and returning (default 2000).
+ * Both return the previous value.
+ */
+int flare_set_split_override(int splits);
+int flare_set_wait_limit_ms(int ms);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FLAREPP_H */

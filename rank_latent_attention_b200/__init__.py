@@ -1,0 +1,223 @@
+"""FLARE++ token-mixer forward for NVIDIA B200 (sm_100a).
+
+Python binding of ``libflarepp.so`` (C ABI declared in ``include/flarepp.h``).
+The functions here only marshal torch CUDA tensors into pointers and sizes
+and call the library with the same names; every step of the computation runs
+in the library's CUDA kernels.  There is no fallback: if the library is not
+built, or a tensor is not on a CUDA device, the call raises.
+
+    seed encode     Q_dyn = softmax_N(Q~ K^T) V
+    routing encode  Z     = softmax_N(Q_dyn K^T) V
+    decode          Y     = softmax_M(K Q_dyn^T) Z          (scale 1 throughout)
+
+Layouts: seeds / fixed queries [H, M, D]; K, V, Y [B, H, N, D]; Q_dyn, Z
+[B, H, M, D]; contiguous; dtype torch.bfloat16 (tensor cores) or
+torch.float32 (CUDA cores).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import re
+
+__all__ = [
+    "FlareError",
+    "lib",
+    "flare_encode",
+    "flare_decode",
+    "flarepp_mix",
+    "flarepp_mix_debug",
+    "flare_encode_workspace_size",
+    "flarepp_workspace_size",
+    "flare_check_status",
+    "flare_last_launch_count",
+    "flare_set_split_override",
+    "flare_set_wait_limit_ms",
+    "LIB_PATH",
+    "HEADER_PATH",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libflarepp.so")
+HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "flarepp.h")
+
+F32, BF16 = 0, 1
+_c_int, _c_i64, _c_size, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
+_SIZES = [_c_int, _c_int, _c_i64, _c_int, _c_int, _c_int]  # B, H, N, M, D, dtype
+
+_SIGNATURES = {
+    "flare_encode_workspace_size": (_c_size, _SIZES),
+    "flarepp_workspace_size": (_c_size, _SIZES),
+    "flare_encode": (_c_int, [_vp, _c_int, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
+    "flare_decode": (_c_int, [_vp, _vp, _c_int, _vp, _vp, *_SIZES, _vp]),
+    "flarepp_mix": (_c_int, [_vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
+    "flarepp_mix_debug": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
+    "flare_check_status": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
+    "flare_status_string": (ctypes.c_char_p, [_c_int]),
+    "flare_last_launch_count": (_c_int, []),
+    "flare_set_split_override": (_c_int, [_c_int]),
+    "flare_set_wait_limit_ms": (_c_int, [_c_int]),
+}
+
+_lib = None
+
+
+class FlareError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {lib().flare_status_string(status).decode()} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """The loaded ``libflarepp.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing; build it with "
+                               "`python -m rank_latent_attention_b200.build`")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGNATURES.items():
+            fn = getattr(handle, name)
+            fn.restype, fn.argtypes = res, args
+        _lib = handle
+    return _lib
+
+
+def header_functions() -> list[str]:
+    """Names of the functions ``include/flarepp.h`` declares."""
+    with open(HEADER_PATH) as f:
+        text = f.read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return re.findall(r"^\s*(?:const\s+)?[A-Za-z_][\w\s\*]*?\b(flare\w*)\s*\(", text, flags=re.M)
+
+
+# ---------------------------------------------------------------- marshalling
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return BF16
+    if t.dtype == torch.float32:
+        return F32
+    raise TypeError(f"unsupported dtype {t.dtype}; use torch.bfloat16 or torch.float32")
+
+
+def _ptr(t, name: str, dtype):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor (no CPU path exists)")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} has dtype {t.dtype}, expected {dtype}")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream()
+    return ctypes.c_void_p(s.cuda_stream)
+
+
+def _check(rc: int, where: str):
+    if rc != 0:
+        raise FlareError(rc, where)
+
+
+def _ws(workspace):
+    if workspace is None:
+        return None, 0
+    return ctypes.c_void_p(workspace.data_ptr()), workspace.numel() * workspace.element_size()
+
+
+def flare_encode_workspace_size(B, H, N, M, D, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (BF16 if "bfloat16" in str(dtype) else F32)
+    return lib().flare_encode_workspace_size(B, H, N, M, D, code)
+
+
+def flarepp_workspace_size(B, H, N, M, D, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (BF16 if "bfloat16" in str(dtype) else F32)
+    return lib().flarepp_workspace_size(B, H, N, M, D, code)
+
+
+def flare_encode(Q, K, V, Z=None, *, workspace=None, stream=None):
+    """FLARE encode Z = softmax_N(Q K^T) V.  Q is [H,M,D] (shared) or [B,H,M,D]."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    q_batched = 1 if Q.dim() == 4 else 0
+    M = Q.shape[-2]
+    if Z is None:
+        Z = torch.empty((B, H, M, D), dtype=K.dtype, device=K.device)
+    ws, wsb = _ws(workspace)
+    _check(lib().flare_encode(_ptr(Q, "Q", K.dtype), q_batched, _ptr(K, "K", K.dtype), _ptr(V, "V", K.dtype),
+                              _ptr(Z, "Z", K.dtype), B, H, N, M, D, _dtype_code(K), ws, wsb, _stream(stream)),
+           "flare_encode")
+    return Z
+
+
+def flare_decode(K, Q, Z, Y=None, *, stream=None):
+    """FLARE decode Y = softmax_M(K Q^T) Z.  Q is [H,M,D] (shared) or [B,H,M,D]."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    q_batched = 1 if Q.dim() == 4 else 0
+    M = Q.shape[-2]
+    if Y is None:
+        Y = torch.empty_like(K)
+    _check(lib().flare_decode(_ptr(K, "K", K.dtype), _ptr(Q, "Q", K.dtype), q_batched, _ptr(Z, "Z", K.dtype),
+                              _ptr(Y, "Y", K.dtype), B, H, N, M, D, _dtype_code(K), _stream(stream)),
+           "flare_decode")
+    return Y
+
+
+def flarepp_mix(seeds, K, V, Y=None, *, workspace=None, stream=None):
+    """FLARE++ mixer forward: seeds [H,M,D], K/V [B,H,N,D] -> Y [B,H,N,D]."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = seeds.shape[1]
+    if Y is None:
+        Y = torch.empty_like(K)
+    ws, wsb = _ws(workspace)
+    _check(lib().flarepp_mix(_ptr(seeds, "seeds", K.dtype), _ptr(K, "K", K.dtype), _ptr(V, "V", K.dtype),
+                             _ptr(Y, "Y", K.dtype), B, H, N, M, D, _dtype_code(K), ws, wsb, _stream(stream)),
+           "flarepp_mix")
+    return Y
+
+
+def flarepp_mix_debug(seeds, K, V, *, workspace=None, stream=None):
+    """As flarepp_mix, also returning the intermediates: (Y, Q_dyn, Z)."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = seeds.shape[1]
+    Y = torch.empty_like(K)
+    Qd = torch.empty((B, H, M, D), dtype=K.dtype, device=K.device)
+    Z = torch.empty_like(Qd)
+    ws, wsb = _ws(workspace)
+    _check(lib().flarepp_mix_debug(_ptr(seeds, "seeds", K.dtype), _ptr(K, "K", K.dtype), _ptr(V, "V", K.dtype),
+                                   _ptr(Y, "Y", K.dtype), _ptr(Qd, "Q_dyn", K.dtype), _ptr(Z, "Z", K.dtype),
+                                   B, H, N, M, D, _dtype_code(K), ws, wsb, _stream(stream)),
+           "flarepp_mix_debug")
+    return Y, Qd, Z
+
+
+def flare_check_status(stream=None) -> tuple[int, int]:
+    """Synchronise the stream and return (status, site) of the device status word (cleared)."""
+    site = ctypes.c_int(0)
+    rc = lib().flare_check_status(_stream(stream), ctypes.byref(site))
+    return rc, site.value
+
+
+def flare_last_launch_count() -> int:
+    return lib().flare_last_launch_count()
+
+
+def flare_set_split_override(splits: int) -> int:
+    return lib().flare_set_split_override(splits)
+
+
+def flare_set_wait_limit_ms(ms: int) -> int:
+    return lib().flare_set_wait_limit_ms(ms)

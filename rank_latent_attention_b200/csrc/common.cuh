@@ -1,0 +1,67 @@
+// Shared definitions of the FLARE++ kernels: status codes, the device status
+// word, tile geometry of the bf16 tensor-core path and smem descriptor helpers.
+#pragma once
+
+#include <stdint.h>
+
+#include "ptx_sm100.cuh"
+
+namespace flare {
+
+// Status codes shared with include/flarepp.h.
+enum : int {
+  kOk = 0,
+  kErrInvalidArg = 1,
+  kErrUnsupported = 2,
+  kErrCuda = 3,
+  kErrTimeout = 4,
+};
+
+// Where a bounded wait gave up (second word of the device status).
+enum : int {
+  kSiteEncProducer = 1,
+  kSiteEncMma = 2,
+  kSiteEncSoftmax = 3,
+  kSiteDecProducer = 4,
+  kSiteDecMma = 5,
+  kSiteDecSoftmax = 6,
+};
+
+constexpr float kLog2e = 1.4426950408889634f;
+constexpr int kTileN = 128;   // tokens per tile (MMA M of the decode, N of the encode)
+constexpr int kLatRows = 128; // latent rows per tcgen05 MMA (M = 128, cta_group::1)
+
+// Record the first failure in the device status word {code, site}.
+__device__ __forceinline__ void record_error(int* status, int code, int site) {
+  if (atomicCAS(status, 0, code) == 0) atomicExch(status + 1, site);
+}
+
+// Geometry of a [rows][D] bf16 tile in shared memory as written by a TMA
+// load with the swizzle matching its row width:
+//   D <= 64 : one block, row pitch 2*D bytes (32/64/128 B swizzle);
+//   D == 128: two 64-column blocks of [rows][64], each with 128 B rows.
+template <int D>
+struct TileGeom {
+  static_assert(D == 16 || D == 32 || D == 64 || D == 128, "D must be 16, 32, 64 or 128");
+  static constexpr int kRowBytes = D >= 64 ? 128 : 2 * D;   // row pitch inside one column block
+  static constexpr int kBlocks = D > 64 ? D / 64 : 1;        // 64-column blocks
+  static constexpr int kBoxCols = D >= 64 ? 64 : D;          // TMA box inner extent (elements)
+  static constexpr uint32_t kSwizzle = D >= 64 ? 2u : (D == 32 ? 4u : 6u);  // descriptor code
+  static constexpr int kAtomBytes = 8 * kRowBytes;           // 8-row swizzle atom
+
+  // K-major operand (rows = M or N of the MMA, D = reduction dim), K step k of 16.
+  __device__ static __forceinline__ uint64_t kmajor(uint32_t base, int rows, int k) {
+    // 16 elements = 32 bytes along the row; past 64 elements, the next column block.
+    const int elem = k * 16;
+    const uint32_t addr = base + (elem / 64) * rows * 128 + (elem % 64) * 2;
+    return ptx::smem_desc(addr, 16, kAtomBytes, kSwizzle);
+  }
+  // MN-major operand (rows = reduction dim, D = N of the MMA), K step k of 16 rows.
+  __device__ static __forceinline__ uint64_t mnmajor(uint32_t base, int rows, int k) {
+    const uint32_t addr = base + k * 16 * kRowBytes;
+    return ptx::smem_desc(addr, rows * 128, kAtomBytes, kSwizzle);
+  }
+  static constexpr int bytes(int rows) { return rows * D * 2; }
+};
+
+}  // namespace flare

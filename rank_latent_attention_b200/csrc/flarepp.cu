@@ -1,0 +1,471 @@
+// C ABI of the FLARE++ mixer forward (include/flarepp.h): argument checks,
+// workspace layout, TMA descriptors and kernel dispatch.  Every step of the
+// computation runs in the kernels included below; this file only marshals.
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stdio.h>
+
+#include <algorithm>
+#include <atomic>
+#include <mutex>
+
+#include "../../include/flarepp.h"
+#include "decode_tc.cuh"
+#include "encode_tc.cuh"
+#include "merge.cuh"
+#include "simt_f32.cuh"
+
+namespace flare {
+namespace {
+
+__device__ int g_status[2];  // {first error code, site} per device
+
+std::atomic<int> g_split_override{0};
+std::atomic<int> g_wait_ms{2000};
+thread_local int t_last_launches = 0;
+
+constexpr int kMaxDevices = 64;
+
+int* status_ptr() {
+  static int* ptrs[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    ptrs[dev] = static_cast<int*>(p);
+  }
+  return ptrs[dev];
+}
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess) cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
+int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+
+int check_sizes(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (dtype != FLARE_F32 && dtype != FLARE_BF16) return FLARE_ERR_INVALID_ARG;
+  if (B < 1 || H < 1 || N < 1 || M < 1) return FLARE_ERR_INVALID_ARG;
+  if (static_cast<int64_t>(B) * H > 65535) return FLARE_ERR_UNSUPPORTED;
+  if (N >= (int64_t(1) << 31) - 256) return FLARE_ERR_UNSUPPORTED;
+  if (!(D == 16 || D == 32 || D == 64 || D == 128)) return FLARE_ERR_UNSUPPORTED;
+  if (M > 256) return FLARE_ERR_UNSUPPORTED;
+  if (dtype == FLARE_BF16 && M % 16 != 0) return FLARE_ERR_UNSUPPORTED;
+  return FLARE_OK;
+}
+
+bool device_ptr(const void* p) {
+  if (!p || (reinterpret_cast<uintptr_t>(p) & 15u)) return false;
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+// CTAs per head along the token axis: enough CTAs to fill whole waves of the
+// SMs (one CTA per SM), at most ~256 tiles of 128 tokens per CTA.
+int choose_splits(int BH, int64_t N) {
+  const int64_t tiles = ceil_div(N, kTileN);
+  int64_t s = g_split_override.load();
+  if (s <= 0) {
+    const int sms = sm_count();
+    const int64_t waves = std::max<int64_t>(1, ceil_div(BH * tiles, int64_t(sms) * 256));
+    s = ceil_div(waves * sms, BH);
+  }
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(s, tiles)));
+}
+
+// Partials per head produced by one encode.
+int partials(int M, int splits, int dtype) {
+  if (dtype == FLARE_F32) return splits;
+  return M > kLatRows ? splits : 2 * splits;  // M <= 128: two slots keep separate partials
+}
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+struct EncodeWs {
+  float* O;
+  float* m;
+  float* l;
+  size_t bytes;
+};
+
+EncodeWs encode_ws_layout(char* base, int BH, int64_t N, int M, int D, int dtype) {
+  const int P = partials(M, choose_splits(BH, N), dtype);
+  const size_t rows = static_cast<size_t>(BH) * P * M;
+  EncodeWs w;
+  size_t off = 0;
+  w.O = reinterpret_cast<float*>(base + off);
+  off += align256(rows * D * sizeof(float));
+  w.m = reinterpret_cast<float*>(base + off);
+  off += align256(rows * sizeof(float));
+  w.l = reinterpret_cast<float*>(base + off);
+  off += align256(rows * sizeof(float));
+  w.bytes = off;
+  return w;
+}
+
+size_t elem_size(int dtype) { return dtype == FLARE_BF16 ? 2 : 4; }
+
+// ------------------------------------------------------------------ TMA descriptors
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_tiled() {
+  static EncodeTiledFn fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      return static_cast<EncodeTiledFn>(nullptr);
+    return reinterpret_cast<EncodeTiledFn>(p);
+  }();
+  return fn;
+}
+
+// 3-D bf16 map over [planes][rows][D] with a {min(D,64), box_rows, 1} box and
+// the swizzle that matches the tile geometry the kernels expect.
+bool make_map(CUtensorMap* map, const void* ptr, int D, int64_t rows, int64_t planes, int box_rows) {
+  EncodeTiledFn fn = encode_tiled();
+  if (!fn) return false;
+  const cuuint64_t dims[3] = {static_cast<cuuint64_t>(D), static_cast<cuuint64_t>(rows),
+                              static_cast<cuuint64_t>(planes)};
+  const cuuint64_t strides[2] = {static_cast<cuuint64_t>(D) * 2, static_cast<cuuint64_t>(rows) * D * 2};
+  const cuuint32_t box[3] = {static_cast<cuuint32_t>(D >= 64 ? 64 : D), static_cast<cuuint32_t>(box_rows), 1};
+  const cuuint32_t estr[3] = {1, 1, 1};
+  const CUtensorMapSwizzle sw = D >= 64 ? CU_TENSOR_MAP_SWIZZLE_128B
+                                        : (D == 32 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_32B);
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, sw, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// ------------------------------------------------------------------ launchers
+template <int D, int NHALF, int NS>
+cudaError_t launch_encode_tc_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                               const EncodeArgs& a, int BH, cudaStream_t st) {
+  using C = EncodeCfg<D, NHALF, NS>;
+  auto kern = encode_tc_kernel<D, NHALF, NS>;
+  static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(q, k, v, a);
+  return cudaGetLastError();
+}
+
+template <int NHALF>
+cudaError_t launch_encode_tc_n(int D, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                               const EncodeArgs& a, int BH, cudaStream_t st) {
+  switch (D) {
+    case 16: return launch_encode_tc_t<16, NHALF, 8>(q, k, v, a, BH, st);
+    case 32: return launch_encode_tc_t<32, NHALF, 6>(q, k, v, a, BH, st);
+    case 64: return launch_encode_tc_t<64, NHALF, 4>(q, k, v, a, BH, st);
+    default: return launch_encode_tc_t<128, NHALF, 2>(q, k, v, a, BH, st);
+  }
+}
+
+template <int D, int MP, int NS>
+cudaError_t launch_decode_tc_t(const CUtensorMap& k, const CUtensorMap& q, const CUtensorMap& z,
+                               const DecodeArgs& a, int BH, cudaStream_t st) {
+  using C = DecodeCfg<D, MP, NS>;
+  auto kern = decode_tc_kernel<D, MP, NS>;
+  static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  kern<<<dim3(a.splits, BH), 384, C::kSmemBytes, st>>>(k, q, z, a);
+  return cudaGetLastError();
+}
+
+template <int MP>
+cudaError_t launch_decode_tc_m(int D, const CUtensorMap& k, const CUtensorMap& q, const CUtensorMap& z,
+                               const DecodeArgs& a, int BH, cudaStream_t st) {
+  switch (D) {
+    case 16: return launch_decode_tc_t<16, MP, 8>(k, q, z, a, BH, st);
+    case 32: return launch_decode_tc_t<32, MP, 8>(k, q, z, a, BH, st);
+    case 64: return launch_decode_tc_t<64, MP, 8>(k, q, z, a, BH, st);
+    default: return launch_decode_tc_t<128, MP, 2>(k, q, z, a, BH, st);
+  }
+}
+
+template <int D>
+cudaError_t launch_encode_f32_t(const EncodeF32Args& a, int BH, cudaStream_t st) {
+  constexpr int RPB = 256 / (D / (D < 32 ? D : 32));
+  encode_f32_kernel<D><<<dim3(a.splits, BH, static_cast<unsigned>(ceil_div(a.M, RPB))), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D>
+cudaError_t launch_decode_f32_t(const DecodeF32Args& a, int BH, cudaStream_t st) {
+  decode_f32_kernel<D><<<dim3(static_cast<unsigned>(ceil_div(a.N, 8)), BH), 256, 0, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <typename T>
+cudaError_t launch_merge(const EncodeWs& w, void* out, int BH, int P, int M, int D, cudaStream_t st) {
+  lse_merge_kernel<T><<<dim3(static_cast<unsigned>(ceil_div(int64_t(M) * D, 256)), BH), 256, 0, st>>>(
+      w.O, w.m, w.l, static_cast<T*>(out), P, M, D);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ steps
+// One encode (partials + merge) into `out`; Q indexed per q_batched.
+int run_encode(const void* Q, int q_batched, const void* K, const void* V, void* out, int B, int H, int64_t N,
+               int M, int D, int dtype, char* ws, cudaStream_t st, int* launches) {
+  const int BH = B * H;
+  const int splits = choose_splits(BH, N);
+  const int P = partials(M, splits, dtype);
+  const EncodeWs w = encode_ws_layout(ws, BH, N, M, D, dtype);
+  int* status = status_ptr();
+  if (!status) return FLARE_ERR_CUDA;
+  cudaError_t e;
+  if (dtype == FLARE_BF16) {
+    CUtensorMap tq, tk, tv;
+    if (!make_map(&tq, Q, D, M, q_batched ? BH : H, kLatRows) || !make_map(&tk, K, D, N, BH, kTileN) ||
+        !make_map(&tv, V, D, N, BH, kTileN))
+      return FLARE_ERR_CUDA;
+    EncodeArgs a;
+    a.N = static_cast<int>(N);
+    a.M = M;
+    a.q_batched = q_batched;
+    a.H = H;
+    a.splits = splits;
+    a.tiles = static_cast<int>(ceil_div(N, kTileN));
+    a.P = P;
+    a.O_part = w.O;
+    a.m_part = w.m;
+    a.l_part = w.l;
+    a.status = status;
+    a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+    e = M > kLatRows ? launch_encode_tc_n<2>(D, tq, tk, tv, a, BH, st) : launch_encode_tc_n<1>(D, tq, tk, tv, a, BH, st);
+    if (e != cudaSuccess) return FLARE_ERR_CUDA;
+    e = launch_merge<__nv_bfloat16>(w, out, BH, P, M, D, st);
+  } else {
+    EncodeF32Args a;
+    a.N = static_cast<int>(N);
+    a.M = M;
+    a.q_batched = q_batched;
+    a.H = H;
+    a.splits = splits;
+    a.tiles = static_cast<int>(ceil_div(N, kTileN));
+    a.P = P;
+    a.Q = static_cast<const float*>(Q);
+    a.K = static_cast<const float*>(K);
+    a.V = static_cast<const float*>(V);
+    a.O_part = w.O;
+    a.m_part = w.m;
+    a.l_part = w.l;
+    switch (D) {
+      case 16: e = launch_encode_f32_t<16>(a, BH, st); break;
+      case 32: e = launch_encode_f32_t<32>(a, BH, st); break;
+      case 64: e = launch_encode_f32_t<64>(a, BH, st); break;
+      default: e = launch_encode_f32_t<128>(a, BH, st); break;
+    }
+    if (e != cudaSuccess) return FLARE_ERR_CUDA;
+    e = launch_merge<float>(w, out, BH, P, M, D, st);
+  }
+  *launches += 2;
+  return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
+}
+
+int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N, int M,
+               int D, int dtype, cudaStream_t st, int* launches) {
+  const int BH = B * H;
+  cudaError_t e;
+  if (dtype == FLARE_BF16) {
+    int* status = status_ptr();
+    if (!status) return FLARE_ERR_CUDA;
+    CUtensorMap tk, tq, tz;
+    if (!make_map(&tk, K, D, N, BH, kTileN) || !make_map(&tq, Q, D, M, q_batched ? BH : H, kLatRows) ||
+        !make_map(&tz, Z, D, M, BH, kLatRows))
+      return FLARE_ERR_CUDA;
+    DecodeArgs a;
+    a.N = static_cast<int>(N);
+    a.M = M;
+    a.q_batched = q_batched;
+    a.H = H;
+    a.splits = choose_splits(BH, N);
+    a.tiles = static_cast<int>(ceil_div(N, kTileN));
+    a.Y = static_cast<__nv_bfloat16*>(Y);
+    a.status = status;
+    a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+    e = M > kLatRows ? launch_decode_tc_m<256>(D, tk, tq, tz, a, BH, st)
+                     : launch_decode_tc_m<128>(D, tk, tq, tz, a, BH, st);
+  } else {
+    DecodeF32Args a;
+    a.N = static_cast<int>(N);
+    a.M = M;
+    a.q_batched = q_batched;
+    a.H = H;
+    a.K = static_cast<const float*>(K);
+    a.Q = static_cast<const float*>(Q);
+    a.Z = static_cast<const float*>(Z);
+    a.Y = static_cast<float*>(Y);
+    switch (D) {
+      case 16: e = launch_decode_f32_t<16>(a, BH, st); break;
+      case 32: e = launch_decode_f32_t<32>(a, BH, st); break;
+      case 64: e = launch_decode_f32_t<64>(a, BH, st); break;
+      default: e = launch_decode_f32_t<128>(a, BH, st); break;
+    }
+  }
+  *launches += 1;
+  return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
+}
+
+size_t mix_ws_bytes(int B, int H, int64_t N, int M, int D, int dtype) {
+  const int BH = B * H;
+  const size_t enc = encode_ws_layout(nullptr, BH, N, M, D, dtype).bytes;
+  const size_t lat = align256(static_cast<size_t>(BH) * M * D * elem_size(dtype));
+  return enc + 2 * lat;
+}
+
+// Scratch resolution: caller's buffer, or a stream-ordered allocation.
+struct Scratch {
+  char* ptr = nullptr;
+  bool owned = false;
+};
+
+int get_scratch(void* ws, size_t have, size_t need, cudaStream_t st, Scratch* out) {
+  if (ws) {
+    if (have < need || (reinterpret_cast<uintptr_t>(ws) & 255u)) return FLARE_ERR_INVALID_ARG;
+    out->ptr = static_cast<char*>(ws);
+    return FLARE_OK;
+  }
+  void* p = nullptr;
+  if (cudaMallocAsync(&p, need, st) != cudaSuccess) return FLARE_ERR_CUDA;
+  out->ptr = static_cast<char*>(p);
+  out->owned = true;
+  return FLARE_OK;
+}
+
+int release_scratch(const Scratch& s, cudaStream_t st) {
+  if (s.owned && cudaFreeAsync(s.ptr, st) != cudaSuccess) return FLARE_ERR_CUDA;
+  return FLARE_OK;
+}
+
+int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_out, void* Z_out, int B, int H,
+             int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (!device_ptr(seeds) || !device_ptr(K) || !device_ptr(V) || !device_ptr(Y)) return FLARE_ERR_INVALID_ARG;
+  if ((Qd_out || Z_out) && (!device_ptr(Qd_out) || !device_ptr(Z_out))) return FLARE_ERR_INVALID_ARG;
+  if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  Scratch s;
+  rc = get_scratch(workspace, workspace_bytes, mix_ws_bytes(B, H, N, M, D, dtype), st, &s);
+  if (rc) return rc;
+  const size_t enc = encode_ws_layout(nullptr, BH, N, M, D, dtype).bytes;
+  const size_t lat = align256(static_cast<size_t>(BH) * M * D * elem_size(dtype));
+  void* Qd = Qd_out ? Qd_out : s.ptr + enc;
+  void* Z = Z_out ? Z_out : s.ptr + enc + lat;
+  int launches = 0;
+  rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  if (!rc) rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  if (!rc) rc = run_decode(K, Qd, 1, Z, Y, B, H, N, M, D, dtype, st, &launches);
+  const int rc2 = release_scratch(s, st);
+  if (!rc) {
+    rc = rc2;
+    t_last_launches = launches;
+  }
+  return rc;
+}
+
+}  // namespace
+}  // namespace flare
+
+using namespace flare;
+
+extern "C" {
+
+size_t flare_encode_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (check_sizes(B, H, N, M, D, dtype)) return 0;
+  return encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
+}
+
+size_t flarepp_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (check_sizes(B, H, N, M, D, dtype)) return 0;
+  return mix_ws_bytes(B, H, N, M, D, dtype);
+}
+
+int flare_encode(const void* Q, int q_batched, const void* K, const void* V, void* Z, int B, int H, int64_t N,
+                 int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
+  if (!device_ptr(Q) || !device_ptr(K) || !device_ptr(V) || !device_ptr(Z)) return FLARE_ERR_INVALID_ARG;
+  if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch s;
+  rc = get_scratch(workspace, workspace_bytes, encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes, st, &s);
+  if (rc) return rc;
+  int launches = 0;
+  rc = run_encode(Q, q_batched, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  const int rc2 = release_scratch(s, st);
+  if (!rc) {
+    rc = rc2;
+    t_last_launches = launches;
+  }
+  return rc;
+}
+
+int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N,
+                 int M, int D, int dtype, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
+  if (!device_ptr(K) || !device_ptr(Q) || !device_ptr(Z) || !device_ptr(Y)) return FLARE_ERR_INVALID_ARG;
+  int launches = 0;
+  rc = run_decode(K, Q, q_batched, Z, Y, B, H, N, M, D, dtype, static_cast<cudaStream_t>(stream), &launches);
+  if (!rc) t_last_launches = launches;
+  return rc;
+}
+
+int flarepp_mix(const void* seeds, const void* K, const void* V, void* Y, int B, int H, int64_t N, int M, int D,
+                int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  return mix_impl(seeds, K, V, Y, nullptr, nullptr, B, H, N, M, D, dtype, workspace, workspace_bytes, stream);
+}
+
+int flarepp_mix_debug(const void* seeds, const void* K, const void* V, void* Y, void* Q_dyn, void* Z, int B, int H,
+                      int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  if (!Q_dyn || !Z) return FLARE_ERR_INVALID_ARG;
+  return mix_impl(seeds, K, V, Y, Q_dyn, Z, B, H, N, M, D, dtype, workspace, workspace_bytes, stream);
+}
+
+int flare_check_status(void* stream, int* site) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FLARE_ERR_CUDA;
+  int* p = status_ptr();
+  if (!p) return FLARE_ERR_CUDA;
+  int h[2] = {0, 0};
+  if (cudaMemcpy(h, p, sizeof(h), cudaMemcpyDeviceToHost) != cudaSuccess) return FLARE_ERR_CUDA;
+  const int zero[2] = {0, 0};
+  if (cudaMemcpy(p, zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess) return FLARE_ERR_CUDA;
+  if (site) *site = h[1];
+  return h[0];
+}
+
+const char* flare_status_string(int status) {
+  switch (status) {
+    case FLARE_OK: return "ok";
+    case FLARE_ERR_INVALID_ARG: return "invalid argument";
+    case FLARE_ERR_UNSUPPORTED: return "unsupported sizes";
+    case FLARE_ERR_CUDA: return "CUDA error";
+    case FLARE_ERR_TIMEOUT: return "kernel wait timed out";
+    default: return "unknown status";
+  }
+}
+
+int flare_last_launch_count(void) { return t_last_launches; }
+
+int flare_set_split_override(int splits) { return g_split_override.exchange(splits < 0 ? 0 : splits); }
+
+int flare_set_wait_limit_ms(int ms) { return g_wait_ms.exchange(ms < 1 ? 1 : ms); }
+
+}  // extern "C"
