@@ -1,0 +1,387 @@
+"""Throughput of the FLARE++ mixer forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+One step = one flarepp_mix call (seed encode, routing encode, decode) over
+the million-token workload: B=1, H=16, N=1,048,576, M=256, D=64, bf16, with
+seeded N(0,1)/sqrt(D) inputs (synthetic; they stand in for the pages'
+million-point meshes, no dataset is read).  Inputs of one step (4.3 GB of
+K/V) are far larger than the 126 MB L2, so no flush is needed between steps.
+
+With N GPUs (one process per GPU, torchrun) every rank runs its own
+million-token cloud (batch element b = rank): weak scaling, no collective in
+the data path.  Rank 0 prints one JSON line:
+
+* value / ms_per_step: tokens/s of the whole job, device-timed with CUDA
+  events around K back-to-back steps (max over ranks), inputs resident in HBM;
+* e2e: the same call through the same API with the inputs in pinned host
+  memory, host->device copies and the device->host copy of Y inside the
+  timed region;
+* roofline: the dominant kernel (the tcgen05 encode, launched twice a step),
+  timed per launch with CUDA events bracketing each launch inside a timed
+  region, against the measured peaks in MEASURED_PEAKS.json;
+* cpu_baseline: the fp64 oracle on a bounded sample, on the host cores.
+
+--impl reference times the oracle (the reference arm of this comparison) on
+the host cores, rank 0 only, and prints the same line with "impl": "reference".
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "FLARE++ mixer fwd tokens/s & TFLOP/s (bf16) at N=1M, M=256; % of roofline"
+WORKLOAD = "million"
+CPU_SAMPLE_TOKENS = 1 << 18  # cpu_baseline sample: one head, its first 262144 tokens (~10 s)
+REFERENCE_BUDGET_S = 150.0   # the reference arm's K + W steps together
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--e2e-steps", type=int, default=5)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--heads", type=int, default=None,
+                    help="run only this many heads (smaller case for profiling captures)")
+    return ap.parse_args()
+
+
+def dist_env():
+    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        info = threadpool_info()
+        return max([i.get("num_threads", 1) for i in info] or [1]), (info[0].get("internal_api") if info else "?")
+    except Exception:
+        return os.cpu_count() or 1, "?"
+
+
+# ---------------------------------------------------------------- CPU oracle
+_SAMPLE = {}
+
+
+def oracle_sample_seconds(w, tokens):
+    """Run all three oracle steps on head (0, 0) restricted to its first `tokens` tokens; return seconds."""
+    import numpy as np
+
+    import oracle
+    from rank_latent_attention_b200 import inputs
+
+    if w.name not in _SAMPLE:
+        K, V = inputs.make_head(w, 0, 0)
+        _SAMPLE[w.name] = (inputs.make_seeds(w)[0].astype(np.float64), K.astype(np.float64), V.astype(np.float64))
+    seeds, K, V = _SAMPLE[w.name]
+    t0 = time.perf_counter()
+    oracle.flarepp_head(seeds, K[:tokens], V[:tokens])
+    return time.perf_counter() - t0
+
+
+def cpu_baseline(w):
+    secs = oracle_sample_seconds(w, CPU_SAMPLE_TOKENS)
+    # the oracle's cost is linear in N and in the number of heads at fixed M, D
+    tokens_per_s = CPU_SAMPLE_TOKENS / (secs * w.H)
+    threads, api = blas_threads()
+    return {"value": tokens_per_s, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+            "sample": f"fp64 NumPy oracle ({api} BLAS, {threads} threads), one head with its first "
+                      f"{CPU_SAMPLE_TOKENS} tokens, all three steps, {secs:.2f} s; tokens/s = sample tokens / "
+                      f"(time x {w.H} heads) for the B={w.B}, H={w.H} workload"}
+
+
+def run_reference(args):
+    rank, world, _ = dist_env()
+    if rank != 0:
+        return
+    from rank_latent_attention_b200 import inputs
+
+    w = inputs.WORKLOADS[WORKLOAD]
+    # size each step's sample so that all K + W steps take about REFERENCE_BUDGET_S
+    probe = 8192
+    t = max(oracle_sample_seconds(w, probe), 1e-3)
+    per_step = REFERENCE_BUDGET_S / (args.steps + args.warmup)
+    tokens = probe
+    while tokens < w.N and t * (2 * tokens / probe) <= per_step:
+        tokens *= 2
+    tokens = max(1024, tokens if t * tokens / probe <= per_step else tokens // 2)
+    for _ in range(args.warmup):
+        oracle_sample_seconds(w, tokens)
+    times = [oracle_sample_seconds(w, tokens) for _ in range(args.steps)]
+    step = sum(times) / len(times)
+    value = tokens / (step * w.H)
+    threads, api = blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": step * 1e3 * w.H * (w.N / tokens),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D,
+                   "sample_tokens": tokens},
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": threads, "kind": "oracle",
+                         "sample": f"fp64 NumPy oracle ({api} BLAS), each step one head with its first "
+                                   f"{tokens} tokens, all three steps; tokens/s = sample tokens / (time x "
+                                   f"{w.H} heads); ms_per_step scaled to the full workload"},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ---------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi clock / throttle samples every 200 ms while running."""
+
+    FIELDS = ["index", "clocks.sm", "clocks.max.sm", "power.draw", "clocks_event_reasons.active",
+              "clocks_event_reasons.hw_slowdown", "clocks_event_reasons.hw_thermal_slowdown",
+              "clocks_event_reasons.sw_thermal_slowdown", "clocks_event_reasons.sw_power_cap"]
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.lines = []
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={','.join(self.FIELDS)}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+            self.thread.join(timeout=2)
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = {5: "hw_slowdown", 6: "hw_thermal_slowdown", 7: "sw_thermal_slowdown", 8: "sw_power_cap"}
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for i, name in names.items():
+                if parts[i].lower() in ("active", "1"):
+                    reasons.add(name)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ---------------------------------------------------------------- native arm
+def run_native(args):
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    import rank_latent_attention_b200 as flare
+    from rank_latent_attention_b200 import inputs
+
+    rank, world, local = dist_env()
+    torch.cuda.set_device(local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    flare.lib()
+
+    base = inputs.WORKLOADS[WORKLOAD]
+    H = args.heads or base.H
+    w = inputs.Workload(base.name, world, H, base.N, base.M, base.D, base.dtype, base.kind, base.index)
+    # this rank's cloud: batch element b = rank of the world-sized batch
+    seeds = inputs.make_seeds(w)
+    Kh = np.empty((1, w.H, w.N, w.D), dtype=np.float32)
+    Vh = np.empty_like(Kh)
+    import concurrent.futures as fut
+    with fut.ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
+        for h, (k, v) in enumerate(ex.map(lambda h: inputs.make_head(w, rank, h), range(w.H))):
+            Kh[0, h], Vh[0, h] = k, v
+    s_h = torch.from_numpy(seeds).to(torch.bfloat16).pin_memory()
+    K_h = torch.from_numpy(Kh).to(torch.bfloat16).pin_memory()
+    V_h = torch.from_numpy(Vh).to(torch.bfloat16).pin_memory()
+    del Kh, Vh
+    dev = torch.device("cuda", local)
+    s_d, K_d, V_d = s_h.to(dev), K_h.to(dev), V_h.to(dev)
+    Y_d = torch.empty_like(K_d)
+    ws = torch.empty(flare.flarepp_workspace_size(1, w.H, w.N, w.M, w.D, 1), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        flare.flarepp_mix(s_d, K_d, V_d, Y_d, workspace=ws)
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x):
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after warm-up: {st}")
+    launches_per_step = flare.flare_last_launch_count()
+
+    # ---- main timed region: K steps, inputs resident
+    barrier()
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(local) as clocks:
+        ev0.record(stream)
+        for _ in range(args.steps):
+            step()
+        ev1.record(stream)
+        barrier()
+    ms = max_over_ranks(ev0.elapsed_time(ev1)) / args.steps
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after timing: {st}")
+
+    # ---- per-kernel durations inside a second timed region (events bracket each launch)
+    nprof = min(args.steps, 50)
+    barrier()
+    flare.flare_profile_begin(nprof * launches_per_step)
+    for _ in range(nprof):
+        step()
+    recs = flare.flare_profile_end()
+    barrier()
+    per_kernel = {}
+    for name, t in recs:
+        per_kernel.setdefault(name, []).append(t)
+    step_kernel_ms = {k: sum(v) / nprof for k, v in per_kernel.items()}
+    enc_ms = max_over_ranks(statistics.mean(per_kernel["encode_tc"]))
+    dec_ms = max_over_ranks(statistics.mean(per_kernel["decode_tc"]))
+
+    # ---- end to end: pinned host inputs, copies inside the timed region
+    Y_host = torch.empty(K_h.shape, dtype=torch.bfloat16).pin_memory()
+    ne = max(1, min(args.e2e_steps, args.steps))
+
+    def e2e_step():
+        s_d.copy_(s_h, non_blocking=True)
+        K_d.copy_(K_h, non_blocking=True)
+        V_d.copy_(V_h, non_blocking=True)
+        flare.flarepp_mix(s_d, K_d, V_d, Y_d, workspace=ws)
+        Y_host.copy_(Y_d, non_blocking=True)
+
+    e2e_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(ne):
+        e2e_step()
+    ev1.record(stream)
+    barrier()
+    e2e_ms = max_over_ranks(ev0.elapsed_time(ev1)) / ne
+    h2d = (s_h.numel() + K_h.numel() + V_h.numel()) * 2
+    d2h = Y_host.numel() * 2
+    assert flare.flare_check_status() == (0, 0)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+
+    peaks, peak_kind = measured_peaks()
+    tokens = world * w.N  # B = 1 per rank
+    value = tokens / (ms * 1e-3)
+    flops_step = 12.0 * w.N * w.M * w.D * w.H * world
+    bytes_step = 12.0 * w.N * w.D * w.H * world  # K,V + K,V + K + Y, bf16
+    t_tensor = flops_step / world / (peaks["bf16_tflops"] * 1e12)
+    t_hbm = bytes_step / world / (peaks["hbm_gbs"] * 1e9)
+    # dominant kernel: the encode (two launches per step); algorithmic work per launch
+    enc_flops = 4.0 * w.N * w.M * w.D * w.H
+    enc_bytes = 4.0 * w.N * w.D * w.H
+    enc_t_tensor = enc_flops / (peaks["bf16_tflops"] * 1e12)
+    enc_t_hbm = enc_bytes / (peaks["hbm_gbs"] * 1e9)
+    if enc_t_tensor >= enc_t_hbm:
+        roof = {"bound": "tensor", "achieved": enc_flops / (enc_ms * 1e-3) / 1e12, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s"}
+    else:
+        roof = {"bound": "hbm", "achieved": enc_bytes / (enc_ms * 1e-3) / 1e9, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s"}
+    roof["frac"] = roof["achieved"] / roof["peak"]
+    roof["traffic"] = None
+    roof["kernel"] = "encode_tc"
+    roof["ms_per_launch"] = enc_ms
+    roof["peak_source"] = f"{peak_kind} (burst bf16 GEMM / STREAM copy)"
+    line = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": ms,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD if w.H == base.H else f"{WORKLOAD}-{w.H}heads", "B_per_gpu": 1, "global_batch": world, "H": w.H, "N": w.N, "M": w.M,
+                   "D": w.D, "parallelism": f"batch-sharded x{world}, no collectives",
+                   "l2": "inputs (4.3 GB K/V per step) larger than L2; no flush"},
+        "tflops": flops_step / (ms * 1e-3) / 1e12,
+        "step_roofline": {"t_roofline_ms": max(t_tensor, t_hbm) * 1e3, "bound": "tensor" if t_tensor >= t_hbm else "hbm",
+                          "frac": max(t_tensor, t_hbm) * 1e3 / ms, "peaks": peak_kind},
+        "roofline": roof,
+        "kernel_ms_per_step": step_kernel_ms,
+        "decode_ms_per_launch": dec_ms,
+        "gpu_launches": launches_per_step * args.steps,
+        "clocks": clocks.summary(),
+        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+                "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ne},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w)
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_native(args)
+
+
+if __name__ == "__main__":
+    main()

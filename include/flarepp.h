@@ -27,8 +27,12 @@
  *     Q_dyn, Z               [B][H][M][D]
  * - dtype is FLARE_BF16 (bf16 storage, fp32 accumulation and fp32 softmax on
  *   the tensor cores; intermediates Q_dyn and Z are stored as bf16, rounded to
- *   nearest) or FLARE_F32 (fp32 everywhere, CUDA-core path).  Every tensor of
- *   a call has that dtype.
+ *   nearest, as three chained bf16 SDPA calls would return them) or FLARE_F32
+ *   (fp32 everywhere, CUDA-core path); every tensor of a call has that dtype.
+ *   FLARE_BF16_F32OUT (flarepp_mix / flarepp_mix_debug only) takes bf16 seeds,
+ *   K and V and computes, stores Q_dyn and Z, and writes Y in fp32 on the
+ *   CUDA cores: for inputs whose outputs are so heavy-tailed that bf16
+ *   storage of Y alone exceeds an accuracy budget.
  * - Supported sizes: B >= 1, H >= 1, B*H <= 65535, 1 <= N < 2^31 - 256,
  *   D in {16, 32, 64, 128}, 1 <= M <= 256; for FLARE_BF16 additionally
  *   M % 16 == 0.  N needs no alignment: the last tile of each head is masked.
@@ -56,7 +60,11 @@
 extern "C" {
 #endif
 
-typedef enum { FLARE_F32 = 0, FLARE_BF16 = 1 } flare_dtype_t;
+typedef enum {
+  FLARE_F32 = 0,         /* fp32 storage and arithmetic (CUDA cores)                            */
+  FLARE_BF16 = 1,        /* bf16 storage; tcgen05 bf16 MMAs, fp32 accumulation and softmax      */
+  FLARE_BF16_F32OUT = 2  /* flarepp_mix only: bf16 seeds/K/V; fp32 arithmetic, fp32 Q_dyn, Z, Y */
+} flare_dtype_t;
 
 typedef enum {
   FLARE_OK = 0,
@@ -102,7 +110,7 @@ int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, voi
  * FLARE++ mixer forward: seed encode -> routing encode -> decode (see top).
  *   seeds      [H][M][D]
  *   K, V       [B][H][N][D]
- *   Y          [B][H][N][D] output
+ *   Y          [B][H][N][D] output (fp32 when dtype is FLARE_BF16_F32OUT)
  * K and V are streamed from memory three times in all (K, V; K, V; K) and Y
  * written once; Q_dyn and Z live in the workspace.
  */
@@ -142,6 +150,27 @@ int flare_last_launch_count(void);
  */
 int flare_set_split_override(int splits);
 int flare_set_wait_limit_ms(int ms);
+
+/* Kernel kinds reported by the launch profiler. */
+typedef enum {
+  FLARE_KERNEL_ENCODE_TC = 1,   /* split-token tcgen05 encode (partials) */
+  FLARE_KERNEL_MERGE = 2,       /* log-sum-exp merge of encode partials  */
+  FLARE_KERNEL_DECODE_TC = 3,   /* tcgen05 decode                        */
+  FLARE_KERNEL_ENCODE_F32 = 4,  /* fp32 CUDA-core encode (partials)      */
+  FLARE_KERNEL_DECODE_F32 = 5   /* fp32 CUDA-core decode                 */
+} flare_kernel_kind_t;
+
+/*
+ * Launch profiler.  flare_profile_begin(n) makes the next n kernel launches
+ * (of any call, on any stream) record a CUDA event just before and just after
+ * the launch on the launching stream; nothing else changes and nothing
+ * synchronises.  flare_profile_end synchronises on those events, writes up to
+ * max_records durations (ms) and kernel kinds in launch order, releases the
+ * events and returns the number of records written (negative status on
+ * error).  Used by bench.py to time each kernel inside a timed region.
+ */
+int flare_profile_begin(int max_launches);
+int flare_profile_end(float* ms, int* kinds, int max_records);
 
 #ifdef __cplusplus
 }

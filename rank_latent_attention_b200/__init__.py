@@ -33,6 +33,8 @@ __all__ = [
     "flare_last_launch_count",
     "flare_set_split_override",
     "flare_set_wait_limit_ms",
+    "flare_profile_begin",
+    "flare_profile_end",
     "LIB_PATH",
     "HEADER_PATH",
 ]
@@ -41,7 +43,7 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libflarepp.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "flarepp.h")
 
-F32, BF16 = 0, 1
+F32, BF16, BF16_F32OUT = 0, 1, 2
 _c_int, _c_i64, _c_size, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 _SIZES = [_c_int, _c_int, _c_i64, _c_int, _c_int, _c_int]  # B, H, N, M, D, dtype
 
@@ -57,7 +59,11 @@ _SIGNATURES = {
     "flare_last_launch_count": (_c_int, []),
     "flare_set_split_override": (_c_int, [_c_int]),
     "flare_set_wait_limit_ms": (_c_int, [_c_int]),
+    "flare_profile_begin": (_c_int, [_c_int]),
+    "flare_profile_end": (_c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int), _c_int]),
 }
+
+KERNEL_NAMES = {1: "encode_tc", 2: "lse_merge", 3: "decode_tc", 4: "encode_f32", 5: "decode_f32"}
 
 _lib = None
 
@@ -174,32 +180,47 @@ def flare_decode(K, Q, Z, Y=None, *, stream=None):
     return Y
 
 
-def flarepp_mix(seeds, K, V, Y=None, *, workspace=None, stream=None):
-    """FLARE++ mixer forward: seeds [H,M,D], K/V [B,H,N,D] -> Y [B,H,N,D]."""
+def _mix_mode(K, out_dtype):
+    """(dtype code, output torch dtype): bf16 K with out_dtype=float32 selects the fp32-output mode."""
+    torch = _torch()
+    if out_dtype is None or out_dtype == K.dtype:
+        return _dtype_code(K), K.dtype
+    if K.dtype == torch.bfloat16 and out_dtype == torch.float32:
+        return BF16_F32OUT, torch.float32
+    raise TypeError(f"unsupported input/output dtypes {K.dtype} -> {out_dtype}")
+
+
+def flarepp_mix(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, stream=None):
+    """FLARE++ mixer forward: seeds [H,M,D], K/V [B,H,N,D] -> Y [B,H,N,D].
+
+    out_dtype=torch.float32 with bf16 inputs selects the fp32-arithmetic,
+    fp32-output mode (FLARE_BF16_F32OUT)."""
     torch = _torch()
     B, H, N, D = K.shape
     M = seeds.shape[1]
+    code, odt = _mix_mode(K, out_dtype)
     if Y is None:
-        Y = torch.empty_like(K)
+        Y = torch.empty(K.shape, dtype=odt, device=K.device)
     ws, wsb = _ws(workspace)
     _check(lib().flarepp_mix(_ptr(seeds, "seeds", K.dtype), _ptr(K, "K", K.dtype), _ptr(V, "V", K.dtype),
-                             _ptr(Y, "Y", K.dtype), B, H, N, M, D, _dtype_code(K), ws, wsb, _stream(stream)),
+                             _ptr(Y, "Y", odt), B, H, N, M, D, code, ws, wsb, _stream(stream)),
            "flarepp_mix")
     return Y
 
 
-def flarepp_mix_debug(seeds, K, V, *, workspace=None, stream=None):
+def flarepp_mix_debug(seeds, K, V, *, out_dtype=None, workspace=None, stream=None):
     """As flarepp_mix, also returning the intermediates: (Y, Q_dyn, Z)."""
     torch = _torch()
     B, H, N, D = K.shape
     M = seeds.shape[1]
-    Y = torch.empty_like(K)
-    Qd = torch.empty((B, H, M, D), dtype=K.dtype, device=K.device)
+    code, odt = _mix_mode(K, out_dtype)
+    Y = torch.empty(K.shape, dtype=odt, device=K.device)
+    Qd = torch.empty((B, H, M, D), dtype=odt, device=K.device)
     Z = torch.empty_like(Qd)
     ws, wsb = _ws(workspace)
     _check(lib().flarepp_mix_debug(_ptr(seeds, "seeds", K.dtype), _ptr(K, "K", K.dtype), _ptr(V, "V", K.dtype),
-                                   _ptr(Y, "Y", K.dtype), _ptr(Qd, "Q_dyn", K.dtype), _ptr(Z, "Z", K.dtype),
-                                   B, H, N, M, D, _dtype_code(K), ws, wsb, _stream(stream)),
+                                   _ptr(Y, "Y", odt), _ptr(Qd, "Q_dyn", odt), _ptr(Z, "Z", odt),
+                                   B, H, N, M, D, code, ws, wsb, _stream(stream)),
            "flarepp_mix_debug")
     return Y, Qd, Z
 
@@ -221,3 +242,17 @@ def flare_set_split_override(splits: int) -> int:
 
 def flare_set_wait_limit_ms(ms: int) -> int:
     return lib().flare_set_wait_limit_ms(ms)
+
+
+def flare_profile_begin(max_launches: int) -> None:
+    _check(lib().flare_profile_begin(max_launches), "flare_profile_begin")
+
+
+def flare_profile_end(max_records: int = 1 << 16) -> list[tuple[str, float]]:
+    """[(kernel name, ms)] for the launches recorded since flare_profile_begin."""
+    ms = (ctypes.c_float * max_records)()
+    kinds = (_c_int * max_records)()
+    n = lib().flare_profile_end(ms, kinds, max_records)
+    if n < 0:
+        raise FlareError(-n, "flare_profile_end")
+    return [(KERNEL_NAMES.get(kinds[i], str(kinds[i])), float(ms[i])) for i in range(n)]

@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <vector>
 
 #include "../../include/flarepp.h"
 #include "decode_tc.cuh"
@@ -27,6 +28,34 @@ std::atomic<int> g_wait_ms{2000};
 thread_local int t_last_launches = 0;
 
 constexpr int kMaxDevices = 64;
+
+// ------------------------------------------------------------------ launch profiling
+// When enabled (flare_profile_begin), every kernel launch is bracketed by two
+// CUDA events on the launching stream; flare_profile_end returns the
+// durations.  Events only, no synchronisation until the end.
+struct Profile {
+  std::mutex mu;
+  bool on = false;
+  int cap = 0, used = 0;
+  std::vector<cudaEvent_t> ev;
+  std::vector<int> kind;
+};
+Profile g_prof;
+
+struct ProfScope {
+  int slot = -1;
+  cudaStream_t st;
+  ProfScope(int kind, cudaStream_t s) : st(s) {
+    std::lock_guard<std::mutex> lock(g_prof.mu);
+    if (!g_prof.on || g_prof.used >= g_prof.cap) return;
+    slot = g_prof.used++;
+    g_prof.kind[slot] = kind;
+    cudaEventRecord(g_prof.ev[2 * slot], st);
+  }
+  ~ProfScope() {
+    if (slot >= 0) cudaEventRecord(g_prof.ev[2 * slot + 1], st);
+  }
+};
 
 int* status_ptr() {
   static int* ptrs[kMaxDevices] = {};
@@ -51,7 +80,7 @@ int sm_count() {
 int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 
 int check_sizes(int B, int H, int64_t N, int M, int D, int dtype) {
-  if (dtype != FLARE_F32 && dtype != FLARE_BF16) return FLARE_ERR_INVALID_ARG;
+  if (dtype != FLARE_F32 && dtype != FLARE_BF16 && dtype != FLARE_BF16_F32OUT) return FLARE_ERR_INVALID_ARG;
   if (B < 1 || H < 1 || N < 1 || M < 1) return FLARE_ERR_INVALID_ARG;
   if (static_cast<int64_t>(B) * H > 65535) return FLARE_ERR_UNSUPPORTED;
   if (N >= (int64_t(1) << 31) - 256) return FLARE_ERR_UNSUPPORTED;
@@ -86,7 +115,7 @@ int choose_splits(int BH, int64_t N) {
 
 // Partials per head produced by one encode.
 int partials(int M, int splits, int dtype) {
-  if (dtype == FLARE_F32) return splits;
+  if (dtype != FLARE_BF16) return splits;
   return M > kLatRows ? splits : 2 * splits;  // M <= 128: two slots keep separate partials
 }
 
@@ -114,6 +143,7 @@ EncodeWs encode_ws_layout(char* base, int BH, int64_t N, int M, int D, int dtype
   return w;
 }
 
+// Storage size of Q_dyn / Z (and of Y): bf16 only on the tensor-core path.
 size_t elem_size(int dtype) { return dtype == FLARE_BF16 ? 2 : 4; }
 
 // ------------------------------------------------------------------ TMA descriptors
@@ -195,17 +225,37 @@ cudaError_t launch_decode_tc_m(int D, const CUtensorMap& k, const CUtensorMap& q
   }
 }
 
-template <int D>
+template <int D, typename TQ, typename TKV>
 cudaError_t launch_encode_f32_t(const EncodeF32Args& a, int BH, cudaStream_t st) {
   constexpr int RPB = 256 / (D / (D < 32 ? D : 32));
-  encode_f32_kernel<D><<<dim3(a.splits, BH, static_cast<unsigned>(ceil_div(a.M, RPB))), 256, 0, st>>>(a);
+  encode_f32_kernel<D, TQ, TKV><<<dim3(a.splits, BH, static_cast<unsigned>(ceil_div(a.M, RPB))), 256, 0, st>>>(a);
   return cudaGetLastError();
 }
 
-template <int D>
+template <typename TQ, typename TKV>
+cudaError_t launch_encode_f32_d(int D, const EncodeF32Args& a, int BH, cudaStream_t st) {
+  switch (D) {
+    case 16: return launch_encode_f32_t<16, TQ, TKV>(a, BH, st);
+    case 32: return launch_encode_f32_t<32, TQ, TKV>(a, BH, st);
+    case 64: return launch_encode_f32_t<64, TQ, TKV>(a, BH, st);
+    default: return launch_encode_f32_t<128, TQ, TKV>(a, BH, st);
+  }
+}
+
+template <int D, typename TK>
 cudaError_t launch_decode_f32_t(const DecodeF32Args& a, int BH, cudaStream_t st) {
-  decode_f32_kernel<D><<<dim3(static_cast<unsigned>(ceil_div(a.N, 8)), BH), 256, 0, st>>>(a);
+  decode_f32_kernel<D, TK><<<dim3(static_cast<unsigned>(ceil_div(a.N, 8)), BH), 256, 0, st>>>(a);
   return cudaGetLastError();
+}
+
+template <typename TK>
+cudaError_t launch_decode_f32_d(int D, const DecodeF32Args& a, int BH, cudaStream_t st) {
+  switch (D) {
+    case 16: return launch_decode_f32_t<16, TK>(a, BH, st);
+    case 32: return launch_decode_f32_t<32, TK>(a, BH, st);
+    case 64: return launch_decode_f32_t<64, TK>(a, BH, st);
+    default: return launch_decode_f32_t<128, TK>(a, BH, st);
+  }
 }
 
 template <typename T>
@@ -217,8 +267,10 @@ cudaError_t launch_merge(const EncodeWs& w, void* out, int BH, int P, int M, int
 
 // ------------------------------------------------------------------ steps
 // One encode (partials + merge) into `out`; Q indexed per q_batched.
+// dtype FLARE_BF16: everything bf16, tensor cores.  FLARE_F32: everything
+// fp32.  FLARE_BF16_F32OUT: K, V bf16, out fp32, Q bf16 if q_bf16 else fp32.
 int run_encode(const void* Q, int q_batched, const void* K, const void* V, void* out, int B, int H, int64_t N,
-               int M, int D, int dtype, char* ws, cudaStream_t st, int* launches) {
+               int M, int D, int dtype, char* ws, cudaStream_t st, int* launches, bool q_bf16 = false) {
   const int BH = B * H;
   const int splits = choose_splits(BH, N);
   const int P = partials(M, splits, dtype);
@@ -244,8 +296,13 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     a.l_part = w.l;
     a.status = status;
     a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
-    e = M > kLatRows ? launch_encode_tc_n<2>(D, tq, tk, tv, a, BH, st) : launch_encode_tc_n<1>(D, tq, tk, tv, a, BH, st);
+    {
+      ProfScope prof(FLARE_KERNEL_ENCODE_TC, st);
+      e = M > kLatRows ? launch_encode_tc_n<2>(D, tq, tk, tv, a, BH, st)
+                       : launch_encode_tc_n<1>(D, tq, tk, tv, a, BH, st);
+    }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
+    ProfScope prof(FLARE_KERNEL_MERGE, st);
     e = launch_merge<__nv_bfloat16>(w, out, BH, P, M, D, st);
   } else {
     EncodeF32Args a;
@@ -256,19 +313,23 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     a.splits = splits;
     a.tiles = static_cast<int>(ceil_div(N, kTileN));
     a.P = P;
-    a.Q = static_cast<const float*>(Q);
-    a.K = static_cast<const float*>(K);
-    a.V = static_cast<const float*>(V);
+    a.Q = Q;
+    a.K = K;
+    a.V = V;
     a.O_part = w.O;
     a.m_part = w.m;
     a.l_part = w.l;
-    switch (D) {
-      case 16: e = launch_encode_f32_t<16>(a, BH, st); break;
-      case 32: e = launch_encode_f32_t<32>(a, BH, st); break;
-      case 64: e = launch_encode_f32_t<64>(a, BH, st); break;
-      default: e = launch_encode_f32_t<128>(a, BH, st); break;
+    {
+      ProfScope prof(FLARE_KERNEL_ENCODE_F32, st);
+      if (dtype == FLARE_F32)
+        e = launch_encode_f32_d<float, float>(D, a, BH, st);
+      else if (q_bf16)
+        e = launch_encode_f32_d<__nv_bfloat16, __nv_bfloat16>(D, a, BH, st);
+      else
+        e = launch_encode_f32_d<float, __nv_bfloat16>(D, a, BH, st);
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
+    ProfScope prof(FLARE_KERNEL_MERGE, st);
     e = launch_merge<float>(w, out, BH, P, M, D, st);
   }
   *launches += 2;
@@ -296,6 +357,7 @@ int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void*
     a.Y = static_cast<__nv_bfloat16*>(Y);
     a.status = status;
     a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+    ProfScope prof(FLARE_KERNEL_DECODE_TC, st);
     e = M > kLatRows ? launch_decode_tc_m<256>(D, tk, tq, tz, a, BH, st)
                      : launch_decode_tc_m<128>(D, tk, tq, tz, a, BH, st);
   } else {
@@ -304,16 +366,12 @@ int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void*
     a.M = M;
     a.q_batched = q_batched;
     a.H = H;
-    a.K = static_cast<const float*>(K);
+    a.K = K;
     a.Q = static_cast<const float*>(Q);
     a.Z = static_cast<const float*>(Z);
     a.Y = static_cast<float*>(Y);
-    switch (D) {
-      case 16: e = launch_decode_f32_t<16>(a, BH, st); break;
-      case 32: e = launch_decode_f32_t<32>(a, BH, st); break;
-      case 64: e = launch_decode_f32_t<64>(a, BH, st); break;
-      default: e = launch_decode_f32_t<128>(a, BH, st); break;
-    }
+    ProfScope prof(FLARE_KERNEL_DECODE_F32, st);
+    e = dtype == FLARE_F32 ? launch_decode_f32_d<float>(D, a, BH, st) : launch_decode_f32_d<__nv_bfloat16>(D, a, BH, st);
   }
   *launches += 1;
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
@@ -367,7 +425,7 @@ int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_
   void* Qd = Qd_out ? Qd_out : s.ptr + enc;
   void* Z = Z_out ? Z_out : s.ptr + enc + lat;
   int launches = 0;
-  rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, /*q_bf16=*/true);
   if (!rc) rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches);
   if (!rc) rc = run_decode(K, Qd, 1, Z, Y, B, H, N, M, D, dtype, st, &launches);
   const int rc2 = release_scratch(s, st);
@@ -399,6 +457,7 @@ int flare_encode(const void* Q, int q_batched, const void* K, const void* V, voi
                  int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
   if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
   if (!device_ptr(Q) || !device_ptr(K) || !device_ptr(V) || !device_ptr(Z)) return FLARE_ERR_INVALID_ARG;
   if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
@@ -420,6 +479,7 @@ int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, voi
                  int M, int D, int dtype, void* stream) {
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
   if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
   if (!device_ptr(K) || !device_ptr(Q) || !device_ptr(Z) || !device_ptr(Y)) return FLARE_ERR_INVALID_ARG;
   int launches = 0;
@@ -467,5 +527,42 @@ int flare_last_launch_count(void) { return t_last_launches; }
 int flare_set_split_override(int splits) { return g_split_override.exchange(splits < 0 ? 0 : splits); }
 
 int flare_set_wait_limit_ms(int ms) { return g_wait_ms.exchange(ms < 1 ? 1 : ms); }
+
+int flare_profile_begin(int max_launches) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (g_prof.on || max_launches < 1) return FLARE_ERR_INVALID_ARG;
+  g_prof.ev.assign(2 * static_cast<size_t>(max_launches), nullptr);
+  for (auto& e : g_prof.ev)
+    if (cudaEventCreate(&e) != cudaSuccess) {
+      for (auto& x : g_prof.ev)
+        if (x) cudaEventDestroy(x);
+      g_prof.ev.clear();
+      return FLARE_ERR_CUDA;
+    }
+  g_prof.kind.assign(max_launches, 0);
+  g_prof.cap = max_launches;
+  g_prof.used = 0;
+  g_prof.on = true;
+  return FLARE_OK;
+}
+
+int flare_profile_end(float* ms, int* kinds, int max_records) {
+  std::lock_guard<std::mutex> lock(g_prof.mu);
+  if (!g_prof.on) return -FLARE_ERR_INVALID_ARG;
+  int n = std::min(g_prof.used, max_records);
+  int rc = n;
+  for (int i = 0; i < g_prof.used; ++i) {
+    if (cudaEventSynchronize(g_prof.ev[2 * i + 1]) != cudaSuccess) rc = -FLARE_ERR_CUDA;
+    if (i < n && rc >= 0) {
+      if (cudaEventElapsedTime(&ms[i], g_prof.ev[2 * i], g_prof.ev[2 * i + 1]) != cudaSuccess) rc = -FLARE_ERR_CUDA;
+      kinds[i] = g_prof.kind[i];
+    }
+  }
+  for (auto& e : g_prof.ev) cudaEventDestroy(e);
+  g_prof.ev.clear();
+  g_prof.on = false;
+  g_prof.used = g_prof.cap = 0;
+  return rc;
+}
 
 }  // extern "C"

@@ -7,6 +7,9 @@
 // throughout so that results stay within 1e-4 of the fp64 definition.
 //   encode_f32_kernel: split-token partials in the same (O, mref, l) format as
 //                      encode_tc_kernel, merged by lse_merge_kernel.
+// Inputs may be stored as bf16 (TQ / TKV / TK = __nv_bfloat16): they are
+// widened on load and everything after that is fp32, which is the
+// bf16-in / fp32-out mode of the library.
 //   decode_f32_kernel: one warp per token; lanes split the latents, the row
 //                      max and sum go through warp shuffles, then lanes split
 //                      the D output channels.
@@ -16,11 +19,22 @@
 
 namespace flare {
 
+template <typename T>
+__device__ __forceinline__ float ld_f32(const T* p);
+template <>
+__device__ __forceinline__ float ld_f32<float>(const float* p) {
+  return *p;
+}
+template <>
+__device__ __forceinline__ float ld_f32<__nv_bfloat16>(const __nv_bfloat16* p) {
+  return __bfloat162float(*p);
+}
+
 struct EncodeF32Args {
   int N, M, q_batched, H, splits, tiles, P;
-  const float* Q;  // [H or BH][M][D]
-  const float* K;  // [BH][N][D]
-  const float* V;
+  const void* Q;  // [H or BH][M][D], TQ
+  const void* K;  // [BH][N][D], TKV
+  const void* V;
   float* O_part;
   float* m_part;
   float* l_part;
@@ -29,7 +43,7 @@ struct EncodeF32Args {
 constexpr int kF32Tile = 32;  // tokens per smem tile
 
 // grid (splits, BH, row groups); 256 threads; D/min(D,32) threads per latent row.
-template <int D>
+template <int D, typename TQ, typename TKV>
 __global__ void __launch_bounds__(256) encode_f32_kernel(const EncodeF32Args a) {
   constexpr int DPT = D < 32 ? D : 32;  // channels per thread
   constexpr int TPR = D / DPT;          // threads per latent row
@@ -46,15 +60,16 @@ __global__ void __launch_bounds__(256) encode_f32_kernel(const EncodeF32Args a) 
   const long long tok1 = static_cast<long long>(split + 1) * a.N / a.splits;
 
   float q[DPT], o[DPT];
-  const float* qrow = a.Q + ((static_cast<size_t>(a.q_batched ? bh : bh % a.H) * a.M) + (active ? row : 0)) * D;
+  const TQ* qrow = static_cast<const TQ*>(a.Q) +
+                   ((static_cast<size_t>(a.q_batched ? bh : bh % a.H) * a.M) + (active ? row : 0)) * D;
 #pragma unroll
   for (int d = 0; d < DPT; ++d) {
-    q[d] = active ? qrow[d0 + d] : 0.f;
+    q[d] = active ? ld_f32(qrow + d0 + d) : 0.f;
     o[d] = 0.f;
   }
   float mref = -INFINITY, l = 0.f;
-  const float* Kh = a.K + static_cast<size_t>(bh) * a.N * D;
-  const float* Vh = a.V + static_cast<size_t>(bh) * a.N * D;
+  const TKV* Kh = static_cast<const TKV*>(a.K) + static_cast<size_t>(bh) * a.N * D;
+  const TKV* Vh = static_cast<const TKV*>(a.V) + static_cast<size_t>(bh) * a.N * D;
 
   for (long long t0 = tok0; t0 < tok1; t0 += kF32Tile) {
     const long long rem = tok1 - t0;
@@ -62,8 +77,8 @@ __global__ void __launch_bounds__(256) encode_f32_kernel(const EncodeF32Args a) 
     __syncthreads();
     for (int i = threadIdx.x; i < kF32Tile * D; i += blockDim.x) {
       const int j = i / D, d = i % D;
-      sK[j][d] = j < cnt ? Kh[(t0 + j) * D + d] : 0.f;
-      sV[j][d] = j < cnt ? Vh[(t0 + j) * D + d] : 0.f;
+      sK[j][d] = j < cnt ? ld_f32(Kh + (t0 + j) * D + d) : 0.f;
+      sV[j][d] = j < cnt ? ld_f32(Vh + (t0 + j) * D + d) : 0.f;
     }
     __syncthreads();
     for (int j = 0; j < cnt; ++j) {
@@ -99,14 +114,14 @@ __global__ void __launch_bounds__(256) encode_f32_kernel(const EncodeF32Args a) 
 
 struct DecodeF32Args {
   int N, M, q_batched, H;
-  const float* K;  // [BH][N][D]
+  const void* K;   // [BH][N][D], TK
   const float* Q;  // [H or BH][M][D]
   const float* Z;  // [BH][M][D]
   float* Y;        // [BH][N][D]
 };
 
 // grid (ceil(N / 8), BH); 256 threads = 8 warps, one token per warp.
-template <int D>
+template <int D, typename TK>
 __global__ void __launch_bounds__(256) decode_f32_kernel(const DecodeF32Args a) {
   __shared__ float sk[8][D];
   __shared__ float sp[8][256];
@@ -114,8 +129,8 @@ __global__ void __launch_bounds__(256) decode_f32_kernel(const DecodeF32Args a) 
   const int bh = blockIdx.y;
   const long long tok = static_cast<long long>(blockIdx.x) * 8 + warp;
   if (tok >= a.N) return;  // whole warp leaves together
-  const float* k = a.K + (static_cast<size_t>(bh) * a.N + tok) * D;
-  for (int d = lane; d < D; d += 32) sk[warp][d] = k[d];
+  const TK* k = static_cast<const TK*>(a.K) + (static_cast<size_t>(bh) * a.N + tok) * D;
+  for (int d = lane; d < D; d += 32) sk[warp][d] = ld_f32(k + d);
   __syncwarp();
   const float* Q = a.Q + static_cast<size_t>(a.q_batched ? bh : bh % a.H) * a.M * D;
   const float* Z = a.Z + static_cast<size_t>(bh) * a.M * D;
