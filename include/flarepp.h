@@ -172,6 +172,36 @@ typedef enum {
 int flare_profile_begin(int max_launches);
 int flare_profile_end(float* ms, int* kinds, int max_records);
 
+/*
+ * flare_encode_noalloc: the FLARE encode of flare_encode (same arguments,
+ * same kernels, same results) for callers that are not allowed to allocate
+ * device memory.  Some code cannot call cudaMalloc or ask its caller for a
+ * workspace: a library layer whose host framework already owns every byte of
+ * the GPU through its own pool, a latency-critical loop where an allocation
+ * (which may synchronise the device or fail under memory pressure) is not
+ * acceptable, or a plug-in whose interface passes only inputs and outputs.
+ * The pages have no counterpart to this entry point; it exists for such
+ * callers only.
+ *
+ * The split-token softmax partials live in one scratch array of
+ * FLARE_NOALLOC_SCRATCH_BYTES bytes that is part of the library itself, so
+ * every GPU the library is loaded on holds that much memory until the
+ * process exits.  The first call on each device looks up that array's
+ * device address (with that device current), so make the first call on a
+ * device before starting any stream capture.  Calls whose partials need more
+ * than FLARE_NOALLOC_SCRATCH_BYTES (see flare_encode_workspace_size) return
+ * FLARE_ERR_UNSUPPORTED before enqueuing anything; use flare_encode with a
+ * workspace for those.  Nothing in the array has to start at zero: each call
+ * writes every partial it later reads.  All calls share the one array, so
+ * two calls whose kernels can overlap on the GPU (different streams without
+ * ordering, or several host threads) race on it; order them on one stream.
+ * dtype FLARE_F32 or FLARE_BF16.  No cudaMalloc, cudaFree or other
+ * allocating call is made.
+ */
+#define FLARE_NOALLOC_SCRATCH_BYTES (16u << 20)
+int flare_encode_noalloc(const void* Q, int q_batched, const void* K, const void* V, void* Z, int B, int H,
+                         int64_t N, int M, int D, int dtype, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -566,3 +566,50 @@ int flare_profile_end(float* ms, int* kinds, int max_records) {
 }
 
 }  // extern "C"
+
+// ------------------------------------------------------------------ no-allocation encode
+// Scratch for flare_encode_noalloc: a fixed array in the library's own device
+// image, so the entry point never allocates.  Host code must not use the
+// symbol itself as a pointer (it is a host-side stand-in); the device address
+// is looked up once per device below.
+static __device__ __align__(256) unsigned char g_noalloc_scratch[FLARE_NOALLOC_SCRATCH_BYTES];
+
+namespace flare {
+namespace {
+
+char* noalloc_scratch() {
+  static char* ptrs[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  if (!ptrs[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess) {
+      cudaGetLastError();
+      return nullptr;
+    }
+    ptrs[dev] = static_cast<char*>(p);
+  }
+  return ptrs[dev];
+}
+
+}  // namespace
+}  // namespace flare
+
+extern "C" int flare_encode_noalloc(const void* Q, int q_batched, const void* K, const void* V, void* Z, int B,
+                                    int H, int64_t N, int M, int D, int dtype, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
+  if (!device_ptr(Q) || !device_ptr(K) || !device_ptr(V) || !device_ptr(Z)) return FLARE_ERR_INVALID_ARG;
+  if (encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes > FLARE_NOALLOC_SCRATCH_BYTES)
+    return FLARE_ERR_UNSUPPORTED;
+  char* ws = noalloc_scratch();
+  if (!ws) return FLARE_ERR_CUDA;
+  int launches = 0;
+  rc = run_encode(Q, q_batched, K, V, Z, B, H, N, M, D, dtype, ws, static_cast<cudaStream_t>(stream), &launches);
+  if (!rc) t_last_launches = launches;
+  return rc;
+}
