@@ -62,6 +62,16 @@ struct TileGeom {
     return ptx::smem_desc(addr, rows * 128, kAtomBytes, kSwizzle);
   }
   static constexpr int bytes(int rows) { return rows * D * 2; }
+
+  // The same descriptors as base + offset: only the start-address field
+  // (bits [0,14), 16-byte units) moves between K steps and ring stages, so
+  // the MMA issuer adds a constant instead of rebuilding 64-bit descriptors.
+  __host__ __device__ static constexpr uint32_t kmajor_step(int rows, int k) {
+    return static_cast<uint32_t>(((k * 16) / 64) * rows * 128 + ((k * 16) % 64) * 2) >> 4;
+  }
+  __host__ __device__ static constexpr uint32_t mnmajor_step(int k) {
+    return static_cast<uint32_t>(k * 16 * kRowBytes) >> 4;
+  }
 };
 
 }  // namespace flare

@@ -10,9 +10,12 @@
 // Work of one CTA: one (b, h), Q and Z of that head resident in shared
 // memory, and a contiguous run of 128-token tiles.
 //   warp 0      TMA producer: Q and Z once, then K tiles into an NS-deep ring
-//   warp 1      TMEM allocator + single-thread tcgen05.mma issuer
+//   warp 1      TMEM allocator + tcgen05.mma issuer of slot 0 (one thread)
+//   warp 2      tcgen05.mma issuer of slot 1 (one thread)
 //   warps 4-7   epilogue warpgroup of slot 0 (even tiles), one thread per token
 //   warps 8-11  epilogue warpgroup of slot 1 (odd tiles)
+// The slots own disjoint TMEM columns and each has its own issuer, so one
+// slot's waits never hold up the other slot's MMAs.
 // Per tile: S = K_tile Q^T (128 x MP, fp32, TMEM), the owning thread takes
 // the max over its row's M valid latents, writes P = 2^(s log2e - max) as bf16
 // over the first MP/2 columns, then O = P Z (128 x D) lands in columns
@@ -101,7 +104,7 @@ __global__ void __launch_bounds__(384, 1)
       ptx::mbar_init(&O_full[s], 1);
       ptx::mbar_init(&O_free[s], 4);
     }
-    ptx::mbar_init(drain, 1);
+    ptx::mbar_init(drain, 2);  // one commit per issuer
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
@@ -148,44 +151,59 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
         ptx::mbar_wait_drain(&full[t % NS], (t / NS) & 1);
     }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
+  } else if (warp == 1 || warp == 2) {
+    // ------------------------------------------------------------ MMA issuers (one per slot)
     if (lane == 0) {
+      static_assert((NS & (NS - 1)) == 0, "ring depth must be a power of two");
+      const int slot = warp - 1;
       bool ok = ptx::mbar_wait(qz_full, 0, s_abort, args.wait_ns);
       ptx::tc_fence_after();
-      const uint32_t sQ = sbase + C::kOffQ;
-      const uint32_t sZ = sbase + C::kOffZ;
-      auto issue_qk = [&](int t) -> bool {
-        const int st = t % NS;
-        const int s = t & 1;
-        if (!ptx::mbar_wait(&full[st], (t / NS) & 1, s_abort, args.wait_ns)) return false;
-        ptx::tc_fence_after();
-        const uint32_t kb = sbase + C::kOffStages + st * C::kTileBytes;
+      // descriptors of stage 0 / K step 0; stages and K steps only move the start address
+      const uint64_t dK0 = G::kmajor(sbase + C::kOffStages, kTileN, 0);
+      const uint64_t dQ0 = G::kmajor(sbase + C::kOffQ, MP, 0);
+      const uint64_t dZ0 = G::mnmajor(sbase + C::kOffZ, MP, 0);
+      const uint32_t tS = tmem + slot * C::kSlotCols;
+      // The issuing thread stalls on any shared-memory access until its own
+      // MMAs have completed: waits go before each group of MMAs.
+      auto wait_stage = [&](int t) -> bool {
+        return ptx::mbar_wait(&full[t & (NS - 1)], (t / NS) & 1, s_abort, args.wait_ns);
+      };
+      auto issue_qk = [&](int t) {
+        const int st = t & (NS - 1);
+        const uint64_t dK = dK0 + static_cast<uint32_t>(st * (C::kTileBytes >> 4));
 #pragma unroll
         for (int k = 0; k < D / 16; ++k)
-          ptx::mma_ss(tmem + s * C::kSlotCols, G::kmajor(kb, kTileN, k), G::kmajor(sQ, MP, k), C::kIdescQK,
-                      k > 0 ? 1u : 0u);
-        ptx::mma_commit(&S_full[s]);
+          ptx::mma_ss(tS, dK + G::kmajor_step(kTileN, k), dQ0 + G::kmajor_step(MP, k), C::kIdescQK, k > 0 ? 1u : 0u);
+        ptx::mma_commit(&S_full[slot]);
         ptx::mma_commit(&empty[st]);
-        return true;
       };
-      auto issue_pv = [&](int t) -> bool {
-        const int s = t & 1;
-        if (!ptx::mbar_wait(&P_full[s], (t >> 1) & 1, s_abort, args.wait_ns)) return false;
-        ptx::tc_fence_after();
-        const uint32_t slot = tmem + s * C::kSlotCols;
+      auto issue_pv = [&]() {
 #pragma unroll
         for (int k = 0; k < MP / 16; ++k)
-          ptx::mma_ts(slot + C::kColO, slot + k * 8, G::mnmajor(sZ, MP, k), C::kIdescPV, k > 0 ? 1u : 0u);
-        ptx::mma_commit(&O_full[s]);
-        return true;
+          ptx::mma_ts(tS + C::kColO, tS + k * 8, dZ0 + G::mnmajor_step(k), C::kIdescPV, k > 0 ? 1u : 0u);
+        ptx::mma_commit(&O_full[slot]);
       };
-      if (ok) ok = issue_qk(0) && (T < 2 || issue_qk(1));
-      for (int t = 0; ok && t < T; ++t) {
-        ok = issue_pv(t);
-        if (ok && t + 2 < T) {
+      // this slot's tiles: t = slot + 2 i
+      if (ok && slot < T) {
+        ok = wait_stage(slot);
+        if (ok) {
+          ptx::tc_fence_after();
+          issue_qk(slot);
+        }
+      }
+      for (int i = 0; ok && slot + 2 * i < T; ++i) {
+        const int t = slot + 2 * i;
+        ok = (t + 2 >= T || wait_stage(t + 2)) && ptx::mbar_wait(&P_full[slot], i & 1, s_abort, args.wait_ns);
+        if (!ok) break;
+        ptx::tc_fence_after();
+        issue_pv();
+        if (t + 2 < T) {
           // the slot's columns are reused once its epilogue has read O of tile t
-          ok = ptx::mbar_wait(&O_free[t & 1], (t >> 1) & 1, s_abort, args.wait_ns) && issue_qk(t + 2);
+          ok = ptx::mbar_wait(&O_free[slot], i & 1, s_abort, args.wait_ns);
+          if (ok) {
+            ptx::tc_fence_after();
+            issue_qk(t + 2);
+          }
         }
       }
       if (!ok) {
@@ -212,8 +230,11 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       ptx::tc_fence_after();
-      // pass 1: row max over the M valid latents (columns >= M are padding)
-      float mx = -INFINITY;
+      // pass 1: row max over the M valid latents (columns >= M are padding;
+      // M is a multiple of 16, so validity is uniform per 16-column group)
+      float pm[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pm[j] = -INFINITY;
 #pragma unroll
       for (int c0 = 0; c0 < MP; c0 += 128) {
         float x[128];
@@ -221,13 +242,17 @@ __global__ void __launch_bounds__(384, 1)
         for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + c0 + 32 * c, x + 32 * c);
         ptx::tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 128; ++c)
-          if (c0 + c < M) mx = fmaxf(mx, x[c]);
+        for (int g = 0; g < 8; ++g)
+          if (c0 + 16 * g < M) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pm[j] = ptx::max3(pm[j], x[16 * g + 2 * j], x[16 * g + 2 * j + 1]);
+          }
       }
-      const float mref = mx * kLog2e;
+      const float mref =
+          ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) * kLog2e;
       // pass 2: P = 2^(s log2e - mref) as bf16 pairs over the first MP/2 columns
       // (P of columns [c0, c0+64) lands in [c0/2, c0/2+32), already read)
-      float l = 0.f;
+      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
 #pragma unroll
       for (int c0 = 0; c0 < MP; c0 += 64) {
         float x[64];
@@ -236,14 +261,23 @@ __global__ void __launch_bounds__(384, 1)
         ptx::tmem_wait_ld();
         uint32_t p[32];
 #pragma unroll
-        for (int c = 0; c < 64; c += 2) {
-          const float p0 = (c0 + c < M) ? ptx::ex2(fmaf(x[c], kLog2e, -mref)) : 0.f;
-          const float p1 = (c0 + c + 1 < M) ? ptx::ex2(fmaf(x[c + 1], kLog2e, -mref)) : 0.f;
-          l += p0 + p1;
-          p[c / 2] = ptx::pack_bf16(p0, p1);
+        for (int g = 0; g < 4; ++g) {
+          if (c0 + 16 * g < M) {
+#pragma unroll
+            for (int c = 16 * g; c < 16 * g + 16; c += 2) {
+              const float p0 = ptx::ex2(fmaf(x[c], kLog2e, -mref));
+              const float p1 = ptx::ex2(fmaf(x[c + 1], kLog2e, -mref));
+              ps[(c / 2) & 7] += p0 + p1;
+              p[c / 2] = ptx::pack_bf16(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int c = 16 * g; c < 16 * g + 16; c += 2) p[c / 2] = 0u;
+          }
         }
         ptx::tmem_st32(tS + c0 / 2, p);
       }
+      const float l = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
       ptx::tmem_wait_st();
       ptx::tc_fence_before();
       __syncwarp();

@@ -101,22 +101,24 @@ bool device_ptr(const void* p) {
 }
 
 // CTAs per head along the token axis: enough CTAs to fill whole waves of the
-// SMs (one CTA per SM), at most ~256 tiles of 128 tokens per CTA.
-int choose_splits(int BH, int64_t N) {
-  const int64_t tiles = ceil_div(N, kTileN);
+// SMs (one CTA per SM), at most ~32768 tokens per CTA; `tile` is the kernel's
+// token tile (64 for the encode, 128 for the decode).
+int choose_splits(int BH, int64_t N, int tile) {
+  const int64_t tiles = ceil_div(N, tile);
   int64_t s = g_split_override.load();
   if (s <= 0) {
     const int sms = sm_count();
-    const int64_t waves = std::max<int64_t>(1, ceil_div(BH * tiles, int64_t(sms) * 256));
+    const int64_t waves = std::max<int64_t>(1, ceil_div(BH * tiles, int64_t(sms) * (32768 / tile)));
     s = ceil_div(waves * sms, BH);
   }
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(s, tiles)));
 }
 
-// Partials per head produced by one encode.
-int partials(int M, int splits, int dtype) {
+// Partials per head produced by one encode: one per split on the CUDA-core
+// path; on the tensor-core path one per (split, slot, buffer) accumulator.
+int partials(int M, int D, int splits, int dtype) {
   if (dtype != FLARE_BF16) return splits;
-  return M > kLatRows ? splits : 2 * splits;  // M <= 128: two slots keep separate partials
+  return splits * encode_partials_per_split(D, M > kLatRows ? 2 : 1);
 }
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -129,7 +131,7 @@ struct EncodeWs {
 };
 
 EncodeWs encode_ws_layout(char* base, int BH, int64_t N, int M, int D, int dtype) {
-  const int P = partials(M, choose_splits(BH, N), dtype);
+  const int P = partials(M, D, choose_splits(BH, N, kEncTile), dtype);
   const size_t rows = static_cast<size_t>(BH) * P * M;
   EncodeWs w;
   size_t off = 0;
@@ -196,10 +198,10 @@ template <int NHALF>
 cudaError_t launch_encode_tc_n(int D, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                                const EncodeArgs& a, int BH, cudaStream_t st) {
   switch (D) {
-    case 16: return launch_encode_tc_t<16, NHALF, 8>(q, k, v, a, BH, st);
-    case 32: return launch_encode_tc_t<32, NHALF, 6>(q, k, v, a, BH, st);
-    case 64: return launch_encode_tc_t<64, NHALF, 4>(q, k, v, a, BH, st);
-    default: return launch_encode_tc_t<128, NHALF, 2>(q, k, v, a, BH, st);
+    case 16: return launch_encode_tc_t<16, NHALF, 16>(q, k, v, a, BH, st);
+    case 32: return launch_encode_tc_t<32, NHALF, 8>(q, k, v, a, BH, st);
+    case 64: return launch_encode_tc_t<64, NHALF, 8>(q, k, v, a, BH, st);
+    default: return launch_encode_tc_t<128, NHALF, 4>(q, k, v, a, BH, st);
   }
 }
 
@@ -272,16 +274,16 @@ cudaError_t launch_merge(const EncodeWs& w, void* out, int BH, int P, int M, int
 int run_encode(const void* Q, int q_batched, const void* K, const void* V, void* out, int B, int H, int64_t N,
                int M, int D, int dtype, char* ws, cudaStream_t st, int* launches, bool q_bf16 = false) {
   const int BH = B * H;
-  const int splits = choose_splits(BH, N);
-  const int P = partials(M, splits, dtype);
+  const int splits = choose_splits(BH, N, kEncTile);
+  const int P = partials(M, D, splits, dtype);
   const EncodeWs w = encode_ws_layout(ws, BH, N, M, D, dtype);
   int* status = status_ptr();
   if (!status) return FLARE_ERR_CUDA;
   cudaError_t e;
   if (dtype == FLARE_BF16) {
     CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, Q, D, M, q_batched ? BH : H, kLatRows) || !make_map(&tk, K, D, N, BH, kTileN) ||
-        !make_map(&tv, V, D, N, BH, kTileN))
+    if (!make_map(&tq, Q, D, M, q_batched ? BH : H, kLatRows) || !make_map(&tk, K, D, N, BH, kEncTile) ||
+        !make_map(&tv, V, D, N, BH, kEncTile))
       return FLARE_ERR_CUDA;
     EncodeArgs a;
     a.N = static_cast<int>(N);
@@ -289,7 +291,7 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     a.q_batched = q_batched;
     a.H = H;
     a.splits = splits;
-    a.tiles = static_cast<int>(ceil_div(N, kTileN));
+    a.tiles = static_cast<int>(ceil_div(N, kEncTile));
     a.P = P;
     a.O_part = w.O;
     a.m_part = w.m;
@@ -352,7 +354,7 @@ int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void*
     a.M = M;
     a.q_batched = q_batched;
     a.H = H;
-    a.splits = choose_splits(BH, N);
+    a.splits = choose_splits(BH, N, kTileN);
     a.tiles = static_cast<int>(ceil_div(N, kTileN));
     a.Y = static_cast<__nv_bfloat16*>(Y);
     a.status = status;
