@@ -31,6 +31,28 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr int kTileN = 128;   // tokens per tile (MMA M of the decode, N of the encode)
 constexpr int kLatRows = 128; // latent rows per tcgen05 MMA (M = 128, cta_group::1)
 
+// 2^x on the FMA/ALU pipes, for the share of a softmax tile's exponentials
+// that would otherwise queue behind the MUFU unit (16 results per clock per
+// SM on sm_100, the binding resource of the softmax).  For -126 <= x <= 64 the
+// relative error is below 7.5e-5 (P is then rounded to bf16, 2^-9); x < -126
+// gives 2^-126 in place of a value below the smallest normal.
+//   x = j + f with j = rint(x), f in [-1/2, 1/2]: adding 1.5 * 2^23 leaves j
+//   in the low mantissa bits of the sum, and subtracting it back gives j
+//   exactly; 2^f is the degree-3 polynomial of minimax relative error on
+//   [-1/2, 1/2] (Remez exchange, coefficients printed by exp2_poly_fit.py);
+//   2^j scales it by adding j to the exponent field (the sum's bits shifted
+//   left by 23 are j << 23, the constant's bits shift out).
+__device__ __forceinline__ float exp2_poly3(float x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  const float xc = fmaxf(x, -126.f);
+  const float r = __fadd_rn(xc, kRound);
+  const float f = __fadd_rn(xc, -__fadd_rn(r, -kRound));
+  float p = fmaf(0.0551716685f, f, 0.242611125f);
+  p = fmaf(p, f, 0.693260968f);
+  p = fmaf(p, f, 0.999928057f);
+  return __uint_as_float(__float_as_uint(p) + (__float_as_uint(r) << 23));
+}
+
 // Record the first failure in the device status word {code, site}.
 __device__ __forceinline__ void record_error(int* status, int code, int site) {
   if (atomicCAS(status, 0, code) == 0) atomicExch(status + 1, site);

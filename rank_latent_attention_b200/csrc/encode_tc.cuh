@@ -8,40 +8,53 @@
 // Engine" review page, section "Основной механизм FLARE", encode step; the
 // split-and-merge of softmax statistics is the exact reduction the FLARE++
 // page ("Contributions Clés", context parallelism) exchanges between devices,
-// applied here between CTAs of one GPU (and between the accumulators of one
-// CTA).  lse_merge (merge.cuh) combines the partials into the normalised
-// M x D result.
+// applied here between CTAs of one GPU.  lse_merge (merge.cuh) combines the
+// partials into the normalised M x D result.
 //
 // Work of one CTA: one (b, h) and a contiguous run of 64-token tiles.
-//   warp 0            TMA producer: Q once, then K/V tiles into an NS-deep ring
-//   warps 1-3, 12     tcgen05.mma issuers, one thread each (warp 1 also
-//                     allocates TMEM)
-//   warps 4-7         softmax warpgroup of slot 0 (one thread per latent row)
-//   warps 8-11        softmax warpgroup of slot 1
+//   warps 0-15   four softmax warpgroups (slot s, column half c): thread r of
+//                group (s, c) owns latent row r of slot s and columns
+//                [32 c, 32 c + 32) of every tile of the slot
+//   warp 16      TMA producer: K/V tiles into an NS-deep ring (and Q when it
+//                stays in shared memory); also allocates TMEM
+//   warps 17-18  tcgen05.mma issuers, one warp per slot
 // With M > 128 the two slots are the two 128-row halves of the latents and
 // both see every tile; with M <= 128 both slots use the same latents and take
 // alternate tiles.
 //
-// Each slot has NB buffers (2 for D <= 64, 1 for D = 128) taken round robin by
-// its tiles, and each (slot, buffer) pair owns an S region, an O accumulator,
-// its own online-softmax state and its own issuer thread.  An issuer waits for
-// P of its buffer, issues P.V into its O and Q.K^T of the buffer's next tile,
-// and commits.  Why one issuer per buffer: a thread that has MMAs in flight
-// stalls on any synchronising instruction until they complete, so a thread
-// serving several buffers would couple their latencies; with one per buffer
-// the path P(t) -> P.V(t) -> Q.K^T(t + NB) -> S ready has the other buffer's
-// tile of softmax time to complete in.  S of a buffer's tile being ready also
-// means the buffer's previous P.V is done (one thread, in order), which is
-// all the rare O rescale needs.
+// Per slot, S is double-buffered in TMEM: while the two groups turn S(i) into
+// P(i), the MMAs of tile i + 1 are already done, and the issuer, once P(i) is
+// stored, issues P(i).V and Q.K^T of tile i + 2 into the freed buffer.  A
+// thread with MMAs in flight stalls on its next synchronising instruction
+// until they complete, which is why the issuers are warps of their own: their
+// next wait (P of the following tile) is a whole softmax phase away.  An
+// issuer warp runs its loop as a whole and issues under elect.sync, which
+// keeps the MMA operands warp-uniform (issue from one divergent thread runs
+// well below the tensor pipe's rate).  Slot 1 starts half a phase late so
+// the two slots' softmax phases interleave.
 //
-// TMEM columns: S of (slot s, buffer b) at [64 (NB s + b), +64) fp32; P (bf16
-// pairs) overwrites the first 32 columns of its S after the scores are read;
-// O of (s, b) at [128 NB + D (NB s + b), +D).  Q stays in shared memory.
+// D <= 64: each group has its own O accumulator and reference max, so the
+// groups never exchange data within a tile; the K steps of P.V over tokens
+// [32 c, +32) go to accumulator (s, c), and the epilogue folds the two
+// accumulators of a slot like any two partials.  D = 128 (TMEM too small for
+// four accumulators): the two groups of a slot share O and agree on each
+// row's reference through shared memory (a named barrier per tile).
+//
+// TMEM columns: S of (slot s, buffer j) at [64 (2 s + j), +64) fp32; group c
+// writes its P (bf16 pairs) over [32 c, +16) of it, inside its own scores.
+// O at [256 + D a, +D) for accumulator a = 2 s + c (D <= 64) or a = s
+// (D = 128); Q after the accumulators as bf16 pairs when it fits (Q.K^T then
+// reads it as the TMEM A operand), else in shared memory.
 //
 // Online softmax with a lazy reference: a row's reference max only moves when
 // a tile's max exceeds it by more than 2^8, so the O rescale in tensor memory
 // is rare.  Any reference gives the same normalised result because P and l
-// use the same one.
+// use the same one.  Of every 16 column pairs, those in kEncPolyPairs take
+// their exponentials from exp2_poly3 (FMA pipe) instead of MUFU.
+//
+// Epilogue: each CTA writes one partial per head (O_part[split] etc.), the
+// accumulators that cover the same latent rows folded with their weights
+// 2^(mref_a - max_a mref_a).
 #pragma once
 
 #include "common.cuh"
@@ -51,6 +64,7 @@ namespace flare {
 constexpr int kEncTile = 64;  // tokens per encode tile
 
 struct EncodeArgs {
+  const void* Q;  // bf16 [BH or H][M][D]: read into TMEM directly when D <= 64
   int N;          // tokens per head
   int M;          // latents
   int q_batched;  // Q indexed by bh (1) or by h = bh % H (0)
@@ -65,60 +79,110 @@ struct EncodeArgs {
   unsigned long long wait_ns;
 };
 
-// Buffers (and accumulators) per slot of the encode for head dim D.
-__host__ __device__ constexpr int encode_buffers(int D) { return D <= 64 ? 2 : 1; }
-
 // Partials per (head, split) written by encode_tc_kernel.
-__host__ __device__ constexpr int encode_partials_per_split(int D, int nhalf) {
-  return encode_buffers(D) * (nhalf == 2 ? 1 : 2);
-}
+__host__ __device__ constexpr int encode_partials_per_split(int /*D*/, int /*nhalf*/) { return 1; }
+
+// Column pairs (bit j: pair j of each 16) whose exponentials go to
+// exp2_poly3: pairs 0, 4, 7, 10, 13, i.e. 5/16 of the tile.
+constexpr uint32_t kEncPolyPairs = 0x2491u;
 
 template <int D, int NHALF, int NS>
 struct EncodeCfg {
   using G = TileGeom<D>;
-  static constexpr int NB = encode_buffers(D);
-  static constexpr int kThreads = 416;
-  static constexpr int kQHalfBytes = G::bytes(kLatRows);
+  // D <= 64: each column-half group accumulates its own O with its own
+  // reference (no exchange of row maxima); D = 128: the two groups of a slot
+  // share one O and agree on the reference through shared memory.
+  static constexpr bool kSplitO = D <= 64;
+  static constexpr int kAccPerSlot = kSplitO ? 2 : 1;
+  static constexpr int kProducerWarp = 16;
+  static constexpr int kIssuerWarp = 17;  // + slot
+  static constexpr int kThreads = 32 * 19;
+  static constexpr uint32_t kColO = 4 * kEncTile;
+  static constexpr uint32_t kColQ = kColO + 2 * kAccPerSlot * D;
+  // Q in TMEM (TS Q.K^T) when it fits beside S and O, else in shared memory (SS)
+  static constexpr bool kQTmem = kColQ + D <= 512;
+  static constexpr int kQHalfBytes = kQTmem ? 0 : G::bytes(kLatRows);
   static constexpr int kTileBytes = G::bytes(kEncTile);
   static constexpr int kStageBytes = 2 * kTileBytes;
   static constexpr int kOffQ = 0;
   static constexpr int kOffStages = NHALF * kQHalfBytes;
   static constexpr int kOffBars = kOffStages + NS * kStageBytes;
-  // full[NS], empty[NS], q_ready, S_full[2 NB], P_full[2 NB], O_final[2 NB], drain
-  static constexpr int kNumBars = 2 * NS + 2 + 6 * NB;
-  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
+  // full[NS], empty[NS], q_ready, S_full[4], P_full[4], pv_done[2], O_final[2], drain
+  static constexpr int kNumBars = 2 * NS + 14;
+  static constexpr int kOffXM = kOffBars + 8 * kNumBars;            // float [2 parity][2 slot][2 half][128]
+  static constexpr int kOffML = kOffXM + 2 * 2 * 2 * kLatRows * 4;  // float2 [2 slot][2 half][128]
+  static constexpr int kOffMisc = kOffML + 2 * 2 * kLatRows * 8;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;  // + slack for 1024-B alignment
   static constexpr uint32_t kTmemCols = 512;
-  static constexpr uint32_t kColO = 2 * NB * kEncTile;
-  static_assert(kColO + 2 * NB * D <= 512, "TMEM budget");
+  static_assert(kColQ <= 512, "TMEM budget");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static_assert((NS & (NS - 1)) == 0, "ring depth must be a power of two");
-  // An issuer at tile t waits for its buffer's next tile, NB (M > 128) or 2 NB
-  // (M <= 128) tiles ahead, whose stage is free once tile t - 1 is released.
-  static_assert(NS >= (NHALF == 2 ? NB : 2 * NB) + 1, "ring too shallow for the look-ahead");
+  // An issuer at local tile i waits for the stage of local tile i + 2 (tile
+  // + 2 or + 4), free once the tile before i is released.
+  static_assert(NS >= (NHALF == 2 ? 2 : 4) + 1, "ring too shallow for the look-ahead");
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16(kLatRows, kEncTile, 0, 0);
   static constexpr uint32_t kIdescPV = ptx::idesc_bf16(kLatRows, D, 0, 1);
-  __host__ __device__ static constexpr uint32_t col_s(int slot, int buf) { return (NB * slot + buf) * kEncTile; }
-  __host__ __device__ static constexpr uint32_t col_o(int slot, int buf) { return kColO + (NB * slot + buf) * D; }
+  __host__ __device__ static constexpr uint32_t col_s(int s, int j) { return (2 * s + j) * kEncTile; }
+  // accumulator of (slot s, column half c): shared by both halves unless kSplitO
+  __host__ __device__ static constexpr uint32_t col_o(int s, int c) {
+    return kColO + (kSplitO ? 2 * s + c : s) * D;
+  }
+  __host__ __device__ static constexpr uint32_t col_q(int s) { return kColQ + (NHALF == 2 ? s : 0) * (D / 2); }
 };
 
+// P = 2^(x log2e - nref) for the 32 scores of one half-row, packed to bf16
+// pairs and stored into 16 TMEM columns at tP; returns the fp32 sum.
+// RAGGED (a tile past the end of the tokens, masked columns at -inf): every
+// exponential on MUFU, and masked columns give exactly 0.
+template <bool RAGGED>
+__device__ __forceinline__ float encode_exp_store(const float* x, float nref, uint32_t tP) {
+  float ps[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+#pragma unroll
+  for (int c0 = 0; c0 < 32; c0 += 16) {
+    uint32_t p[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int c = c0 + 2 * u;
+      const float a0 = fmaf(x[c], kLog2e, -nref);
+      const float a1 = fmaf(x[c + 1], kLog2e, -nref);
+      float p0, p1;
+      if (!RAGGED && ((kEncPolyPairs >> ((c / 2) & 15)) & 1u)) {
+        p0 = exp2_poly3(a0);
+        p1 = exp2_poly3(a1);
+      } else {
+        p0 = ptx::ex2(a0);
+        p1 = ptx::ex2(a1);
+        if (RAGGED) {  // a half-row may be fully masked with no reference yet (-inf - -inf)
+          p0 = x[c] == -INFINITY ? 0.f : p0;
+          p1 = x[c + 1] == -INFINITY ? 0.f : p1;
+        }
+      }
+      ps[u & 3] += p0 + p1;
+      p[u] = ptx::pack_bf16(p0, p1);
+    }
+    ptx::tmem_st8(tP + c0 / 2, p);
+  }
+  return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+}
+
 template <int D, int NHALF, int NS>
-__global__ void __launch_bounds__(416, 1)
+__global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                      const __grid_constant__ CUtensorMap tmV, const EncodeArgs args) {
   using C = EncodeCfg<D, NHALF, NS>;
   using G = typename C::G;
-  constexpr int NB = C::NB;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* full = bars;
   uint64_t* empty = bars + NS;
   uint64_t* q_ready = bars + 2 * NS;
-  uint64_t* S_full = bars + 2 * NS + 1;            // [NB slot + buf]
-  uint64_t* P_full = bars + 2 * NS + 1 + 2 * NB;   // [NB slot + buf]
-  uint64_t* O_final = bars + 2 * NS + 1 + 4 * NB;  // [NB slot + buf]
-  uint64_t* drain = bars + 2 * NS + 1 + 6 * NB;
+  uint64_t* S_full = bars + 2 * NS + 1;    // [2 slot + buffer]
+  uint64_t* P_full = bars + 2 * NS + 5;    // [2 slot + buffer]
+  uint64_t* pv_done = bars + 2 * NS + 9;   // [slot]
+  uint64_t* O_final = bars + 2 * NS + 11;  // [slot]
+  uint64_t* drain = bars + 2 * NS + 13;
+  float* s_xm = reinterpret_cast<float*>(smem + C::kOffXM);
+  float2* s_ml = reinterpret_cast<float2*>(smem + C::kOffML);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -126,6 +190,7 @@ __global__ void __launch_bounds__(416, 1)
   const int lane = threadIdx.x & 31;
   const int split = blockIdx.x;
   const int bh = blockIdx.y;
+  const int qidx = args.q_batched ? bh : bh % args.H;
   const int tile0 = static_cast<int>((static_cast<long long>(split) * args.tiles) / args.splits);
   const int tile1 = static_cast<int>((static_cast<long long>(split + 1) * args.tiles) / args.splits);
   const int T = tile1 - tile0;
@@ -138,17 +203,21 @@ __global__ void __launch_bounds__(416, 1)
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], NHALF == 2 ? 2 : 1);  // both slots read every stage when M > 128
     }
-    ptx::mbar_init(q_ready, 1);
-    for (int i = 0; i < 2 * NB; ++i) {
+    // Q in TMEM: one arrival per softmax warp that stores a part of it
+    ptx::mbar_init(q_ready, C::kQTmem ? 4 * (NHALF == 2 ? 2 : 1) * (D >= 32 ? 2 : 1) : 1);
+    for (int i = 0; i < 4; ++i) {
       ptx::mbar_init(&S_full[i], 1);
-      ptx::mbar_init(&P_full[i], 4);  // one arrival per softmax warp of the slot
+      ptx::mbar_init(&P_full[i], 8);  // one arrival per warp of the slot's two groups
+    }
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&pv_done[i], 1);
       ptx::mbar_init(&O_final[i], 1);
     }
-    ptx::mbar_init(drain, 2 * NB);  // one commit per issuer
+    ptx::mbar_init(drain, 64);  // one commit per lane of the two issuer warps
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == C::kProducerWarp) {
     ptx::tmem_alloc(s_tmem, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -157,25 +226,24 @@ __global__ void __launch_bounds__(416, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = ptx::smem_u32(smem);
-  // issuer index of this warp (-1: not an issuer)
-  const int issuer = warp == 1 ? 0 : warp == 2 ? 1 : warp == 3 ? 2 : warp == 12 ? 3 : -1;
 
-  if (warp == 0) {
+  if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
-      const int qidx = args.q_batched ? bh : bh % args.H;
       ptx::prefetch_tmap(&tmK);
       ptx::prefetch_tmap(&tmV);
-      ptx::prefetch_tmap(&tmQ);
-      ptx::mbar_arrive_expect_tx(q_ready, NHALF * C::kQHalfBytes);
-      for (int h = 0; h < NHALF; ++h)
-        for (int b = 0; b < G::kBlocks; ++b)
-          ptx::tma_load_3d(smem + C::kOffQ + h * C::kQHalfBytes + b * kLatRows * 128, &tmQ, q_ready, b * 64,
-                           h * kLatRows, qidx);
+      if constexpr (!C::kQTmem) {
+        ptx::prefetch_tmap(&tmQ);
+        ptx::mbar_arrive_expect_tx(q_ready, NHALF * C::kQHalfBytes);
+        for (int h = 0; h < NHALF; ++h)
+          for (int b = 0; b < G::kBlocks; ++b)
+            ptx::tma_load_3d(smem + C::kOffQ + h * C::kQHalfBytes + b * kLatRows * 128, &tmQ, q_ready, b * 64,
+                             h * kLatRows, qidx);
+      }
       const uint64_t pol = ptx::policy_evict_first();
       int issued = 0;
       for (int t = 0; t < T; ++t) {
-        const int st = t & (NS - 1);
+        const int st = t % NS;
         if (t >= NS && !ptx::mbar_wait(&empty[st], ((t / NS) - 1) & 1, s_abort, args.wait_ns)) {
           record_error(args.status, kErrTimeout, kSiteEncProducer);
           *s_abort = 1;
@@ -192,204 +260,284 @@ __global__ void __launch_bounds__(416, 1)
         issued = t + 1;
       }
       // Every load issued must land before the CTA may exit (matters on the abort path only).
-      ptx::mbar_wait_drain(q_ready, 0);
+      if constexpr (!C::kQTmem) ptx::mbar_wait_drain(q_ready, 0);
       for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
-        ptx::mbar_wait_drain(&full[t & (NS - 1)], (t / NS) & 1);
+        ptx::mbar_wait_drain(&full[t % NS], (t / NS) & 1);
     }
-  } else if (issuer >= 0) {
+  } else if (warp >= C::kIssuerWarp) {
     // ------------------------------------------------------------ MMA issuers
-    if (lane == 0 && issuer < 2 * NB) {
-      const int s = issuer / NB;  // slot
-      const int b = issuer % NB;  // buffer
-      const int count = count_of(s);
-      const int half = NHALF == 2 ? s : 0;
-      bool ok = true;
-      if (b < count) {
-        // Descriptors of stage 0 / K step 0; a stage adds kStageBytes >> 4 to
-        // the start-address field, a K step adds a compile-time constant.
-        const uint64_t dK0 = G::kmajor(sbase + C::kOffStages, kEncTile, 0);
-        const uint64_t dV0 = G::mnmajor(sbase + C::kOffStages + C::kTileBytes, kEncTile, 0);
-        const uint64_t dQ = G::kmajor(sbase + C::kOffQ + half * C::kQHalfBytes, kLatRows, 0);
-        const uint32_t tS = tmem + C::col_s(s, b);
-        const uint32_t tO = tmem + C::col_o(s, b);
-        auto wait_stage = [&](int t) -> bool {
-          return ptx::mbar_wait(&full[t & (NS - 1)], (t / NS) & 1, s_abort, args.wait_ns);
-        };
-        auto issue_qk = [&](int t) {
-          const uint64_t dK = dK0 + static_cast<uint32_t>((t & (NS - 1)) * (C::kStageBytes >> 4));
+    // The whole warp runs the loop (waits are warp-wide); one elected lane
+    // issues each batch of MMAs and the commits that track them.
+    const int s = warp - C::kIssuerWarp;
+    const int count = count_of(s);
+    const uint64_t dK0 = G::kmajor(sbase + C::kOffStages, kEncTile, 0);
+    const uint64_t dV0 = G::mnmajor(sbase + C::kOffStages + C::kTileBytes, kEncTile, 0);
+    const uint64_t dQ = G::kmajor(sbase + C::kOffQ + (NHALF == 2 ? s : 0) * C::kQHalfBytes, kLatRows, 0);
+    const uint32_t tQ = tmem + C::col_q(s);
+    auto wait_stage = [&](int t) -> bool {
+      return ptx::mbar_wait(&full[t % NS], (t / NS) & 1, s_abort, args.wait_ns);
+    };
+    auto issue_qk = [&](int i) {
+      const int t = tile_of(s, i);
+      const uint32_t tS = tmem + C::col_s(s, i & 1);
+      const uint64_t dK = dK0 + static_cast<uint32_t>((t % NS) * (C::kStageBytes >> 4));
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k)
-            ptx::mma_ss(tS, dQ + G::kmajor_step(kLatRows, k), dK + G::kmajor_step(kEncTile, k), C::kIdescQK,
-                        k > 0 ? 1u : 0u);
-          ptx::mma_commit(&S_full[issuer]);
-        };
-        ok = ptx::mbar_wait(q_ready, 0, s_abort, args.wait_ns) && wait_stage(tile_of(s, b));
-        if (ok) {
-          ptx::tc_fence_after();
-          issue_qk(tile_of(s, b));
-        }
-        // this buffer's tiles: local i = b + NB k
-        for (int i = b, k = 0; ok && i < count; i += NB, ++k) {
-          const int t = tile_of(s, i);
-          const int tn = i + NB < count ? tile_of(s, i + NB) : -1;
-          // every wait before the MMAs: a wait after them would stall until they complete
-          ok = (tn < 0 || wait_stage(tn)) && ptx::mbar_wait(&P_full[issuer], k & 1, s_abort, args.wait_ns);
-          if (!ok) break;
-          ptx::tc_fence_after();
-          const uint64_t dV = dV0 + static_cast<uint32_t>((t & (NS - 1)) * (C::kStageBytes >> 4));
-#pragma unroll
-          for (int kk = 0; kk < kEncTile / 16; ++kk)
-            ptx::mma_ts(tO, tS + kk * 8, dV + G::mnmajor_step(kk), C::kIdescPV, (k > 0 || kk > 0) ? 1u : 0u);
-          ptx::mma_commit(&empty[t & (NS - 1)]);
-          if (tn >= 0)
-            issue_qk(tn);  // reuses S of tile t: after its P.V in issue order
-          else
-            ptx::mma_commit(&O_final[issuer]);
-        }
+      for (int k = 0; k < D / 16; ++k) {
+        if constexpr (C::kQTmem)
+          ptx::mma_ts(tS, tQ + k * 8, dK + G::kmajor_step(kEncTile, k), C::kIdescQK, k > 0 ? 1u : 0u);
+        else
+          ptx::mma_ss(tS, dQ + G::kmajor_step(kLatRows, k), dK + G::kmajor_step(kEncTile, k), C::kIdescQK,
+                      k > 0 ? 1u : 0u);
       }
-      if (!ok) {
-        record_error(args.status, kErrTimeout, kSiteEncMma);
-        *s_abort = 1;
+      ptx::mma_commit(&S_full[2 * s + (i & 1)]);
+    };
+    bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(q_ready, 0, s_abort, args.wait_ns));
+    // Slot 1 starts once slot 0's first P is stored, so that the two slots'
+    // softmax phases interleave instead of running in step.
+    if (s == 1 && count_of(0) > 0)
+      ok = ok && __all_sync(0xffffffffu, ptx::mbar_wait(&P_full[0], 0, s_abort, args.wait_ns));
+    for (int i = 0; ok && i < 2 && i < count; ++i) {
+      ok = __all_sync(0xffffffffu, wait_stage(tile_of(s, i)));
+      if (ok) {
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) issue_qk(i);
+        __syncwarp();
       }
-      // Drain: wait for every MMA issued by the issuers before TMEM is released.
-      ptx::mma_commit(drain);
-      ptx::mbar_wait_drain(drain, 0);
     }
-  } else if (warp >= 4 && warp < 12) {
-    // ------------------------------------------------------------ softmax warpgroups
-    const int s = (warp - 4) >> 2;         // slot
+    for (int i = 0; ok && i < count; ++i) {
+      const int t = tile_of(s, i);
+      // every wait before the MMAs: a wait after them would stall until they complete
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&P_full[2 * s + (i & 1)], (i >> 1) & 1, s_abort, args.wait_ns) &&
+                                       (i + 2 >= count || wait_stage(tile_of(s, i + 2))));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+        const uint32_t tP = tmem + C::col_s(s, i & 1);
+        const uint64_t dV = dV0 + static_cast<uint32_t>((t % NS) * (C::kStageBytes >> 4));
+        // K steps 0-1 carry the tokens of column half 0, steps 2-3 those of half 1
+#pragma unroll
+        for (int kk = 0; kk < kEncTile / 16; ++kk) {
+          const int cu = kk / 2;
+          const bool acc = i > 0 || (C::kSplitO ? (kk & 1) : kk) > 0;
+          ptx::mma_ts(tmem + C::col_o(s, cu), tP + cu * 32 + (kk & 1) * 8, dV + G::mnmajor_step(kk), C::kIdescPV,
+                      acc ? 1u : 0u);
+        }
+        ptx::mma_commit(&empty[t % NS]);
+        ptx::mma_commit(&pv_done[s]);
+        if (i + 2 < count) issue_qk(i + 2);  // into the buffer P(i) came from: after its P.V in issue order
+        if (i + 1 == count) ptx::mma_commit(&O_final[s]);
+      }
+      __syncwarp();
+    }
+    if (!ok && lane == 0) {
+      record_error(args.status, kErrTimeout, kSiteEncMma);
+      *s_abort = 1;
+    }
+    // Drain: every lane commits (a lane that issued nothing arrives at once),
+    // so every MMA issued completes before TMEM is released.
+    ptx::mma_commit(drain);
+    ptx::mbar_wait_drain(drain, 0);
+  } else {
+    // ------------------------------------------------------------ softmax groups
+    const int g = warp >> 2;               // group
+    const int s = g >> 1;                  // slot
+    const int c = g & 1;                   // column half
     const int r = (warp & 3) * 32 + lane;  // TMEM lane = latent row within the half
     const int m = (NHALF == 2 ? s : 0) * kLatRows + r;
     const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
     const int count = count_of(s);
 
-    float mref[NB], l[NB];  // per-buffer reference max (log2 domain) and running sum
+    if constexpr (C::kQTmem) {
+      // Q row m into TMEM as bf16 pairs; group c stores its half of the columns.
+      constexpr int kQCols = D / 2;  // 32-bit columns per row
+      constexpr int kPart = kQCols >= 16 ? kQCols / 2 : kQCols;
+      if ((NHALF == 2 || s == 0) && (kQCols >= 16 || c == 0)) {
+        uint32_t qv[kPart];
+        const int col0 = kQCols >= 16 ? c * kPart : 0;
+        if (m < args.M) {
+          const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(args.Q) +
+                                                            (static_cast<size_t>(qidx) * args.M + m) * D) +
+                             col0 / 4;
 #pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      mref[b] = -INFINITY;
-      l[b] = 0.f;
+          for (int z = 0; z < kPart / 4; ++z) {
+            const uint4 v = src[z];
+            qv[4 * z] = v.x;
+            qv[4 * z + 1] = v.y;
+            qv[4 * z + 2] = v.z;
+            qv[4 * z + 3] = v.w;
+          }
+        } else {
+#pragma unroll
+          for (int z = 0; z < kPart; ++z) qv[z] = 0u;
+        }
+        const uint32_t ta = tmem + lane_off + C::col_q(s) + col0;
+        if constexpr (kPart == 16) ptx::tmem_st16(ta, qv); else ptx::tmem_st8(ta, qv);
+        ptx::tmem_wait_st();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(q_ready);
+      }
     }
+
+    float mref = -INFINITY, l = 0.f;  // reference max (log2 domain), running sum of this half-row
     bool ok = true;
-    for (int i0 = 0; ok && i0 < count; i0 += NB) {
+    const int bar_id = 1 + s;  // named barrier of the slot's two groups (shared O only)
+    constexpr int kOCols = C::kSplitO ? D : D / 2;  // O columns this group rescales
+    const uint32_t tOwn = tmem + lane_off + C::col_o(s, c) + (C::kSplitO ? 0 : c * (D / 2));
+    for (int i = 0; i < count; ++i) {
+      const int t = tile_of(s, i);
+      const int j = i & 1;
+      const uint32_t tS = tmem + lane_off + C::col_s(s, j);
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&S_full[2 * s + j], (i >> 1) & 1, s_abort, args.wait_ns))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      float x[32];
+      ptx::tmem_ld32(tS + 32 * c, x);
+      ptx::tmem_wait_ld();
+      const int valid = args.N - (tile0 + t) * kEncTile - 32 * c;
+      if (valid < 32) {
 #pragma unroll
-      for (int b = 0; b < NB; ++b) {
-        const int i = i0 + b;
-        if (i >= count) break;
-        const int k = i0 / NB;  // index of the tile among the buffer's tiles
-        const int t = tile_of(s, i);
-        const int q = NB * s + b;
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&S_full[q], k & 1, s_abort, args.wait_ns))) {
+        for (int z = 0; z < 32; ++z)
+          if (z >= valid) x[z] = -INFINITY;
+      }
+      // half-row max as 8 independent 3-input chains
+      float pm[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pm[u] = fmaxf(x[2 * u], x[2 * u + 1]);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) pm[u] = ptx::max3(pm[u], x[16 + 2 * u], x[17 + 2 * u]);
+      float mx = ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+      if constexpr (!C::kSplitO) {
+        // shared O: agree on the row max with the other group of the slot
+        // (buffers alternate by tile parity, so a fast group cannot overwrite
+        // a value not yet read); after the barrier both groups have read
+        // their scores and P may overwrite S
+        float* xm = s_xm + ((j * 2 + s) * 2) * kLatRows;
+        xm[c * kLatRows + r] = mx;
+        asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");
+        mx = fmaxf(mx, xm[(c ^ 1) * kLatRows + r]);
+      }
+      mx *= kLog2e;
+      const bool need = mx > mref + 8.f;
+      const float nref = need ? mx : mref;
+      // 0 on the first tile; 1 while a fully masked half-row has no reference
+      const float alpha = nref == mref ? 1.f : ptx::ex2(mref - nref);
+      mref = nref;
+      // P overwrites the first 16 of this group's own 32 score columns
+      const float lt = valid < 32 ? encode_exp_store<true>(x, nref, tS + 32 * c)
+                                  : encode_exp_store<false>(x, nref, tS + 32 * c);
+      l = fmaf(l, alpha, lt);
+      // Rare: the reference moved, so rescale this group's part of O, once the
+      // previous P.V (issued after P(i - 1)) has completed; the next one waits
+      // for P_full.
+      if (i > 0 && __any_sync(0xffffffffu, need)) {
+        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&pv_done[s], (i - 1) & 1, s_abort, args.wait_ns))) {
           ok = false;
           break;
         }
         ptx::tc_fence_after();
-        const uint32_t tS = tmem + lane_off + C::col_s(s, b);
-        float x[kEncTile];
-        ptx::tmem_ld32(tS, x);
-        ptx::tmem_ld32(tS + 32, x + 32);
-        ptx::tmem_wait_ld();
-        const int valid = args.N - (tile0 + t) * kEncTile;
-        if (valid < kEncTile) {
+        constexpr int kChunk = kOCols < 32 ? kOCols : 32;
 #pragma unroll
-          for (int c = 0; c < kEncTile; ++c)
-            if (c >= valid) x[c] = -INFINITY;
-        }
-        // row max as 8 independent 3-input chains
-        float pm[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) pm[u] = fmaxf(x[2 * u], x[2 * u + 1]);
-#pragma unroll
-        for (int c = 16; c < kEncTile; c += 16)
-#pragma unroll
-          for (int u = 0; u < 8; ++u) pm[u] = ptx::max3(pm[u], x[c + 2 * u], x[c + 2 * u + 1]);
-        const float mx =
-            ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) * kLog2e;
-        const bool need = mx > mref[b] + 8.f;
-        const float nref = need ? mx : mref[b];
-        const float alpha = ptx::ex2(mref[b] - nref);  // 0 on the buffer's first tile
-        l[b] *= alpha;
-        mref[b] = nref;
-        {
-          uint32_t p[kEncTile / 2];
-          float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};  // independent partial sums
-#pragma unroll
-          for (int c = 0; c < kEncTile; c += 2) {
-            const float p0 = ptx::ex2(fmaf(x[c], kLog2e, -nref));
-            const float p1 = ptx::ex2(fmaf(x[c + 1], kLog2e, -nref));
-            ps[(c / 2) & 7] += p0 + p1;
-            p[c / 2] = ptx::pack_bf16(p0, p1);
-          }
-          ptx::tmem_st32(tS, p);
-          l[b] += ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-        }
-        // Rare: the reference moved, so rescale this row of the buffer's O.
-        // No MMA writes it now: its previous P.V completed before this S was
-        // signalled (same issuer, in order) and its next one waits for P_full.
-        if (k > 0 && __any_sync(0xffffffffu, need)) {
-          const uint32_t tO = tmem + lane_off + C::col_o(s, b);
-          constexpr int kChunk = D < 32 ? D : 32;
-#pragma unroll
-          for (int c = 0; c < D / kChunk; ++c) {
-            float o[kChunk];
-            if constexpr (kChunk == 32) ptx::tmem_ld32(tO + c * 32, o); else ptx::tmem_ld16(tO, o);
-            ptx::tmem_wait_ld();
-            uint32_t u[kChunk];
-#pragma unroll
-            for (int z = 0; z < kChunk; ++z) u[z] = __float_as_uint(o[z] * alpha);
-            if constexpr (kChunk == 32) ptx::tmem_st32(tO + c * 32, u); else ptx::tmem_st16(tO, u);
-          }
-        }
-        ptx::tmem_wait_st();
-        ptx::tc_fence_before();
-        __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&P_full[q]);
-      }
-    }
-
-    // Epilogue: one partial per (slot, buffer); O streamed out of TMEM in chunks.
-#pragma unroll
-    for (int b = 0; b < NB; ++b) {
-      const bool has = b < count;
-      if (ok && has) {
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&O_final[NB * s + b], 0, s_abort, args.wait_ns));
-        if (ok) ptx::tc_fence_after();
-      }
-      if (!ok) break;
-      const int p = NHALF == 2 ? split * NB + b : (split * 2 + s) * NB + b;
-      const size_t row = (static_cast<size_t>(bh) * args.P + p) * args.M + m;
-      float4* dst = reinterpret_cast<float4*>(args.O_part + row * D);
-      const uint32_t tO = tmem + lane_off + C::col_o(s, b);
-      constexpr int kChunk = D < 32 ? D : 32;
-#pragma unroll
-      for (int c = 0; c < D / kChunk; ++c) {
-        float o[kChunk];
-        if (has) {
-          if constexpr (kChunk == 32) ptx::tmem_ld32(tO + c * 32, o); else ptx::tmem_ld16(tO, o);
+        for (int z0 = 0; z0 < kOCols; z0 += kChunk) {
+          float o[kChunk];
+          const uint32_t ta = tOwn + z0;
+          if constexpr (kChunk == 32) ptx::tmem_ld32(ta, o); else if constexpr (kChunk == 16) ptx::tmem_ld16(ta, o); else ptx::tmem_ld8(ta, o);
           ptx::tmem_wait_ld();
-        } else {
+          uint32_t u[kChunk];
 #pragma unroll
-          for (int z = 0; z < kChunk; ++z) o[z] = 0.f;
-        }
-        if (m < args.M) {
-#pragma unroll
-          for (int z = 0; z < kChunk / 4; ++z)
-            dst[c * (kChunk / 4) + z] = make_float4(o[4 * z], o[4 * z + 1], o[4 * z + 2], o[4 * z + 3]);
+          for (int z = 0; z < kChunk; ++z) u[z] = __float_as_uint(o[z] * alpha);
+          if constexpr (kChunk == 32) ptx::tmem_st32(ta, u); else if constexpr (kChunk == 16) ptx::tmem_st16(ta, u); else ptx::tmem_st8(ta, u);
         }
       }
-      if (m < args.M) {
-        args.m_part[row] = has ? mref[b] : -INFINITY;
-        args.l_part[row] = has ? l[b] : 0.f;
-      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&P_full[2 * s + j]);
     }
     if (!ok) {
       record_error(args.status, kErrTimeout, kSiteEncSoftmax);
       *s_abort = 1;
     }
+
+    // ---------------------------------------------------------- epilogue
+    // Every group publishes (mref, l); the writer groups (both groups of a
+    // slot when M > 128, slot 0's when M <= 128) fold the accumulators that
+    // cover their rows into one partial, group c writing columns
+    // [c D / 2, +D / 2).
+    s_ml[(s * 2 + c) * kLatRows + r] = make_float2(count > 0 ? mref : -INFINITY, count > 0 ? l : 0.f);
+    __syncwarp();
+    asm volatile("bar.sync 3, 512;" ::: "memory");  // all four groups
+    const bool writer = NHALF == 2 || s == 0;
+    if (writer && ok) {
+      constexpr int kSlotsIn = NHALF == 2 ? 1 : 2;      // slots folded into the partial
+      constexpr int kAcc = kSlotsIn * C::kAccPerSlot;  // accumulators folded
+      float w[kAcc], ms = -INFINITY, lsum = 0.f;
+#pragma unroll
+      for (int u = 0; u < kSlotsIn; ++u) {
+        const int su = NHALF == 2 ? s : u;
+        if (count_of(su) == 0) continue;  // uniform
+#pragma unroll
+        for (int cu = 0; cu < C::kAccPerSlot; ++cu) ms = fmaxf(ms, s_ml[(su * 2 + cu) * kLatRows + r].x);
+        ok = ok && __all_sync(0xffffffffu, ptx::mbar_wait(&O_final[su], 0, s_abort, args.wait_ns));
+      }
+#pragma unroll
+      for (int u = 0; u < kSlotsIn; ++u) {
+        const int su = NHALF == 2 ? s : u;
+        const float2 a0 = s_ml[(su * 2) * kLatRows + r], a1 = s_ml[(su * 2 + 1) * kLatRows + r];
+        if constexpr (C::kSplitO) {
+          w[2 * u] = count_of(su) > 0 ? ptx::ex2(a0.x - ms) : 0.f;
+          w[2 * u + 1] = count_of(su) > 0 ? ptx::ex2(a1.x - ms) : 0.f;
+          lsum = fmaf(w[2 * u], a0.y, fmaf(w[2 * u + 1], a1.y, lsum));
+        } else {
+          // one accumulator, one reference per slot; both halves' sums
+          w[u] = count_of(su) > 0 ? ptx::ex2(a0.x - ms) : 0.f;
+          lsum = fmaf(w[u], a0.y + a1.y, lsum);
+        }
+      }
+      if (ok) {
+        ptx::tc_fence_after();
+        const size_t row = (static_cast<size_t>(bh) * args.P + split) * args.M + m;
+        constexpr int kHalfD = D / 2;
+        constexpr int kChunk = kHalfD < 32 ? kHalfD : 32;
+        float4* dst = reinterpret_cast<float4*>(args.O_part + row * D + c * kHalfD);
+#pragma unroll
+        for (int z0 = 0; z0 < kHalfD; z0 += kChunk) {
+          float acc[kChunk];
+#pragma unroll
+          for (int z = 0; z < kChunk; ++z) acc[z] = 0.f;
+#pragma unroll
+          for (int a = 0; a < kAcc; ++a) {
+            const int su = NHALF == 2 ? s : a / C::kAccPerSlot;
+            if (count_of(su) == 0) continue;  // its accumulator was never written
+            float o[kChunk];
+            const uint32_t ta = tmem + lane_off + C::col_o(su, a % C::kAccPerSlot) + c * kHalfD + z0;
+            if constexpr (kChunk == 32) ptx::tmem_ld32(ta, o); else if constexpr (kChunk == 16) ptx::tmem_ld16(ta, o); else ptx::tmem_ld8(ta, o);
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int z = 0; z < kChunk; ++z) acc[z] = fmaf(w[a], o[z], acc[z]);
+          }
+          if (m < args.M) {
+#pragma unroll
+            for (int z = 0; z < kChunk / 4; ++z)
+              dst[z0 / 4 + z] = make_float4(acc[4 * z], acc[4 * z + 1], acc[4 * z + 2], acc[4 * z + 3]);
+          }
+        }
+        if (m < args.M && c == 0) {
+          args.m_part[row] = ms;
+          args.l_part[row] = lsum;
+        }
+      } else {
+        record_error(args.status, kErrTimeout, kSiteEncSoftmax);
+        *s_abort = 1;
+      }
+    }
   }
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::kProducerWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }

@@ -201,7 +201,7 @@ cudaError_t launch_encode_tc_n(int D, const CUtensorMap& q, const CUtensorMap& k
     case 16: return launch_encode_tc_t<16, NHALF, 16>(q, k, v, a, BH, st);
     case 32: return launch_encode_tc_t<32, NHALF, 8>(q, k, v, a, BH, st);
     case 64: return launch_encode_tc_t<64, NHALF, 8>(q, k, v, a, BH, st);
-    default: return launch_encode_tc_t<128, NHALF, 4>(q, k, v, a, BH, st);
+    default: return launch_encode_tc_t<128, NHALF, NHALF == 2 ? 4 : 5>(q, k, v, a, BH, st);
   }
 }
 
@@ -286,6 +286,7 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
         !make_map(&tv, V, D, N, BH, kEncTile))
       return FLARE_ERR_CUDA;
     EncodeArgs a;
+    a.Q = Q;
     a.N = static_cast<int>(N);
     a.M = M;
     a.q_batched = q_batched;
