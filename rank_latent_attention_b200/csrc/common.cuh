@@ -53,6 +53,26 @@ __device__ __forceinline__ float exp2_poly3(float x) {
   return __uint_as_float(__float_as_uint(p) + (__float_as_uint(r) << 23));
 }
 
+// exp2_poly3 on a packed pair (lo, hi): the same steps, the fp32 adds and
+// multiply-adds as f32x2 instructions.
+__device__ __forceinline__ uint64_t exp2_poly3_x2(uint64_t x) {
+  constexpr float kRound = 12582912.f;  // 1.5 * 2^23
+  float x0, x1;
+  ptx::f2_split(x, x0, x1);
+  const uint64_t xc = ptx::f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t r = ptx::add2(xc, ptx::f2(kRound, kRound));
+  const uint64_t j = ptx::add2(r, ptx::f2(-kRound, -kRound));
+  const uint64_t f = ptx::fma2(j, ptx::f2(-1.f, -1.f), xc);  // xc - j, exact product, one rounding
+  uint64_t p = ptx::fma2(ptx::f2(0.0551716685f, 0.0551716685f), f, ptx::f2(0.242611125f, 0.242611125f));
+  p = ptx::fma2(p, f, ptx::f2(0.693260968f, 0.693260968f));
+  p = ptx::fma2(p, f, ptx::f2(0.999928057f, 0.999928057f));
+  float p0, p1, r0, r1;
+  ptx::f2_split(p, p0, p1);
+  ptx::f2_split(r, r0, r1);
+  return ptx::f2(__uint_as_float(__float_as_uint(p0) + (__float_as_uint(r0) << 23)),
+                 __uint_as_float(__float_as_uint(p1) + (__float_as_uint(r1) << 23)));
+}
+
 // Record the first failure in the device status word {code, site}.
 __device__ __forceinline__ void record_error(int* status, int code, int site) {
   if (atomicCAS(status, 0, code) == 0) atomicExch(status + 1, site);

@@ -135,33 +135,42 @@ struct EncodeCfg {
 // exponential on MUFU, and masked columns give exactly 0.
 template <bool RAGGED>
 __device__ __forceinline__ float encode_exp_store(const float* x, float nref, uint32_t tP) {
-  float ps[4] = {0.f, 0.f, 0.f, 0.f};  // independent partial sums
+  // pairs of columns as packed fp32 (f32x2): x log2e - nref, the polynomial
+  // exponentials and the running sums take one instruction per pair
+  const uint64_t kL2 = ptx::f2(kLog2e, kLog2e);
+  const uint64_t nn = ptx::f2(-nref, -nref);
+  uint64_t ps[2] = {0ull, 0ull};  // two independent packed partial sums (+0.0f pairs)
 #pragma unroll
   for (int c0 = 0; c0 < 32; c0 += 16) {
     uint32_t p[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int c = c0 + 2 * u;
-      const float a0 = fmaf(x[c], kLog2e, -nref);
-      const float a1 = fmaf(x[c + 1], kLog2e, -nref);
-      float p0, p1;
+      const uint64_t a = ptx::fma2(ptx::f2(x[c], x[c + 1]), kL2, nn);
+      uint64_t e;
       if (!RAGGED && ((kEncPolyPairs >> ((c / 2) & 15)) & 1u)) {
-        p0 = exp2_poly3(a0);
-        p1 = exp2_poly3(a1);
+        e = exp2_poly3_x2(a);
       } else {
-        p0 = ptx::ex2(a0);
-        p1 = ptx::ex2(a1);
+        float a0, a1;
+        ptx::f2_split(a, a0, a1);
+        float p0 = ptx::ex2(a0), p1 = ptx::ex2(a1);
         if (RAGGED) {  // a half-row may be fully masked with no reference yet (-inf - -inf)
           p0 = x[c] == -INFINITY ? 0.f : p0;
           p1 = x[c + 1] == -INFINITY ? 0.f : p1;
         }
+        e = ptx::f2(p0, p1);
       }
-      ps[u & 3] += p0 + p1;
-      p[u] = ptx::pack_bf16(p0, p1);
+      ps[u & 1] = ptx::add2(ps[u & 1], e);
+      float e0, e1;
+      ptx::f2_split(e, e0, e1);
+      p[u] = ptx::pack_bf16(e0, e1);
     }
     ptx::tmem_st8(tP + c0 / 2, p);
   }
-  return (ps[0] + ps[1]) + (ps[2] + ps[3]);
+  float s0, s1, s2, s3;
+  ptx::f2_split(ps[0], s0, s1);
+  ptx::f2_split(ps[1], s2, s3);
+  return (s0 + s1) + (s2 + s3);
 }
 
 template <int D, int NHALF, int NS>
