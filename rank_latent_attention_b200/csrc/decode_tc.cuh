@@ -8,21 +8,35 @@
 // attention routing", "Méthodologie : FLARE++", routing encode-decode).
 //
 // Work of one CTA: one (b, h), Q and Z of that head resident in shared
-// memory, and a contiguous run of 128-token tiles.
-//   warp 0      TMA producer: Q and Z once, then K tiles into an NS-deep ring
-//   warp 1      TMEM allocator + tcgen05.mma issuer of slot 0 (one thread)
-//   warp 2      tcgen05.mma issuer of slot 1 (one thread)
-//   warps 4-7   epilogue warpgroup of slot 0 (even tiles), one thread per token
-//   warps 8-11  epilogue warpgroup of slot 1 (odd tiles)
-// The slots own disjoint TMEM columns and each has its own issuer, so one
-// slot's waits never hold up the other slot's MMAs.
-// Per tile: S = K_tile Q^T (128 x MP, fp32, TMEM), the owning thread takes
-// the max over its row's M valid latents, writes P = 2^(s log2e - max) as bf16
-// over the first MP/2 columns, then O = P Z (128 x D) lands in columns
-// [128, 128 + D) of the slot; the thread scales by 1/sum and stores its
-// token's row of Y as bf16.
+// memory, and a contiguous run of 128-token tiles, taken alternately by two
+// slots.
+//   warps 0-15   four softmax warpgroups (slot s, latent half c): thread r of
+//                group (s, c) owns token r of the slot's tiles and latents
+//                [c MP / 2, (c + 1) MP / 2)
+//   warp 16      TMA producer: Q and Z once, then K tiles into an NS ring;
+//                also allocates TMEM
+//   warps 17-18  tcgen05.mma issuers, one warp per slot
+// Per tile of a slot: S = K_tile Q^T (128 x MP fp32 in TMEM); each group takes
+// the max over its half-row, the two groups exchange it through shared
+// memory (named barrier), each writes P = 2^(s log2e - max) as bf16 pairs
+// into its own score columns and keeps its half of the row sum; then
+// O = P Z (128 x D) in TMEM, and each group scales half of O's columns by
+// 1 / (sum of both halves) and stores them as bf16 rows of Y.  S of the
+// slot's next tile is computed as soon as its columns are free: the latent
+// half whose columns hold no O with P.V, the other once O has been read.
+// The slots take turns at the exponentials, so one slot's softmax overlaps
+// the other's MMAs and epilogue.
 //
-// TMEM: slot s owns columns [256 s, 256 s + 256).
+// The issuer warps run their loop as a whole and issue under elect.sync,
+// which keeps the MMA operands warp-uniform.  The softmax arithmetic runs on
+// packed fp32 pairs (f32x2), and 5 of every 16 column pairs take their
+// exponentials from exp2_poly3 (FMA pipe) instead of MUFU.
+//
+// TMEM: slot s owns columns [256 s, 256 s + 256): S at [0, MP); P of group 0
+// at [0, MP / 4) (latent pairs in order, written over scores already read);
+// P of group 1 at [3 MP / 4, MP) (its chunks processed last to first, so each
+// P chunk lands on scores already read); O at kColO: [MP / 4, MP / 4 + D) for
+// MP = 256 (free once both groups have stored P), [128, 128 + D) for MP = 128.
 #pragma once
 
 #include "common.cuh"
@@ -41,31 +55,211 @@ struct DecodeArgs {
   unsigned long long wait_ns;
 };
 
+// Column pairs (bit j: pair j of each 16) whose exponentials go to
+// exp2_poly3 in the decode softmax.
+constexpr uint32_t kDecPolyPairs = 0x2491u;
+
 template <int D, int MP, int NS>
 struct DecodeCfg {
   using G = TileGeom<D>;
   static_assert(MP == 128 || MP == 256, "padded latent count");
+  static constexpr int kHalf = MP / 2;      // latents per group
+  static constexpr int kChunks = kHalf / 32;  // 32-latent chunks per group
+  static constexpr int kProducerWarp = 16;
+  static constexpr int kIssuerWarp = 17;  // + slot
+  static constexpr int kThreads = 32 * 19;
   static constexpr int kLatBytes = G::bytes(MP);
   static constexpr int kTileBytes = G::bytes(kTileN);
   static constexpr int kOffQ = 0;
   static constexpr int kOffZ = kLatBytes;
   static constexpr int kOffStages = 2 * kLatBytes;
   static constexpr int kOffBars = kOffStages + NS * kTileBytes;
-  // full[NS], empty[NS], qz_full, S_full[2], P_full[2], O_full[2], O_free[2], drain
-  static constexpr int kNumBars = 2 * NS + 10;
-  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
+  // full[NS], empty[NS], qz_full, S_full[2], P_full[2], O_full[2], O_free[2], turn[2], drain
+  static constexpr int kNumBars = 2 * NS + 12;
+  static constexpr int kOffXM = kOffBars + 8 * kNumBars;  // float [2 slot][2 half][128]: half-row max
+  static constexpr int kOffXL = kOffXM + 2 * 2 * 128 * 4;  // float [2 slot][2 half][128]: half-row sum
+  static constexpr int kOffMisc = kOffXL + 2 * 2 * 128 * 4;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSlotCols = 256;
-  static constexpr uint32_t kColO = 128;  // O inside a slot
-  static_assert(MP / 2 <= kColO && kColO + D <= kSlotCols, "TMEM slot layout");
+  static constexpr uint32_t kColP1 = 3 * MP / 4;
+  static constexpr uint32_t kColO = MP == 256 ? MP / 4 : 128;
+  static_assert(kColO + D <= (MP == 256 ? kColP1 : kSlotCols), "TMEM slot layout");
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16(kTileN, MP, 0, 0);
+  static constexpr uint32_t kIdescQKHalf = ptx::idesc_bf16(kTileN, kLatRows, 0, 0);  // one latent half
   static constexpr uint32_t kIdescPV = ptx::idesc_bf16(kTileN, D, 0, 1);
+  // TMEM column (within the slot) of P for latents [16 kk, +16): the PV K step kk
+  __host__ __device__ static constexpr uint32_t col_pk(int kk) {
+    return kk < MP / 32 ? 8 * kk : kColP1 + 8 * (kk - MP / 32);
+  }
+};
+
+// P for one 32-latent chunk of a row: 2^(x log2e - mref) for the valid
+// columns (16-column groups at or past M give P = 0), packed to bf16 pairs
+// into 16 TMEM columns at tP; returns the fp32 sum.
+template <int MP>
+__device__ __forceinline__ float decode_exp_chunk(const float* x, float mref, int col0, int M, uint32_t tP) {
+  const uint64_t kL2 = ptx::f2(kLog2e, kLog2e);
+  const uint64_t nn = ptx::f2(-mref, -mref);
+  uint64_t ps[2] = {0ull, 0ull};
+#pragma unroll
+  for (int g = 0; g < 2; ++g) {
+    uint32_t p[8];
+    if (col0 + 16 * g < M) {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int c = 16 * g + 2 * u;
+        const uint64_t a = ptx::fma2(ptx::f2(x[c], x[c + 1]), kL2, nn);
+        uint64_t e;
+        if ((kDecPolyPairs >> (u + 8 * g)) & 1u) {
+          e = exp2_poly3_x2(a);
+        } else {
+          float a0, a1;
+          ptx::f2_split(a, a0, a1);
+          e = ptx::f2(ptx::ex2(a0), ptx::ex2(a1));
+        }
+        ps[u & 1] = ptx::add2(ps[u & 1], e);
+        float e0, e1;
+        ptx::f2_split(e, e0, e1);
+        p[u] = ptx::pack_bf16(e0, e1);
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 8; ++u) p[u] = 0u;
+    }
+    ptx::tmem_st8(tP + 8 * g, p);
+  }
+  float s0, s1, s2, s3;
+  ptx::f2_split(ps[0], s0, s1);
+  ptx::f2_split(ps[1], s2, s3);
+  return (s0 + s1) + (s2 + s3);
+}
+
+// The softmax / epilogue loop of one group (slot s, latent half CH).
+template <int D, int MP, int NS>
+struct DecodeGroup {
+  using C = DecodeCfg<D, MP, NS>;
+  const DecodeArgs& args;
+  uint32_t tmem;
+  int warp, lane, s, tile0, T;
+  uint64_t *S_full, *P_full, *O_full, *O_free, *turn;
+  float* xm;  // [2 half][128] of this slot
+  float* xl;
+  volatile int* s_abort;
+
+  template <int CH>
+  __device__ __forceinline__ void run() {
+    const int r = (warp & 3) * 32 + lane;  // token row within the tile
+    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_off + s * C::kSlotCols;
+    const int count = s == 0 ? (T + 1) / 2 : T / 2;
+    const int M = args.M;
+    constexpr int kLat0 = CH * C::kHalf;  // first latent (S column) of this group
+    bool ok = true;
+    for (int i = 0; i < count; ++i) {
+      const int t = 2 * i + s;
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&S_full[s], i & 1, s_abort, args.wait_ns))) {
+        ok = false;
+        break;
+      }
+      ptx::tc_fence_after();
+      // pass 1: max over this group's valid latents (M is a multiple of 16,
+      // so validity is uniform per 16-column group)
+      float pm[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) pm[j] = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < C::kChunks; ++k) {
+        float x[32];
+        ptx::tmem_ld32(tS + kLat0 + 32 * k, x);
+        ptx::tmem_wait_ld();
+#pragma unroll
+        for (int h = 0; h < 2; ++h)
+          if (kLat0 + 32 * k + 16 * h < M) {
+#pragma unroll
+            for (int j = 0; j < 8; ++j) pm[j] = ptx::max3(pm[j], x[16 * h + 2 * j], x[16 * h + 2 * j + 1]);
+          }
+      }
+      // exchange with the other group of the slot: the row max over all latents
+      xm[CH * 128 + r] = ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+      asm volatile("bar.sync %0, 256;" ::"r"(1 + s) : "memory");
+      const float mref = fmaxf(xm[r], xm[128 + r]) * kLog2e;
+      // The slots take turns at the exponentials (slot 0's tile i, slot 1's
+      // tile i, slot 0's tile i + 1, ...): one slot computes while the other
+      // slot's P.V, epilogue and next Q.K^T run.
+      if ((s == 1 || i > 0) &&
+          !__all_sync(0xffffffffu, ptx::mbar_wait(&turn[s], (s == 1 ? i : i - 1) & 1, s_abort, args.wait_ns))) {
+        ok = false;
+        break;
+      }
+      // pass 2: P chunk by chunk (group 1 last to first, see the layout note)
+      float l = 0.f;
+#pragma unroll
+      for (int q = 0; q < C::kChunks; ++q) {
+        const int k = CH == 0 ? q : C::kChunks - 1 - q;
+        float x[32];
+        ptx::tmem_ld32(tS + kLat0 + 32 * k, x);
+        ptx::tmem_wait_ld();
+        l += decode_exp_chunk<MP>(x, mref, kLat0 + 32 * k, M, tS + (CH == 0 ? 16 * k : C::kColP1 + 16 * k));
+      }
+      xl[CH * 128 + r] = l;
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&turn[s ^ 1]);
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&P_full[s]);
+
+      // epilogue: O = P Z; this group scales columns [CH D / 2, +D / 2)
+      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&O_full[s], i & 1, s_abort, args.wait_ns))) {
+        ok = false;
+        break;
+      }
+      asm volatile("bar.sync %0, 256;" ::"r"(3 + s) : "memory");  // both halves' sums are in xl
+      const float inv = 1.f / (xl[r] + xl[128 + r]);
+      ptx::tc_fence_after();
+      constexpr int kHD = D / 2;
+      const uint32_t tO = tS + C::kColO + CH * kHD;
+      float o[kHD];
+      if constexpr (kHD == 64) {
+        ptx::tmem_ld32(tO, o);
+        ptx::tmem_ld32(tO + 32, o + 32);
+      } else if constexpr (kHD == 32) {
+        ptx::tmem_ld32(tO, o);
+      } else if constexpr (kHD == 16) {
+        ptx::tmem_ld16(tO, o);
+      } else {
+        ptx::tmem_ld8(tO, o);
+      }
+      ptx::tmem_wait_ld();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(&O_free[s]);
+
+      const long long tok = static_cast<long long>(tile0 + t) * kTileN + r;
+      if (tok < args.N) {
+        uint4* dst = reinterpret_cast<uint4*>(args.Y + (static_cast<size_t>(blockIdx.y) * args.N + tok) * D + CH * kHD);
+#pragma unroll
+        for (int z = 0; z < kHD / 8; ++z) {
+          uint4 v;
+          v.x = ptx::pack_bf16(o[8 * z + 0] * inv, o[8 * z + 1] * inv);
+          v.y = ptx::pack_bf16(o[8 * z + 2] * inv, o[8 * z + 3] * inv);
+          v.z = ptx::pack_bf16(o[8 * z + 4] * inv, o[8 * z + 5] * inv);
+          v.w = ptx::pack_bf16(o[8 * z + 6] * inv, o[8 * z + 7] * inv);
+          dst[z] = v;
+        }
+      }
+    }
+    if (!ok) {
+      record_error(args.status, kErrTimeout, kSiteDecSoftmax);
+      *s_abort = 1;
+    }
+  }
 };
 
 template <int D, int MP, int NS>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
                      const __grid_constant__ CUtensorMap tmZ, const DecodeArgs args) {
   using C = DecodeCfg<D, MP, NS>;
@@ -80,7 +274,10 @@ __global__ void __launch_bounds__(384, 1)
   uint64_t* P_full = bars + 2 * NS + 3;
   uint64_t* O_full = bars + 2 * NS + 5;
   uint64_t* O_free = bars + 2 * NS + 7;
-  uint64_t* drain = bars + 2 * NS + 9;
+  uint64_t* turn = bars + 2 * NS + 9;  // [slot]: the other slot has finished its exponentials
+  uint64_t* drain = bars + 2 * NS + 11;
+  float* s_xm = reinterpret_cast<float*>(smem + C::kOffXM);
+  float* s_xl = reinterpret_cast<float*>(smem + C::kOffXL);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -100,15 +297,16 @@ __global__ void __launch_bounds__(384, 1)
     ptx::mbar_init(qz_full, 1);
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&S_full[s], 1);
-      ptx::mbar_init(&P_full[s], 4);
+      ptx::mbar_init(&P_full[s], 8);  // one arrival per warp of the slot's two groups
       ptx::mbar_init(&O_full[s], 1);
-      ptx::mbar_init(&O_free[s], 4);
+      ptx::mbar_init(&O_free[s], 8);
+      ptx::mbar_init(&turn[s], 8);
     }
-    ptx::mbar_init(drain, 2);  // one commit per issuer
+    ptx::mbar_init(drain, 64);  // one commit per lane of the two issuer warps
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
-  if (warp == 1) {
+  if (warp == C::kProducerWarp) {
     ptx::tmem_alloc(s_tmem, C::kTmemCols);
     ptx::tmem_relinquish();
   }
@@ -118,7 +316,7 @@ __global__ void __launch_bounds__(384, 1)
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = ptx::smem_u32(smem);
 
-  if (warp == 0) {
+  if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       ptx::prefetch_tmap(&tmK);
@@ -151,179 +349,104 @@ __global__ void __launch_bounds__(384, 1)
       for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
         ptx::mbar_wait_drain(&full[t % NS], (t / NS) & 1);
     }
-  } else if (warp == 1 || warp == 2) {
-    // ------------------------------------------------------------ MMA issuers (one per slot)
-    if (lane == 0) {
-      static_assert((NS & (NS - 1)) == 0, "ring depth must be a power of two");
-      const int slot = warp - 1;
-      bool ok = ptx::mbar_wait(qz_full, 0, s_abort, args.wait_ns);
-      ptx::tc_fence_after();
-      // descriptors of stage 0 / K step 0; stages and K steps only move the start address
-      const uint64_t dK0 = G::kmajor(sbase + C::kOffStages, kTileN, 0);
-      const uint64_t dQ0 = G::kmajor(sbase + C::kOffQ, MP, 0);
-      const uint64_t dZ0 = G::mnmajor(sbase + C::kOffZ, MP, 0);
-      const uint32_t tS = tmem + slot * C::kSlotCols;
-      // The issuing thread stalls on any shared-memory access until its own
-      // MMAs have completed: waits go before each group of MMAs.
-      auto wait_stage = [&](int t) -> bool {
-        return ptx::mbar_wait(&full[t & (NS - 1)], (t / NS) & 1, s_abort, args.wait_ns);
-      };
-      auto issue_qk = [&](int t) {
-        const int st = t & (NS - 1);
-        const uint64_t dK = dK0 + static_cast<uint32_t>(st * (C::kTileBytes >> 4));
+  } else if (warp >= C::kIssuerWarp) {
+    // ------------------------------------------------------------ MMA issuers (one warp per slot)
+    // The whole warp runs the loop (waits are warp-wide); one elected lane
+    // issues each batch of MMAs and the commits that track them.
+    const int slot = warp - C::kIssuerWarp;
+    const uint64_t dK0 = G::kmajor(sbase + C::kOffStages, kTileN, 0);
+    const uint64_t dQ0 = G::kmajor(sbase + C::kOffQ, MP, 0);
+    const uint64_t dZ0 = G::mnmajor(sbase + C::kOffZ, MP, 0);
+    const uint32_t tS = tmem + slot * C::kSlotCols;
+    auto wait_stage = [&](int t) -> bool {
+      return ptx::mbar_wait(&full[t % NS], (t / NS) & 1, s_abort, args.wait_ns);
+    };
+    // Q.K^T of tile t over latent half h ([128 h, +128), N = 128), or over
+    // all MP latents (h < 0)
+    auto issue_qk = [&](int t, int h) {
+      const uint64_t dK = dK0 + static_cast<uint32_t>((t % NS) * (C::kTileBytes >> 4));
+      const uint64_t dQ = dQ0 + static_cast<uint32_t>(((h > 0 ? h : 0) * kLatRows * G::kRowBytes) >> 4);
+      const uint32_t tD = tS + (h > 0 ? h * kLatRows : 0);
+      const uint32_t idesc = h < 0 ? C::kIdescQK : C::kIdescQKHalf;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k)
-          ptx::mma_ss(tS, dK + G::kmajor_step(kTileN, k), dQ0 + G::kmajor_step(MP, k), C::kIdescQK, k > 0 ? 1u : 0u);
-        ptx::mma_commit(&S_full[slot]);
-        ptx::mma_commit(&empty[st]);
-      };
-      auto issue_pv = [&]() {
+      for (int k = 0; k < D / 16; ++k)
+        ptx::mma_ss(tD, dK + G::kmajor_step(kTileN, k), dQ + G::kmajor_step(MP, k), idesc, k > 0 ? 1u : 0u);
+    };
+    auto commit_s = [&](int t) {
+      ptx::mma_commit(&S_full[slot]);
+      ptx::mma_commit(&empty[t % NS]);  // both halves of Q.K^T(t) have read the stage
+    };
+    bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(qz_full, 0, s_abort, args.wait_ns));
+    // this slot's tiles: t = slot + 2 i
+    if (ok && slot < T) {
+      ok = __all_sync(0xffffffffu, wait_stage(slot));
+      if (ok) {
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
+          issue_qk(slot, -1);
+          commit_s(slot);
+        }
+        __syncwarp();
+      }
+    }
+    // Batch of tile t: P(t).V, then the part of Q.K^T(t + 2) whose columns
+    // hold no O (MP = 256: latents 128-255; MP = 128: all of S, O lies past
+    // it); with MP = 256 the other half follows once O has been read.  With
+    // MP = 128 the next P.V waits for O to be read instead.
+    for (int i = 0; ok && slot + 2 * i < T; ++i) {
+      const int t = slot + 2 * i;
+      const bool next = t + 2 < T;
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&P_full[slot], i & 1, s_abort, args.wait_ns) &&
+                                       (MP == 256 || i == 0 ||
+                                        ptx::mbar_wait(&O_free[slot], (i - 1) & 1, s_abort, args.wait_ns)) &&
+                                       (!next || wait_stage(t + 2)));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
 #pragma unroll
         for (int k = 0; k < MP / 16; ++k)
-          ptx::mma_ts(tS + C::kColO, tS + k * 8, dZ0 + G::mnmajor_step(k), C::kIdescPV, k > 0 ? 1u : 0u);
+          ptx::mma_ts(tS + C::kColO, tS + C::col_pk(k), dZ0 + G::mnmajor_step(k), C::kIdescPV, k > 0 ? 1u : 0u);
         ptx::mma_commit(&O_full[slot]);
-      };
-      // this slot's tiles: t = slot + 2 i
-      if (ok && slot < T) {
-        ok = wait_stage(slot);
-        if (ok) {
-          ptx::tc_fence_after();
-          issue_qk(slot);
+        if (next) {
+          if constexpr (MP == 256) {
+            issue_qk(t + 2, 1);
+          } else {
+            issue_qk(t + 2, -1);
+            commit_s(t + 2);
+          }
         }
       }
-      for (int i = 0; ok && slot + 2 * i < T; ++i) {
-        const int t = slot + 2 * i;
-        ok = (t + 2 >= T || wait_stage(t + 2)) && ptx::mbar_wait(&P_full[slot], i & 1, s_abort, args.wait_ns);
+      __syncwarp();
+      if (MP == 256 && next) {
+        // latents 0-127 share their columns with O: once both groups have read it
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&O_free[slot], i & 1, s_abort, args.wait_ns));
         if (!ok) break;
         ptx::tc_fence_after();
-        issue_pv();
-        if (t + 2 < T) {
-          // the slot's columns are reused once its epilogue has read O of tile t
-          ok = ptx::mbar_wait(&O_free[slot], i & 1, s_abort, args.wait_ns);
-          if (ok) {
-            ptx::tc_fence_after();
-            issue_qk(t + 2);
-          }
+        if (ptx::elect_one()) {
+          issue_qk(t + 2, 0);
+          commit_s(t + 2);
         }
-      }
-      if (!ok) {
-        record_error(args.status, kErrTimeout, kSiteDecMma);
-        *s_abort = 1;
-      }
-      ptx::mma_commit(drain);
-      ptx::mbar_wait_drain(drain, 0);
-    }
-  } else if (warp >= 4) {
-    // ------------------------------------------------------------ softmax / epilogue warpgroups
-    const int s = (warp - 4) >> 2;
-    const int r = (warp & 3) * 32 + lane;  // token row within the tile
-    const uint32_t lane_off = static_cast<uint32_t>((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_off + s * C::kSlotCols;
-    const uint32_t tO = tS + C::kColO;
-    const int count = s == 0 ? (T + 1) / 2 : T / 2;
-    const int M = args.M;
-    bool ok = true;
-    for (int i = 0; i < count; ++i) {
-      const int t = 2 * i + s;
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&S_full[s], i & 1, s_abort, args.wait_ns))) {
-        ok = false;
-        break;
-      }
-      ptx::tc_fence_after();
-      // pass 1: row max over the M valid latents (columns >= M are padding;
-      // M is a multiple of 16, so validity is uniform per 16-column group)
-      float pm[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) pm[j] = -INFINITY;
-#pragma unroll
-      for (int c0 = 0; c0 < MP; c0 += 128) {
-        float x[128];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) ptx::tmem_ld32(tS + c0 + 32 * c, x + 32 * c);
-        ptx::tmem_wait_ld();
-#pragma unroll
-        for (int g = 0; g < 8; ++g)
-          if (c0 + 16 * g < M) {
-#pragma unroll
-            for (int j = 0; j < 8; ++j) pm[j] = ptx::max3(pm[j], x[16 * g + 2 * j], x[16 * g + 2 * j + 1]);
-          }
-      }
-      const float mref =
-          ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7])) * kLog2e;
-      // pass 2: P = 2^(s log2e - mref) as bf16 pairs over the first MP/2 columns
-      // (P of columns [c0, c0+64) lands in [c0/2, c0/2+32), already read)
-      float ps[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
-#pragma unroll
-      for (int c0 = 0; c0 < MP; c0 += 64) {
-        float x[64];
-        ptx::tmem_ld32(tS + c0, x);
-        ptx::tmem_ld32(tS + c0 + 32, x + 32);
-        ptx::tmem_wait_ld();
-        uint32_t p[32];
-#pragma unroll
-        for (int g = 0; g < 4; ++g) {
-          if (c0 + 16 * g < M) {
-#pragma unroll
-            for (int c = 16 * g; c < 16 * g + 16; c += 2) {
-              const float p0 = ptx::ex2(fmaf(x[c], kLog2e, -mref));
-              const float p1 = ptx::ex2(fmaf(x[c + 1], kLog2e, -mref));
-              ps[(c / 2) & 7] += p0 + p1;
-              p[c / 2] = ptx::pack_bf16(p0, p1);
-            }
-          } else {
-#pragma unroll
-            for (int c = 16 * g; c < 16 * g + 16; c += 2) p[c / 2] = 0u;
-          }
-        }
-        ptx::tmem_st32(tS + c0 / 2, p);
-      }
-      const float l = ((ps[0] + ps[1]) + (ps[2] + ps[3])) + ((ps[4] + ps[5]) + (ps[6] + ps[7]));
-      ptx::tmem_wait_st();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&P_full[s]);
-
-      if (!__all_sync(0xffffffffu, ptx::mbar_wait(&O_full[s], i & 1, s_abort, args.wait_ns))) {
-        ok = false;
-        break;
-      }
-      ptx::tc_fence_after();
-      float o[D];
-      if constexpr (D >= 32) {
-#pragma unroll
-        for (int c = 0; c < D / 32; ++c) ptx::tmem_ld32(tO + 32 * c, o + 32 * c);
-      } else {
-        ptx::tmem_ld16(tO, o);
-      }
-      ptx::tmem_wait_ld();
-      ptx::tc_fence_before();
-      __syncwarp();
-      if (lane == 0) ptx::mbar_arrive(&O_free[s]);
-
-      const long long tok = static_cast<long long>(tile0 + t) * kTileN + r;
-      if (tok < args.N) {
-        const float inv = 1.f / l;
-        uint4* dst = reinterpret_cast<uint4*>(args.Y + (static_cast<size_t>(bh) * args.N + tok) * D);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          uint4 v;
-          v.x = ptx::pack_bf16(o[8 * c + 0] * inv, o[8 * c + 1] * inv);
-          v.y = ptx::pack_bf16(o[8 * c + 2] * inv, o[8 * c + 3] * inv);
-          v.z = ptx::pack_bf16(o[8 * c + 4] * inv, o[8 * c + 5] * inv);
-          v.w = ptx::pack_bf16(o[8 * c + 6] * inv, o[8 * c + 7] * inv);
-          dst[c] = v;
-        }
+        __syncwarp();
       }
     }
-    if (!ok) {
-      record_error(args.status, kErrTimeout, kSiteDecSoftmax);
+    if (!ok && lane == 0) {
+      record_error(args.status, kErrTimeout, kSiteDecMma);
       *s_abort = 1;
     }
+    // Drain: every lane commits (a lane that issued nothing arrives at once).
+    ptx::mma_commit(drain);
+    ptx::mbar_wait_drain(drain, 0);
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue groups
+    const int s = warp >> 3;  // slot
+    DecodeGroup<D, MP, NS> grp{args, tmem, warp, lane, s, tile0, T, S_full, P_full, O_full, O_free, turn,
+                               s_xm + (s * 2) * 128, s_xl + (s * 2) * 128, s_abort};
+    if ((warp >> 2) & 1) grp.template run<1>(); else grp.template run<0>();
   }
 
   ptx::tc_fence_before();
   __syncthreads();
-  if (warp == 1) {
+  if (warp == C::kProducerWarp) {
     ptx::tc_fence_after();
     ptx::tmem_dealloc(tmem, C::kTmemCols);
   }

@@ -212,7 +212,7 @@ cudaError_t launch_decode_tc_t(const CUtensorMap& k, const CUtensorMap& q, const
   auto kern = decode_tc_kernel<D, MP, NS>;
   static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  kern<<<dim3(a.splits, BH), 384, C::kSmemBytes, st>>>(k, q, z, a);
+  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(k, q, z, a);
   return cudaGetLastError();
 }
 
