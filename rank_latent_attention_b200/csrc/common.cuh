@@ -33,9 +33,11 @@ constexpr int kLatRows = 128; // latent rows per tcgen05 MMA (M = 128, cta_group
 
 // 2^x on the FMA/ALU pipes, for the share of a softmax tile's exponentials
 // that would otherwise queue behind the MUFU unit (16 results per clock per
-// SM on sm_100, the binding resource of the softmax).  For -126 <= x <= 64 the
-// relative error is below 7.5e-5 (P is then rounded to bf16, 2^-9); x < -126
-// gives 2^-126 in place of a value below the smallest normal.
+// SM on sm_100, the binding resource of the softmax).  For -125 <= x <= 64 the
+// relative error is below 7.5e-5 (P is then rounded to bf16, 2^-9); x < -125
+// gives about 2^-125 (2.4e-38) in place of a smaller value.  The clamp keeps
+// the exponent field of the result at 1 or more: p(f) can fall just below 1,
+// and 2^-126 scaling would then produce a denormal.
 //   x = j + f with j = rint(x), f in [-1/2, 1/2]: adding 1.5 * 2^23 leaves j
 //   in the low mantissa bits of the sum, and subtracting it back gives j
 //   exactly; 2^f is the degree-3 polynomial of minimax relative error on
@@ -44,7 +46,7 @@ constexpr int kLatRows = 128; // latent rows per tcgen05 MMA (M = 128, cta_group
 //   left by 23 are j << 23, the constant's bits shift out).
 __device__ __forceinline__ float exp2_poly3(float x) {
   constexpr float kRound = 12582912.f;  // 1.5 * 2^23
-  const float xc = fmaxf(x, -126.f);
+  const float xc = fmaxf(x, -125.f);
   const float r = __fadd_rn(xc, kRound);
   const float f = __fadd_rn(xc, -__fadd_rn(r, -kRound));
   float p = fmaf(0.0551716685f, f, 0.242611125f);
@@ -59,7 +61,7 @@ __device__ __forceinline__ uint64_t exp2_poly3_x2(uint64_t x) {
   constexpr float kRound = 12582912.f;  // 1.5 * 2^23
   float x0, x1;
   ptx::f2_split(x, x0, x1);
-  const uint64_t xc = ptx::f2(fmaxf(x0, -126.f), fmaxf(x1, -126.f));
+  const uint64_t xc = ptx::f2(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
   const uint64_t r = ptx::add2(xc, ptx::f2(kRound, kRound));
   const uint64_t j = ptx::add2(r, ptx::f2(-kRound, -kRound));
   const uint64_t f = ptx::fma2(j, ptx::f2(-1.f, -1.f), xc);  // xc - j, exact product, one rounding
