@@ -20,7 +20,10 @@ the data path.  Rank 0 prints one JSON line:
 * roofline: the dominant kernel (the tcgen05 encode, launched twice a step),
   timed per launch with CUDA events bracketing each launch inside a timed
   region, against the measured peaks in MEASURED_PEAKS.json;
-* cpu_baseline: the fp64 oracle on a bounded sample, on the host cores.
+* cpu_baseline: the fp64 oracle on a bounded sample, on the host cores;
+* flare_fixed_query: FLARE with the seeds as fixed latent queries (one
+  encode, one decode) on the same inputs, and the FLARE++ : FLARE step-time
+  ratio.
 
 --impl reference times the oracle (the reference arm of this comparison) on
 the host cores, rank 0 only, and prints the same line with "impl": "reference".
@@ -59,7 +62,10 @@ def parse():
 
 
 def dist_env():
-    return int(os.environ.get("RANK", 0)), int(os.environ.get("WORLD_SIZE", 1)), int(os.environ.get("LOCAL_RANK", 0))
+    from rank_latent_attention_b200.ranks import RankEnv
+
+    e = RankEnv.from_environ()
+    return e.rank, e.world, e.local
 
 
 # DRAM bytes (read + write) per full-size launch of the encode, from one
@@ -228,25 +234,24 @@ def run_native(args):
     import torch.distributed as dist
 
     import rank_latent_attention_b200 as flare
-    from rank_latent_attention_b200 import inputs
+    from rank_latent_attention_b200 import inputs, ranks
 
-    rank, world, local = dist_env()
+    env = ranks.RankEnv.from_environ()
+    rank, world, local = env.rank, env.world, env.local
     torch.cuda.set_device(local)
     if world > 1:
         dist.init_process_group("nccl", timeout=__import__("datetime").timedelta(seconds=120),
                                 device_id=torch.device("cuda", local))
     flare.lib()
 
-    base = inputs.WORKLOADS[WORKLOAD]
-    H = args.heads or base.H
-    w = inputs.Workload(base.name, world, H, base.N, base.M, base.D, base.dtype, base.kind, base.index)
-    # this rank's cloud: batch element b = rank of the world-sized batch
+    w = ranks.rank_workload(inputs.WORKLOADS[WORKLOAD], world, args.heads)
+    b = ranks.rank_batch_element(env)  # this rank's cloud of the world-sized batch
     seeds = inputs.make_seeds(w)
     Kh = np.empty((1, w.H, w.N, w.D), dtype=np.float32)
     Vh = np.empty_like(Kh)
     import concurrent.futures as fut
     with fut.ThreadPoolExecutor(min(16, os.cpu_count() or 1)) as ex:
-        for h, (k, v) in enumerate(ex.map(lambda h: inputs.make_head(w, rank, h), range(w.H))):
+        for h, (k, v) in enumerate(ex.map(lambda h: inputs.make_head(w, b, h), range(w.H))):
             Kh[0, h], Vh[0, h] = k, v
     s_h = torch.from_numpy(seeds).to(torch.bfloat16).pin_memory()
     K_h = torch.from_numpy(Kh).to(torch.bfloat16).pin_memory()
@@ -267,11 +272,7 @@ def run_native(args):
         torch.cuda.synchronize()
 
     def max_over_ranks(x):
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return ranks.max_over_ranks(x, env, dev)
 
     for _ in range(args.warmup):
         step()
@@ -309,6 +310,29 @@ def run_native(args):
     enc_ms = max_over_ranks(statistics.mean(per_kernel["encode_tc"]))
     dec_ms = max_over_ranks(statistics.mean(per_kernel["decode_tc"]))
 
+    # ---- FLARE with fixed (learned) latent queries on the same inputs: one
+    # encode with the seeds as queries, one decode; same timing discipline
+    Zf = torch.empty((1, w.H, w.M, w.D), dtype=torch.bfloat16, device=dev)
+    wsf = torch.empty(flare.flare_encode_workspace_size(1, w.H, w.N, w.M, w.D, 1), dtype=torch.uint8, device=dev)
+
+    def flare_step():
+        flare.flare_encode(s_d, K_d, V_d, Zf, workspace=wsf)
+        flare.flare_decode(K_d, s_d, Zf, Y_d)
+
+    nf = max(1, min(args.steps, 100))
+    for _ in range(3):
+        flare_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(nf):
+        flare_step()
+    ev1.record(stream)
+    barrier()
+    flare_ms = max_over_ranks(ev0.elapsed_time(ev1)) / nf
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after the fixed-query FLARE steps: {st}")
+
     # ---- end to end: pinned host inputs, copies inside the timed region
     Y_host = torch.empty(K_h.shape, dtype=torch.bfloat16).pin_memory()
     ne = max(1, min(args.e2e_steps, args.steps))
@@ -334,12 +358,11 @@ def run_native(args):
 
     if world > 1:
         dist.destroy_process_group()
-    if rank != 0:
+    if not ranks.reports(env):
         return
 
     peaks, peak_kind = measured_peaks()
-    tokens = world * w.N  # B = 1 per rank
-    value = tokens / (ms * 1e-3)
+    value = ranks.job_tokens_per_s(w.N, env, ms)  # B = 1 per rank
     flops_step = 12.0 * w.N * w.M * w.D * w.H * world
     bytes_step = 12.0 * w.N * w.D * w.H * world  # K,V + K,V + K + Y, bf16
     # every number here is timed inside a long run of steps: the sustained
@@ -378,7 +401,7 @@ def run_native(args):
         "vs_baseline": None,
         "dtype": "bf16",
         "data": "synthetic",
-        "config": {"workload": WORKLOAD if w.H == base.H else f"{WORKLOAD}-{w.H}heads", "B_per_gpu": 1, "global_batch": world, "H": w.H, "N": w.N, "M": w.M,
+        "config": {"workload": WORKLOAD if w.H == inputs.WORKLOADS[WORKLOAD].H else f"{WORKLOAD}-{w.H}heads", "B_per_gpu": 1, "global_batch": world, "H": w.H, "N": w.N, "M": w.M,
                    "D": w.D, "parallelism": f"batch-sharded x{world}, no collectives",
                    "l2": "inputs (4.3 GB K/V per step) larger than L2; no flush"},
         "tflops": flops_step / (ms * 1e-3) / 1e12,
@@ -389,7 +412,9 @@ def run_native(args):
         "decode_ms_per_launch": dec_ms,
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks.summary(),
-        "e2e": {"value": tokens / (e2e_ms * 1e-3), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+        "flare_fixed_query": {"ms_per_step": flare_ms, "tokens_per_s": ranks.job_tokens_per_s(w.N, env, flare_ms),
+                              "flarepp_over_flare": ms / flare_ms, "steps": nf},
+        "e2e": {"value": ranks.job_tokens_per_s(w.N, env, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ne},
     }
     if world == 1 and not args.no_cpu_baseline:
