@@ -29,8 +29,8 @@
 //
 // The issuer warps run their loop as a whole and issue under elect.sync,
 // which keeps the MMA operands warp-uniform.  The softmax arithmetic runs on
-// packed fp32 pairs (f32x2), and 5 of every 16 column pairs take their
-// exponentials from exp2_poly3 (FMA pipe) instead of MUFU.
+// packed fp32 pairs (f32x2); the column pairs in kDecPolyPairs would take
+// their exponentials from exp2_poly3 (FMA pipe) instead of MUFU.
 //
 // TMEM: slot s owns columns [256 s, 256 s + 256): S at [0, MP); P of group 0
 // at [0, MP / 4) (latent pairs in order, written over scores already read);
@@ -56,8 +56,9 @@ struct DecodeArgs {
 };
 
 // Column pairs (bit j: pair j of each 16) whose exponentials go to
-// exp2_poly3 in the decode softmax.
-constexpr uint32_t kDecPolyPairs = 0x2491u;
+// exp2_poly3 in the decode softmax: none, as in the encode (measured
+// faster with every exponential on MUFU).
+constexpr uint32_t kDecPolyPairs = 0x0000u;
 
 template <int D, int MP, int NS>
 struct DecodeCfg {
