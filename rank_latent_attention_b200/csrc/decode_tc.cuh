@@ -56,8 +56,8 @@ struct DecodeArgs {
 };
 
 // Column pairs (bit j: pair j of each 16) whose exponentials go to
-// exp2_poly3 in the decode softmax: none, as in the encode (measured
-// faster with every exponential on MUFU).
+// exp2_poly3 in the decode softmax: none (A/B measured: 1/16 makes no
+// difference, 2/16 is slower, 5/16 much slower).
 constexpr uint32_t kDecPolyPairs = 0x0000u;
 
 template <int D, int MP, int NS>

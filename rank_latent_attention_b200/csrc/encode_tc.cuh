@@ -50,8 +50,7 @@
 // a tile's max exceeds it by more than 2^8, so the O rescale in tensor memory
 // is rare.  Any reference gives the same normalised result because P and l
 // use the same one.  Of every 16 column pairs, those in kEncPolyPairs take
-// their exponentials from exp2_poly3 (FMA pipe) instead of MUFU (none at
-// present, see kEncPolyPairs).
+// their exponentials from exp2_poly3 (FMA pipe) instead of MUFU.
 //
 // Epilogue: each CTA writes one partial per head (O_part[split] etc.), the
 // accumulators that cover the same latent rows folded with their weights
@@ -84,12 +83,13 @@ struct EncodeArgs {
 __host__ __device__ constexpr int encode_partials_per_split(int /*D*/, int /*nhalf*/) { return 1; }
 
 // Column pairs (bit j: pair j of each 16) whose exponentials go to
-// exp2_poly3 instead of MUFU.  None: with every exponential on MUFU the
-// million-token step measured 4.84 ms against 5.23-5.33 ms with 5 pairs of
-// 16 on the polynomial; in these kernels the polynomial's extra FMA/ALU
-// instructions cost more issue slots (and power, the kernels run
+// exp2_poly3 instead of MUFU: pair 0, 1/16 of the tile.  Measured A/B on the
+// million-token workload (same GPU, builds alternating): 1/16 on the
+// polynomial is 6-7% faster than none, 2/16 and 3/16 sit between, and 5/16
+// is slower than none: past a small share the polynomial's extra FMA/ALU
+// instructions cost more issue slots (and power; the kernels run
 // power-capped) than the MUFU time they free.
-constexpr uint32_t kEncPolyPairs = 0x0000u;
+constexpr uint32_t kEncPolyPairs = 0x0001u;
 
 template <int D, int NHALF, int NS>
 struct EncodeCfg {
