@@ -333,6 +333,28 @@ def run_native(args):
     if st != (0, 0):
         raise RuntimeError(f"device status after the fixed-query FLARE steps: {st}")
 
+    # ---- communication matrix of the routing (C = W_enc W_dec per head, M x M)
+    # with the step's routing queries Q_dyn, the spectral-analysis tool
+    Yd, Qd, Zd = flare.flarepp_mix_debug(s_d, K_d, V_d)
+    del Yd, Zd
+    wsc = torch.empty(flare.lib().flare_communication_workspace_size(1, w.H, w.N, w.M, w.D, 1), dtype=torch.uint8,
+                      device=dev)
+    Cm = torch.empty((1, w.H, w.M, w.M), dtype=torch.bfloat16, device=dev)
+    flare.flare_communication_matrix(Qd, K_d, Cm, workspace=wsc)
+    comm_launches = flare.flare_last_launch_count()
+    nc = 3
+    barrier()
+    ev0.record(stream)
+    for _ in range(nc):
+        flare.flare_communication_matrix(Qd, K_d, Cm, workspace=wsc)
+    ev1.record(stream)
+    barrier()
+    comm_ms = max_over_ranks(ev0.elapsed_time(ev1)) / nc
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after the communication matrix: {st}")
+    del wsc, Cm, Qd
+
     # ---- end to end: pinned host inputs, copies inside the timed region
     Y_host = torch.empty(K_h.shape, dtype=torch.bfloat16).pin_memory()
     ne = max(1, min(args.e2e_steps, args.steps))
@@ -414,6 +436,8 @@ def run_native(args):
         "clocks": clocks.summary(),
         "flare_fixed_query": {"ms_per_step": flare_ms, "tokens_per_s": ranks.job_tokens_per_s(w.N, env, flare_ms),
                               "flarepp_over_flare": ms / flare_ms, "steps": nf},
+        "communication_matrix": {"ms_per_call": comm_ms, "launches": comm_launches,
+                                 "what": "C = softmax_N(Q_dyn K^T) softmax_M(K Q_dyn^T), M x M per head"},
         "e2e": {"value": ranks.job_tokens_per_s(w.N, env, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ne},
     }

@@ -151,6 +151,33 @@ int flare_last_launch_count(void);
 int flare_set_split_override(int splits);
 int flare_set_wait_limit_ms(int ms);
 
+/*
+ * Communication matrix of the latent routing, per head (b, h):
+ *   C = W_enc W_dec   (M x M),  W_enc = softmax_N(Q K^T) (M x N, over tokens),
+ *                                W_dec = softmax_M(K Q^T) (N x M, over latents),
+ * scale 1.  The token-to-token matrix W = W_dec W_enc (N x N, "FLARE: Fast
+ * Low-rank Attention Routing Engine" review page, section "Матрица
+ * коммуникации низкого ранга") has rank at most M, and its nonzero
+ * eigenvalues are those of C (same page, section "Спектральный анализ": the
+ * spectrum in O(M^3 + M^2 N)); C is row-stochastic, so its leading
+ * eigenvalue is 1.  For FLARE++ pass the routing queries Q_dyn as Q
+ * (q_batched = 1).
+ *
+ * Q: [H][M][D] (q_batched = 0) or [B][H][M][D]; K: [B][H][N][D]; C:
+ * [B][H][M][M], in the storage type of dtype (FLARE_F32: fp32 throughout on
+ * CUDA cores; FLARE_BF16: bf16 inputs and C, tensor-core steps).  All
+ * pointers are device memory owned by the caller, 16-byte aligned.
+ * Computed with the library's own decode and encode: ceil(M / D) rounds of a
+ * decode with Z = D columns of the M x M identity (giving those columns of
+ * W_dec) and an encode with that block as V.  workspace: at least
+ * flare_communication_workspace_size() bytes (it holds one N x D block of
+ * W_dec per head), or NULL to allocate on the stream.  Errors as for
+ * flare_encode; FLARE_BF16_F32OUT is FLARE_ERR_UNSUPPORTED.
+ */
+size_t flare_communication_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+int flare_communication_matrix(const void* Q, int q_batched, const void* K, void* C, int B, int H, int64_t N, int M,
+                               int D, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
 /* Kernel kinds reported by the launch profiler. */
 typedef enum {
   FLARE_KERNEL_ENCODE_TC = 1,   /* split-token tcgen05 encode (partials) */

@@ -29,6 +29,8 @@ __all__ = [
     "flarepp_mix_debug",
     "flare_encode_workspace_size",
     "flarepp_workspace_size",
+    "flare_communication_matrix",
+    "flare_communication_eigenvalues",
     "flare_check_status",
     "flare_last_launch_count",
     "flare_set_split_override",
@@ -57,6 +59,8 @@ _SIGNATURES = {
     "flare_check_status": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
     "flare_status_string": (ctypes.c_char_p, [_c_int]),
     "flare_last_launch_count": (_c_int, []),
+    "flare_communication_workspace_size": (_c_size, _SIZES),
+    "flare_communication_matrix": (_c_int, [_vp, _c_int, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_set_split_override": (_c_int, [_c_int]),
     "flare_set_wait_limit_ms": (_c_int, [_c_int]),
     "flare_profile_begin": (_c_int, [_c_int]),
@@ -178,6 +182,37 @@ def flare_decode(K, Q, Z, Y=None, *, stream=None):
                               _ptr(Y, "Y", K.dtype), B, H, N, M, D, _dtype_code(K), _stream(stream)),
            "flare_decode")
     return Y
+
+
+def flare_communication_matrix(Q, K, C=None, *, workspace=None, stream=None):
+    """C = softmax_N(Q K^T) softmax_M(K Q^T) per head: [B,H,M,M], row-stochastic.
+
+    Its eigenvalues are the nonzero eigenvalues of the rank-M token-to-token
+    communication matrix W = W_dec W_enc.  Q is [H,M,D] (shared) or
+    [B,H,M,D] (e.g. FLARE++'s routing queries Q_dyn)."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    q_batched = 1 if Q.dim() == 4 else 0
+    M = Q.shape[-2]
+    if C is None:
+        C = torch.empty((B, H, M, M), dtype=K.dtype, device=K.device)
+    ws, wsb = _ws(workspace)
+    _check(lib().flare_communication_matrix(_ptr(Q, "Q", K.dtype), q_batched, _ptr(K, "K", K.dtype),
+                                            _ptr(C, "C", K.dtype), B, H, N, M, D, _dtype_code(K), ws, wsb,
+                                            _stream(stream)), "flare_communication_matrix")
+    return C
+
+
+def flare_communication_eigenvalues(Q, K, *, stream=None):
+    """Eigenvalues of each head's communication matrix, [B,H,M] complex128,
+    sorted by decreasing modulus.  The O(M^2 N) product C runs in the
+    library's kernels; the O(M^3) eigen-solve of the M x M matrices is a
+    LAPACK call on the host (torch.linalg.eigvals in float64)."""
+    torch = _torch()
+    C = flare_communication_matrix(Q, K, stream=stream)
+    ev = torch.linalg.eigvals(C.to("cpu", torch.float64))
+    order = torch.argsort(ev.abs(), dim=-1, descending=True)
+    return torch.gather(ev, -1, order)
 
 
 def _mix_mode(K, out_dtype):

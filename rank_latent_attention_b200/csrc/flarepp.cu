@@ -444,6 +444,79 @@ int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_
 
 using namespace flare;
 
+// ------------------------------------------------------------------ communication matrix
+// C = W_enc W_dec (M x M per head) from the existing steps: a decode with
+// Z = columns [j D, j D + D) of the M x M identity gives those columns of
+// W_dec = softmax_M(K Q^T) (N x M), and an encode with that block as V gives
+// the same columns of C = softmax_N(Q K^T) W_dec.
+template <typename T>
+__device__ __forceinline__ T from_float(float v);
+template <>
+__device__ __forceinline__ float from_float<float>(float v) { return v; }
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_float<__nv_bfloat16>(float v) { return __float2bfloat16_rn(v); }
+
+// Zid[bh][m][d] = 1 if m == j D + d, else 0.
+template <typename T>
+__global__ void identity_block_kernel(T* Z, size_t total, int M, int D, int j) {
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int d = static_cast<int>(idx % D);
+  const int m = static_cast<int>((idx / D) % M);
+  Z[idx] = from_float<T>(m == j * D + d ? 1.f : 0.f);
+}
+
+// C[bh][m][j D + d] = Cb[bh][m][d] for the columns inside [0, M).
+template <typename T>
+__global__ void scatter_block_kernel(const T* Cb, T* C, size_t total, int M, int D, int j) {
+  const size_t idx = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (idx >= total) return;
+  const int d = static_cast<int>(idx % D);
+  const size_t row = idx / D;  // bh * M + m
+  const int col = j * D + d;
+  if (col < M) C[row * M + col] = Cb[idx];
+}
+
+struct CommWs {
+  size_t enc, zid, y, cb, bytes;
+};
+
+CommWs comm_ws_layout(int B, int H, int64_t N, int M, int D, int dtype) {
+  const int BH = B * H;
+  const size_t es = elem_size(dtype);
+  CommWs w;
+  w.enc = encode_ws_layout(nullptr, BH, N, M, D, dtype).bytes;
+  w.zid = align256(static_cast<size_t>(BH) * M * D * es);
+  w.y = align256(static_cast<size_t>(BH) * N * D * es);
+  w.cb = align256(static_cast<size_t>(BH) * M * D * es);
+  w.bytes = w.enc + w.zid + w.y + w.cb;
+  return w;
+}
+
+template <typename T>
+int run_comm(const void* Q, int q_batched, const void* K, void* C, int B, int H, int64_t N, int M, int D, int dtype,
+             char* ws, cudaStream_t st, int* launches) {
+  const int BH = B * H;
+  const CommWs w = comm_ws_layout(B, H, N, M, D, dtype);
+  T* Zid = reinterpret_cast<T*>(ws + w.enc);
+  T* Yj = reinterpret_cast<T*>(ws + w.enc + w.zid);
+  T* Cb = reinterpret_cast<T*>(ws + w.enc + w.zid + w.y);
+  const size_t blk = static_cast<size_t>(BH) * M * D;
+  const unsigned grid = static_cast<unsigned>((blk + 255) / 256);
+  for (int j = 0; j * D < M; ++j) {
+    identity_block_kernel<T><<<grid, 256, 0, st>>>(Zid, blk, M, D, j);
+    if (cudaGetLastError() != cudaSuccess) return FLARE_ERR_CUDA;
+    ++*launches;
+    int rc = run_decode(K, Q, q_batched, Zid, Yj, B, H, N, M, D, dtype, st, launches);
+    if (!rc) rc = run_encode(Q, q_batched, K, Yj, Cb, B, H, N, M, D, dtype, ws, st, launches);
+    if (rc) return rc;
+    scatter_block_kernel<T><<<grid, 256, 0, st>>>(Cb, static_cast<T*>(C), blk, M, D, j);
+    if (cudaGetLastError() != cudaSuccess) return FLARE_ERR_CUDA;
+    ++*launches;
+  }
+  return FLARE_OK;
+}
+
 extern "C" {
 
 size_t flare_encode_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
@@ -500,6 +573,34 @@ int flarepp_mix_debug(const void* seeds, const void* K, const void* V, void* Y, 
                       int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
   if (!Q_dyn || !Z) return FLARE_ERR_INVALID_ARG;
   return mix_impl(seeds, K, V, Y, Q_dyn, Z, B, H, N, M, D, dtype, workspace, workspace_bytes, stream);
+}
+
+size_t flare_communication_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (check_sizes(B, H, N, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
+  return comm_ws_layout(B, H, N, M, D, dtype).bytes;
+}
+
+int flare_communication_matrix(const void* Q, int q_batched, const void* K, void* C, int B, int H, int64_t N, int M,
+                               int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
+  if (!device_ptr(Q) || !device_ptr(K) || !device_ptr(C)) return FLARE_ERR_INVALID_ARG;
+  if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch s;
+  rc = get_scratch(workspace, workspace_bytes, comm_ws_layout(B, H, N, M, D, dtype).bytes, st, &s);
+  if (rc) return rc;
+  int launches = 0;
+  rc = dtype == FLARE_BF16 ? run_comm<__nv_bfloat16>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches)
+                           : run_comm<float>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  const int rc2 = release_scratch(s, st);
+  if (!rc) {
+    rc = rc2;
+    t_last_launches = launches;
+  }
+  return rc;
 }
 
 int flare_check_status(void* stream, int* site) {
