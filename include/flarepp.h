@@ -126,6 +126,26 @@ int flarepp_mix_debug(const void* seeds, const void* K, const void* V, void* Y, 
                       int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream);
 
 /*
+ * flarepp_mix_host: flarepp_mix with seeds, K, V and Y in HOST memory (same
+ * layouts and dtypes; page-locked memory lets the copies run asynchronously,
+ * pageable memory works but its copies stage through the driver).  The
+ * (b, h) heads are independent ("FLARE++" page, "Méthodologie : FLARE++":
+ * each head routes only its own tokens), so the call streams them through the
+ * GPU one head at a time: the copy of head c + 1 in, the mix of head c and the
+ * copy of head c - 1 out overlap on two library-owned copy streams and the
+ * caller's stream, using both directions of the host link at once.  Returns
+ * once everything is enqueued; when `stream` has completed, Y holds the
+ * result.  workspace: device memory of at least
+ * flarepp_mix_host_workspace_size() bytes (two heads' K, V and Y, the seeds
+ * and one head's mix workspace), or NULL to allocate on `stream`.  Calls are
+ * serialised within a process while they enqueue.  Errors as for flarepp_mix;
+ * a device pointer where host memory is expected is FLARE_ERR_INVALID_ARG.
+ */
+size_t flarepp_mix_host_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+int flarepp_mix_host(const void* seeds, const void* K, const void* V, void* Y, int B, int H, int64_t N, int M, int D,
+                     int dtype, void* workspace, size_t workspace_bytes, void* stream);
+
+/*
  * Synchronises `stream`, then reads and clears the current device's status
  * word.  Returns FLARE_OK or the first error a kernel recorded since the last
  * check (FLARE_ERR_TIMEOUT); *site (if not NULL) receives the kernel role

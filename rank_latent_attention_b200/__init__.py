@@ -29,6 +29,7 @@ __all__ = [
     "flarepp_mix_debug",
     "flare_encode_workspace_size",
     "flarepp_workspace_size",
+    "flarepp_mix_host",
     "flare_communication_matrix",
     "flare_communication_eigenvalues",
     "flare_check_status",
@@ -59,6 +60,8 @@ _SIGNATURES = {
     "flare_check_status": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
     "flare_status_string": (ctypes.c_char_p, [_c_int]),
     "flare_last_launch_count": (_c_int, []),
+    "flarepp_mix_host_workspace_size": (_c_size, _SIZES),
+    "flarepp_mix_host": (_c_int, [_vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_communication_workspace_size": (_c_size, _SIZES),
     "flare_communication_matrix": (_c_int, [_vp, _c_int, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_set_split_override": (_c_int, [_c_int]),
@@ -181,6 +184,28 @@ def flare_decode(K, Q, Z, Y=None, *, stream=None):
     _check(lib().flare_decode(_ptr(K, "K", K.dtype), _ptr(Q, "Q", K.dtype), q_batched, _ptr(Z, "Z", K.dtype),
                               _ptr(Y, "Y", K.dtype), B, H, N, M, D, _dtype_code(K), _stream(stream)),
            "flare_decode")
+    return Y
+
+
+def flarepp_mix_host(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, stream=None):
+    """flarepp_mix with seeds, K, V and Y in host memory (CPU tensors; pin
+    them for asynchronous copies).  The library streams the heads through
+    the GPU, overlapping copies in, compute and copies out; Y is complete
+    once `stream` (default: the current CUDA stream) has completed."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = seeds.shape[-2]
+    code, ydt = _mix_mode(K, out_dtype)
+    for name, t in (("seeds", seeds), ("K", K), ("V", V)):
+        if t.device.type != "cpu" or not t.is_contiguous():
+            raise ValueError(f"{name} must be a contiguous CPU tensor")
+    if Y is None:
+        Y = torch.empty((B, H, N, D), dtype=ydt, pin_memory=K.is_pinned())
+    if Y.device.type != "cpu" or not Y.is_contiguous() or Y.dtype != ydt:
+        raise ValueError("Y must be a contiguous CPU tensor of the output dtype")
+    ws, wsb = _ws(workspace)
+    _check(lib().flarepp_mix_host(seeds.data_ptr(), K.data_ptr(), V.data_ptr(), Y.data_ptr(), B, H, N, M, D, code,
+                                  ws, wsb, _stream(stream)), "flarepp_mix_host")
     return Y
 
 

@@ -517,6 +517,65 @@ int run_comm(const void* Q, int q_batched, const void* K, void* C, int B, int H,
   return FLARE_OK;
 }
 
+// ------------------------------------------------------------------ host-resident inputs
+// flarepp_mix_host streams (b, h) chunks through the GPU: the copy of chunk
+// c + 1 in, the mix of chunk c and the copy of chunk c - 1 out run at once on
+// two copy streams and the caller's stream, with two device slots per chunk
+// buffer.  One stream pair and one set of events per device, created once;
+// calls are serialised by a mutex while they enqueue.
+struct HostPipe {
+  bool ready = false;
+  cudaStream_t in = nullptr, out = nullptr;
+  cudaEvent_t ev_in[2], ev_comp[2], ev_out[2], ev_seeds;
+};
+
+std::mutex g_pipe_mu;
+
+HostPipe* host_pipe() {
+  static HostPipe pipes[64];
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  HostPipe& p = pipes[dev];
+  if (!p.ready) {
+    if (cudaStreamCreateWithFlags(&p.in, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    if (cudaStreamCreateWithFlags(&p.out, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+    for (int i = 0; i < 2; ++i)
+      if (cudaEventCreateWithFlags(&p.ev_in[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&p.ev_comp[i], cudaEventDisableTiming) != cudaSuccess ||
+          cudaEventCreateWithFlags(&p.ev_out[i], cudaEventDisableTiming) != cudaSuccess)
+        return nullptr;
+    if (cudaEventCreateWithFlags(&p.ev_seeds, cudaEventDisableTiming) != cudaSuccess) return nullptr;
+    p.ready = true;
+  }
+  return &p;
+}
+
+struct HostWs {
+  size_t seeds, chunk_in, chunk_out, mix, bytes;
+};
+
+HostWs host_ws_layout(int H, int64_t N, int M, int D, int dtype) {
+  const size_t in_es = dtype == FLARE_F32 ? 4 : 2;
+  const size_t out_es = dtype == FLARE_BF16 ? 2 : 4;
+  HostWs w;
+  w.seeds = align256(static_cast<size_t>(H) * M * D * in_es);
+  w.chunk_in = align256(static_cast<size_t>(N) * D * in_es);
+  w.chunk_out = align256(static_cast<size_t>(N) * D * out_es);
+  w.mix = mix_ws_bytes(1, 1, N, M, D, dtype);
+  w.bytes = w.seeds + 2 * (2 * w.chunk_in + w.chunk_out) + w.mix;
+  return w;
+}
+
+bool host_ptr(const void* p) {
+  if (!p) return false;
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return true;  // not known to CUDA: pageable host memory
+  }
+  return attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeUnregistered;
+}
+
 extern "C" {
 
 size_t flare_encode_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
@@ -596,6 +655,77 @@ int flare_communication_matrix(const void* Q, int q_batched, const void* K, void
   rc = dtype == FLARE_BF16 ? run_comm<__nv_bfloat16>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches)
                            : run_comm<float>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches);
   const int rc2 = release_scratch(s, st);
+  if (!rc) {
+    rc = rc2;
+    t_last_launches = launches;
+  }
+  return rc;
+}
+
+size_t flarepp_mix_host_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (check_sizes(B, H, N, M, D, dtype)) return 0;
+  return host_ws_layout(H, N, M, D, dtype).bytes;
+}
+
+int flarepp_mix_host(const void* seeds, const void* K, const void* V, void* Y, int B, int H, int64_t N, int M, int D,
+                     int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (!host_ptr(seeds) || !host_ptr(K) || !host_ptr(V) || !host_ptr(Y)) return FLARE_ERR_INVALID_ARG;
+  if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
+  std::lock_guard<std::mutex> lock(g_pipe_mu);
+  HostPipe* pipe = host_pipe();
+  if (!pipe) return FLARE_ERR_CUDA;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const HostWs w = host_ws_layout(H, N, M, D, dtype);
+  Scratch s;
+  rc = get_scratch(workspace, workspace_bytes, w.bytes, st, &s);
+  if (rc) return rc;
+  // the copy streams start after the caller's earlier work (workspace reuse)
+  auto ok = [](cudaError_t e) { return e == cudaSuccess; };
+  bool good = ok(cudaEventRecord(pipe->ev_seeds, st)) && ok(cudaStreamWaitEvent(pipe->in, pipe->ev_seeds, 0)) &&
+              ok(cudaStreamWaitEvent(pipe->out, pipe->ev_seeds, 0));
+  const size_t in_es = dtype == FLARE_F32 ? 4 : 2;
+  const size_t out_es = dtype == FLARE_BF16 ? 2 : 4;
+  const size_t in_bytes = static_cast<size_t>(N) * D * in_es, out_bytes = static_cast<size_t>(N) * D * out_es;
+  char* seeds_d = s.ptr;
+  char* slot_base[2] = {s.ptr + w.seeds, s.ptr + w.seeds + 2 * w.chunk_in + w.chunk_out};
+  char* mix_ws = s.ptr + w.seeds + 2 * (2 * w.chunk_in + w.chunk_out);
+  good = good && ok(cudaMemcpyAsync(seeds_d, seeds, static_cast<size_t>(H) * M * D * in_es, cudaMemcpyHostToDevice,
+                                    pipe->in)) &&
+         ok(cudaEventRecord(pipe->ev_seeds, pipe->in)) && ok(cudaStreamWaitEvent(st, pipe->ev_seeds, 0));
+  int launches = 0;
+  const int chunks = B * H;
+  for (int c = 0; good && !rc && c < chunks; ++c) {
+    const int sl = c & 1, h = c % H;
+    char* Kd = slot_base[sl];
+    char* Vd = Kd + w.chunk_in;
+    char* Yd = Vd + w.chunk_in;
+    const char* Kh = static_cast<const char*>(K) + static_cast<size_t>(c) * in_bytes;
+    const char* Vh = static_cast<const char*>(V) + static_cast<size_t>(c) * in_bytes;
+    char* Yh = static_cast<char*>(Y) + static_cast<size_t>(c) * out_bytes;
+    // in: once the mix of chunk c - 2 has read this slot
+    if (c >= 2) good = ok(cudaStreamWaitEvent(pipe->in, pipe->ev_comp[sl], 0));
+    good = good && ok(cudaMemcpyAsync(Kd, Kh, in_bytes, cudaMemcpyHostToDevice, pipe->in)) &&
+           ok(cudaMemcpyAsync(Vd, Vh, in_bytes, cudaMemcpyHostToDevice, pipe->in)) &&
+           ok(cudaEventRecord(pipe->ev_in[sl], pipe->in));
+    // mix: once the inputs are in and Y of chunk c - 2 has left this slot
+    good = good && ok(cudaStreamWaitEvent(st, pipe->ev_in[sl], 0)) &&
+           (c < 2 || ok(cudaStreamWaitEvent(st, pipe->ev_out[sl], 0)));
+    if (!good) break;
+    rc = mix_impl(seeds_d + static_cast<size_t>(h) * M * D * in_es, Kd, Vd, Yd, nullptr, nullptr, 1, 1, N, M, D,
+                  dtype, mix_ws, w.mix, st);
+    launches += t_last_launches;
+    // out: once the mix is done
+    good = good && !rc && ok(cudaEventRecord(pipe->ev_comp[sl], st)) &&
+           ok(cudaStreamWaitEvent(pipe->out, pipe->ev_comp[sl], 0)) &&
+           ok(cudaMemcpyAsync(Yh, Yd, out_bytes, cudaMemcpyDeviceToHost, pipe->out)) &&
+           ok(cudaEventRecord(pipe->ev_out[sl], pipe->out));
+  }
+  // the caller's stream completes after every copy out
+  for (int sl = 0; good && sl < 2 && sl < chunks; ++sl) good = ok(cudaStreamWaitEvent(st, pipe->ev_out[sl], 0));
+  const int rc2 = release_scratch(s, st);
+  if (!rc && !good) rc = FLARE_ERR_CUDA;
   if (!rc) {
     rc = rc2;
     t_last_launches = launches;
