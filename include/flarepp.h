@@ -107,6 +107,51 @@ int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, voi
                  int M, int D, int dtype, void* stream);
 
 /*
+ * Token-sharded (context-parallel) encode, in two calls.  The FLARE++ page
+ * ("FLARE++: Low-rank attention with dynamic attention routing", section
+ * "Contributions Clés", multi-GPU context-parallelism item) shards the input
+ * tokens over devices and exchanges only the latent outputs and the softmax
+ * statistics, never the tokens.  With shard r's logits s_mn = Q_m . K_n over
+ * its tokens n in r:
+ *   O_r[m]   = sum_{n in r} exp(s_mn) V_n / sum_{n in r} exp(s_mn)
+ *   lse_r[m] = ln sum_{n in r} exp(s_mn)
+ * and the encode over the union of the shards is exactly
+ *   out[m] = sum_r exp(lse_r[m] - L[m]) O_r[m],   L[m] = ln sum_r exp(lse_r[m]).
+ *
+ * flare_encode_lse: one shard's (O_r, lse_r).
+ *   Q          [H][M][D] (q_batched 0) or [B][H][M][D] (q_batched 1), dtype
+ *   K, V       [B][H][N][D] this shard's tokens, dtype; may be NULL when N == 0
+ *   O          [B][H][M][D] fp32 output, whatever dtype is
+ *   lse        [B][H][M] fp32 output (natural log); needs 4-byte alignment only
+ *   N          the shard's token count, N >= 0.  N == 0 (an empty shard)
+ *              writes O = 0 and lse = -inf, which carry no weight when combined.
+ * dtype FLARE_BF16 or FLARE_F32 (the inputs' type and the arithmetic as in
+ * flare_encode); workspace as flare_encode (flare_encode_lse_workspace_size;
+ * 0 bytes for N == 0).
+ *
+ * flare_lse_combine: the exact combination of R shards' results.
+ *   O_parts    R arrays [B][H][M][D] fp32 (one flare_encode_lse output per
+ *              shard, in any order: it changes only the rounding)
+ *   lse_parts  R arrays [B][H][M] fp32 (4-byte alignment)
+ *   part_stride  floats from shard r's arrays to shard r+1's, the same for
+ *              O_parts and lse_parts; 0 = dense stacks [R][B][H][M][D] and
+ *              [R][B][H][M].  With one buffer of R rows [O_r | lse_r] (what
+ *              one all-gather of each device's [O | lse] returns), pass
+ *              O_parts = buf, lse_parts = buf + B*H*M*D and
+ *              part_stride = B*H*M*(D+1).
+ *   out        [B][H][M][D] output, dtype (FLARE_BF16: rounded to nearest)
+ *   lse_out    [B][H][M] fp32 output L, or NULL
+ * A latent whose shards are all empty gets out = 0 and L = -inf.  One kernel;
+ * no workspace.  Sizes as flare_encode with N = 1.
+ */
+size_t flare_encode_lse_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+int flare_encode_lse(const void* Q, int q_batched, const void* K, const void* V, float* O, float* lse, int B,
+                     int H, int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes,
+                     void* stream);
+int flare_lse_combine(const float* O_parts, const float* lse_parts, int R, int64_t part_stride, void* out,
+                      float* lse_out, int B, int H, int M, int D, int dtype, void* stream);
+
+/*
  * FLARE++ mixer forward: seed encode -> routing encode -> decode (see top).
  *   seeds      [H][M][D]
  *   K, V       [B][H][N][D]

@@ -21,6 +21,11 @@ Sources (page title, section):
   W_decode = softmax(K Q^T) (NxM, normalised over latents) and
   Y = (W_decode W_encode) V with W of rank at most M.
 * "FLARE++: Low-rank attention with dynamic attention routing", section
+  "Contributions Clés", multi-GPU context-parallelism item: the tokens are
+  sharded over devices, each device encodes its own shard, and only the
+  latent outputs and the softmax statistics cross devices
+  (``encode_shard`` / ``combine_shards``).
+* same page, section
   "Méthodologie : FLARE++": learned seeds Q~_h drive one extra encode call
   whose M outputs become the routing queries Q_h(X) (dynamic query
   synthesis), which then replace the learned queries in FLARE's encode-decode
@@ -54,6 +59,8 @@ __all__ = [
     "flarepp_decode_rows",
     "communication_matrix",
     "communication_eigenvalues",
+    "encode_shard",
+    "combine_shards",
 ]
 
 
@@ -155,3 +162,48 @@ def communication_eigenvalues(Q: np.ndarray, K: np.ndarray) -> np.ndarray:
     W_dec = attention_weights(K, Q)
     ev = np.linalg.eigvals(W_enc @ W_dec)
     return ev[np.argsort(-np.abs(ev))]
+
+
+def encode_shard(Q: np.ndarray, K: np.ndarray, V: np.ndarray):
+    """One token shard's encode: (O, lse), O MxD, lse length M.
+
+    ``FLARE++`` page, "Contributions Clés", multi-GPU context parallelism:
+    a device holds only its shard of the tokens and sends out only latent
+    outputs and softmax statistics.  With the shard's logits s_mn = Q_m . K_n:
+    O[m] = softmax over the shard's tokens of s_m., applied to V (the
+    shard-local encode) and lse[m] = log sum_n exp(s_mn).  A shard without
+    tokens has O = 0 and lse = -inf.
+    """
+    Q = np.asarray(Q, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    M, D = Q.shape[0], V.shape[1]
+    if K.shape[0] == 0:
+        return np.zeros((M, D)), np.full(M, -np.inf)
+    S = Q @ K.T
+    top = S.max(axis=1, keepdims=True)
+    E = np.exp(S - top)
+    tot = E.sum(axis=1)
+    return (E @ V) / tot[:, None], top[:, 0] + np.log(tot)
+
+
+def combine_shards(O_parts, lse_parts):
+    """The encode over the union of disjoint token shards from their (O, lse).
+
+    Token n of shard r has full-softmax weight exp(s_mn - L_m) =
+    exp(s_mn - lse_r[m]) * exp(lse_r[m] - L_m), with L = log sum_r exp(lse_r),
+    so out[m] = sum_r exp(lse_r[m] - L_m) O_r[m].  Returns (out, L); latents
+    whose shards are all empty get out = 0 and L = -inf.
+    """
+    lse = np.stack([np.asarray(x, dtype=np.float64) for x in lse_parts])  # R x M
+    O = np.stack([np.asarray(x, dtype=np.float64) for x in O_parts])  # R x M x D
+    top = lse.max(axis=0)
+    live = np.isfinite(top)
+    w = np.zeros_like(lse)
+    w[:, live] = np.exp(lse[:, live] - top[live])
+    tot = w.sum(axis=0)
+    out = np.zeros(O.shape[1:])
+    out[live] = np.einsum("rm,rmd->md", w[:, live], O[:, live]) / tot[live, None]
+    L = np.full(top.shape, -np.inf)
+    L[live] = top[live] + np.log(tot[live])
+    return out, L

@@ -28,6 +28,9 @@ __all__ = [
     "flarepp_mix",
     "flarepp_mix_debug",
     "flare_encode_workspace_size",
+    "flare_encode_lse",
+    "flare_encode_lse_workspace_size",
+    "flare_lse_combine",
     "flarepp_workspace_size",
     "flarepp_mix_host",
     "flare_communication_matrix",
@@ -55,6 +58,10 @@ _SIGNATURES = {
     "flarepp_workspace_size": (_c_size, _SIZES),
     "flare_encode": (_c_int, [_vp, _c_int, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_decode": (_c_int, [_vp, _vp, _c_int, _vp, _vp, *_SIZES, _vp]),
+    "flare_encode_lse_workspace_size": (_c_size, _SIZES),
+    "flare_encode_lse": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
+    "flare_lse_combine": (_c_int, [_vp, _vp, _c_int, _c_i64, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
+                                   _vp]),
     "flarepp_mix": (_c_int, [_vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flarepp_mix_debug": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_check_status": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
@@ -185,6 +192,55 @@ def flare_decode(K, Q, Z, Y=None, *, stream=None):
                               _ptr(Y, "Y", K.dtype), B, H, N, M, D, _dtype_code(K), _stream(stream)),
            "flare_decode")
     return Y
+
+
+def flare_encode_lse_workspace_size(B, H, N, M, D, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (BF16 if "bfloat16" in str(dtype) else F32)
+    return lib().flare_encode_lse_workspace_size(B, H, N, M, D, code)
+
+
+def flare_encode_lse(Q, K, V, O=None, lse=None, *, workspace=None, stream=None):
+    """One token shard's encode: O = softmax over the shard's tokens of Q K^T,
+    times V (fp32 [B,H,M,D]), and lse = log-sum-exp of those logits (fp32
+    [B,H,M], natural log).  K and V may hold no tokens (N = 0): O = 0 and
+    lse = -inf.  Returns (O, lse)."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    q_batched = 1 if Q.dim() == 4 else 0
+    M = Q.shape[-2]
+    if O is None:
+        O = torch.empty((B, H, M, D), dtype=torch.float32, device=Q.device)
+    if lse is None:
+        lse = torch.empty((B, H, M), dtype=torch.float32, device=Q.device)
+    kv = (None, None) if N == 0 else (_ptr(K, "K", K.dtype), _ptr(V, "V", K.dtype))
+    ws, wsb = _ws(workspace)
+    _check(lib().flare_encode_lse(_ptr(Q, "Q", K.dtype), q_batched, kv[0], kv[1], _ptr(O, "O", torch.float32),
+                                  _ptr(lse, "lse", torch.float32), B, H, N, M, D, _dtype_code(K), ws, wsb,
+                                  _stream(stream)),
+           "flare_encode_lse")
+    return O, lse
+
+
+def flare_lse_combine(O_parts, lse_parts, out=None, lse_out=None, *, dtype=None, shape=None, part_stride=0,
+                      stream=None):
+    """Exact combination of R token shards' (O, lse): out = sum_r
+    exp(lse_r - L) O_r with L = log sum_r exp(lse_r).
+
+    Dense form: O_parts [R,B,H,M,D] and lse_parts [R,B,H,M] fp32.  Strided
+    form (``part_stride`` > 0, ``shape`` = (R, B, H, M, D)): O_parts and
+    lse_parts are flat fp32 tensors whose shard r starts ``r * part_stride``
+    floats in.  ``out`` [B,H,M,D] has ``dtype`` (default: out's, else
+    bfloat16); ``lse_out`` [B,H,M] fp32 is written when given."""
+    torch = _torch()
+    R, B, H, M, D = shape if shape is not None else O_parts.shape
+    if out is None:
+        out = torch.empty((B, H, M, D), dtype=dtype or torch.bfloat16, device=O_parts.device)
+    _check(lib().flare_lse_combine(_ptr(O_parts, "O_parts", torch.float32), _ptr(lse_parts, "lse_parts", torch.float32),
+                                   R, part_stride, _ptr(out, "out", out.dtype),
+                                   _ptr(lse_out, "lse_out", torch.float32), B, H, M, D, _dtype_code(out),
+                                   _stream(stream)),
+           "flare_lse_combine")
+    return out
 
 
 def flarepp_mix_host(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, stream=None):

@@ -1,0 +1,118 @@
+"""Token-sharded (context-parallel) FLARE++ mixer over torch.distributed.
+
+"FLARE++: Low-rank attention with dynamic attention routing", section
+"Contributions Clés", multi-GPU context-parallelism item: the input tokens
+are split over the devices, the encoder gathers them into latent tokens that
+every device holds a copy of, and the devices exchange only latent outputs
+and softmax statistics, never the N tokens.
+
+Per rank r, holding tokens [start_r, stop_r) of every head:
+
+1. seed encode on the local shard: (O_r, lse_r) = flare_encode_lse(seeds, K_r, V_r)
+2. one all-gather of the B*H*M*(D+1) floats [O_r | lse_r] from every rank
+3. Q_dyn = flare_lse_combine(gathered)            (identical on every rank)
+4. routing encode on the local shard, all-gather, combine -> Z
+5. decode of the local tokens: Y_r = flare_decode(K_r, Q_dyn, Z)
+
+Every rank takes the same two collectives in the same order.  The kernels are
+the library's; this module only slices, allocates and calls the collective.
+``ops`` lets the CPU tests run the same sequence with other implementations
+of the four steps (the library itself has no CPU path).
+"""
+from __future__ import annotations
+
+__all__ = ["token_range", "shard_tokens", "LibraryOps", "flarepp_mix_cp", "exchange_floats"]
+
+
+def token_range(N: int, world: int, rank: int) -> tuple[int, int]:
+    """Rank ``rank``'s contiguous token range [start, stop) of ``N`` tokens
+    over ``world`` ranks; sizes differ by at most one, and ranks past N get
+    an empty range."""
+    if not (0 <= rank < world) or N < 0:
+        raise ValueError(f"bad shard request N={N} world={world} rank={rank}")
+    return (rank * N) // world, ((rank + 1) * N) // world
+
+
+def shard_tokens(X, world: int, rank: int):
+    """This rank's tokens of X [B, H, N, D], contiguous."""
+    a, b = token_range(X.shape[2], world, rank)
+    return X[:, :, a:b].contiguous()
+
+
+def exchange_floats(B: int, H: int, M: int, D: int) -> int:
+    """Floats each rank sends per encode: O [B,H,M,D] then lse [B,H,M]."""
+    return B * H * M * (D + 1)
+
+
+def gather_rows(send, group=None):
+    """All-gather of one flat tensor per rank into [world, numel] (rank order).
+    Without an initialised process group the job is one rank."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()):
+        return send.unsqueeze(0)
+    world = dist.get_world_size(group)
+    recv = torch.empty(world * send.numel(), dtype=send.dtype, device=send.device)
+    dist.all_gather_into_tensor(recv, send, group=group)
+    return recv.view(world, send.numel())
+
+
+class LibraryOps:
+    """The GPU steps: the library's kernels and a NCCL all-gather."""
+
+    exchange_dtype = "float32"  # what flare_encode_lse writes and flare_lse_combine reads
+
+    def __init__(self, group=None):
+        self.group = group
+
+    def encode_lse(self, Q, K, V, send):
+        import rank_latent_attention_b200 as flare
+
+        B, H, _, D = K.shape
+        M = Q.shape[-2]
+        n = B * H * M * D
+        flare.flare_encode_lse(Q, K, V, O=send[:n].view(B, H, M, D), lse=send[n:].view(B, H, M))
+
+    def all_gather(self, send):
+        return gather_rows(send, self.group)
+
+    def combine(self, recv, B, H, M, D, dtype):
+        import rank_latent_attention_b200 as flare
+
+        flat = recv.view(-1)
+        n = B * H * M * D
+        return flare.flare_lse_combine(flat, flat[n:], dtype=dtype, shape=(recv.shape[0], B, H, M, D),
+                                       part_stride=recv.shape[1])
+
+    def decode(self, K, Q, Z):
+        import torch
+
+        import rank_latent_attention_b200 as flare
+
+        if K.shape[2] == 0:  # a rank without tokens has nothing to decode
+            return torch.empty_like(K)
+        return flare.flare_decode(K, Q, Z)
+
+
+def flarepp_mix_cp(seeds, K, V, *, group=None, ops=None, return_intermediates=False):
+    """FLARE++ forward of this rank's token shard.
+
+    seeds [H, M, D] (every rank the same); K, V [B, H, N_r, D]: this rank's
+    tokens (N_r may be 0).  Returns Y [B, H, N_r, D] for the local tokens,
+    and with ``return_intermediates`` also the replicated Q_dyn and Z
+    [B, H, M, D].
+    """
+    import torch
+
+    ops = ops or LibraryOps(group)
+    B, H, _, D = K.shape
+    M = seeds.shape[-2]
+    send = torch.empty(exchange_floats(B, H, M, D), dtype=getattr(torch, ops.exchange_dtype), device=K.device)
+
+    ops.encode_lse(seeds, K, V, send)
+    Q_dyn = ops.combine(ops.all_gather(send), B, H, M, D, K.dtype)
+    ops.encode_lse(Q_dyn, K, V, send)
+    Z = ops.combine(ops.all_gather(send), B, H, M, D, K.dtype)
+    Y = ops.decode(K, Q_dyn, Z)
+    return (Y, Q_dyn, Z) if return_intermediates else Y

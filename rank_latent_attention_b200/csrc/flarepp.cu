@@ -260,10 +260,15 @@ cudaError_t launch_decode_f32_d(int D, const DecodeF32Args& a, int BH, cudaStrea
   }
 }
 
+// Merge of one encode's split partials ([BH][P][M] in the workspace) into
+// `out`; lse_out (optional) receives the natural-log log-sum-exp per latent.
 template <typename T>
-cudaError_t launch_merge(const EncodeWs& w, void* out, int BH, int P, int M, int D, cudaStream_t st) {
-  lse_merge_kernel<T><<<dim3(static_cast<unsigned>(ceil_div(int64_t(M) * D, 256)), BH), 256, 0, st>>>(
-      w.O, w.m, w.l, static_cast<T*>(out), P, M, D);
+cudaError_t launch_merge(const EncodeWs& w, void* out, float* lse_out, int BH, int P, int M, int D,
+                         cudaStream_t st) {
+  const MergeGeom g{P, M, D, static_cast<long long>(P) * M * D, static_cast<long long>(M) * D,
+                    static_cast<long long>(P) * M, M};
+  lse_merge_kernel<T, false><<<dim3(static_cast<unsigned>(ceil_div(int64_t(M) * D, 256)), BH), 256, 0, st>>>(
+      w.O, w.m, w.l, static_cast<T*>(out), lse_out, g);
   return cudaGetLastError();
 }
 
@@ -271,8 +276,11 @@ cudaError_t launch_merge(const EncodeWs& w, void* out, int BH, int P, int M, int
 // One encode (partials + merge) into `out`; Q indexed per q_batched.
 // dtype FLARE_BF16: everything bf16, tensor cores.  FLARE_F32: everything
 // fp32.  FLARE_BF16_F32OUT: K, V bf16, out fp32, Q bf16 if q_bf16 else fp32.
+// lse_out: when set, `out` is fp32 whatever the dtype and the merge also
+// writes the natural-log log-sum-exp of each latent's logits ([B][H][M]).
 int run_encode(const void* Q, int q_batched, const void* K, const void* V, void* out, int B, int H, int64_t N,
-               int M, int D, int dtype, char* ws, cudaStream_t st, int* launches, bool q_bf16 = false) {
+               int M, int D, int dtype, char* ws, cudaStream_t st, int* launches, bool q_bf16 = false,
+               float* lse_out = nullptr) {
   const int BH = B * H;
   const int splits = choose_splits(BH, N, kEncTile);
   const int P = partials(M, D, splits, dtype);
@@ -306,7 +314,8 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
     ProfScope prof(FLARE_KERNEL_MERGE, st);
-    e = launch_merge<__nv_bfloat16>(w, out, BH, P, M, D, st);
+    e = lse_out ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st)
+                : launch_merge<__nv_bfloat16>(w, out, nullptr, BH, P, M, D, st);
   } else {
     EncodeF32Args a;
     a.N = static_cast<int>(N);
@@ -333,7 +342,7 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
     ProfScope prof(FLARE_KERNEL_MERGE, st);
-    e = launch_merge<float>(w, out, BH, P, M, D, st);
+    e = launch_merge<float>(w, out, lse_out, BH, P, M, D, st);
   }
   *launches += 2;
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
@@ -576,6 +585,25 @@ bool host_ptr(const void* p) {
   return attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeUnregistered;
 }
 
+// fp32 tensor in device memory with 4-byte alignment (the per-latent
+// statistics of a slice of a gathered [R][B][H][M] array need no more).
+bool device_ptr_f32(const void* p) {
+  if (!p || (reinterpret_cast<uintptr_t>(p) & 3u)) return false;
+  cudaPointerAttributes attr;
+  if (cudaPointerGetAttributes(&attr, p) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
+}
+
+// A token shard with no tokens: O = 0, lse = -inf (it then carries no weight).
+__global__ void empty_shard_kernel(float* O, float* lse, size_t rows, int D) {
+  const size_t i = static_cast<size_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i < rows * D) O[i] = 0.f;
+  if (i < rows) lse[i] = -INFINITY;
+}
+
 extern "C" {
 
 size_t flare_encode_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
@@ -608,6 +636,71 @@ int flare_encode(const void* Q, int q_batched, const void* K, const void* V, voi
     t_last_launches = launches;
   }
   return rc;
+}
+
+size_t flare_encode_lse_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (N <= 0) return 0;  // an empty shard needs none
+  if (check_sizes(B, H, N, M, D, dtype)) return 0;
+  return encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
+}
+
+int flare_encode_lse(const void* Q, int q_batched, const void* K, const void* V, float* O, float* lse, int B,
+                     int H, int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes,
+                     void* stream) {
+  if (N < 0) return FLARE_ERR_INVALID_ARG;
+  int rc = check_sizes(B, H, N == 0 ? 1 : N, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
+  if (!device_ptr(Q) || !device_ptr(O) || !device_ptr_f32(lse)) return FLARE_ERR_INVALID_ARG;
+  if (N > 0 && (!device_ptr(K) || !device_ptr(V))) return FLARE_ERR_INVALID_ARG;
+  if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (N == 0) {
+    const size_t rows = static_cast<size_t>(B) * H * M;
+    empty_shard_kernel<<<static_cast<unsigned>(ceil_div(static_cast<int64_t>(rows * D), 256)), 256, 0, st>>>(
+        O, lse, rows, D);
+    if (cudaGetLastError() != cudaSuccess) return FLARE_ERR_CUDA;
+    t_last_launches = 1;
+    return FLARE_OK;
+  }
+  Scratch s;
+  rc = get_scratch(workspace, workspace_bytes, encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes, st, &s);
+  if (rc) return rc;
+  int launches = 0;
+  rc = run_encode(Q, q_batched, K, V, O, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse);
+  const int rc2 = release_scratch(s, st);
+  if (!rc) {
+    rc = rc2;
+    t_last_launches = launches;
+  }
+  return rc;
+}
+
+int flare_lse_combine(const float* O_parts, const float* lse_parts, int R, int64_t part_stride, void* out,
+                      float* lse_out, int B, int H, int M, int D, int dtype, void* stream) {
+  int rc = check_sizes(B, H, 1, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  if (R < 1 || part_stride < 0) return FLARE_ERR_INVALID_ARG;
+  if (!device_ptr(O_parts) || !device_ptr_f32(lse_parts) || !device_ptr(out)) return FLARE_ERR_INVALID_ARG;
+  if (lse_out && !device_ptr_f32(lse_out)) return FLARE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int BH = B * H;
+  const long long rows = static_cast<long long>(BH) * M;
+  const MergeGeom g{R, M, D, static_cast<long long>(M) * D, part_stride ? part_stride : rows * D, M,
+                    part_stride ? part_stride : rows};
+  const dim3 grid(static_cast<unsigned>(ceil_div(int64_t(M) * D, 256)), BH);
+  ProfScope prof(FLARE_KERNEL_MERGE, st);
+  if (dtype == FLARE_BF16)
+    lse_merge_kernel<__nv_bfloat16, true><<<grid, 256, 0, st>>>(O_parts, lse_parts, nullptr,
+                                                               static_cast<__nv_bfloat16*>(out), lse_out, g);
+  else
+    lse_merge_kernel<float, true><<<grid, 256, 0, st>>>(O_parts, lse_parts, nullptr, static_cast<float*>(out),
+                                                       lse_out, g);
+  if (cudaGetLastError() != cudaSuccess) return FLARE_ERR_CUDA;
+  t_last_launches = 1;
+  return FLARE_OK;
 }
 
 int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N,

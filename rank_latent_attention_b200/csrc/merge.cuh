@@ -8,7 +8,8 @@
 // FLARE++ page describes for its token-sharded encoder ("FLARE++: Low-rank
 // attention with dynamic attention routing", "Contributions Clés",
 // context-parallel item: only latent outputs and softmax statistics are
-// exchanged).  Partials with l_p = 0 (no tokens) are skipped.
+// exchanged).  Partials with l_p = 0 (no tokens) are skipped.  The same kernel
+// combines the per-device (O, lse) results of a token-sharded encode.
 #pragma once
 
 #include <cuda_bf16.h>
@@ -28,34 +29,64 @@ __device__ __forceinline__ __nv_bfloat16 to_out<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
 }
 
+// Where the partials of (bh, p) sit, in floats: O element (m, d) at
+// O_part[bh * o_head + p * o_part + m * D + d], its statistics at
+// [bh * s_head + p * s_part + m].  The encode's own workspace is [BH][P][M][D]
+// (o_head = P*M*D, o_part = M*D, s_head = P*M, s_part = M); the per-device
+// results of a token-sharded encode, gathered, are [R][BH][M][D] with any
+// stride between devices (o_head = M*D, s_head = M, o_part = s_part = the
+// stride).
+struct MergeGeom {
+  int P, M, D;
+  long long o_head, o_part, s_head, s_part;
+};
+
 // grid (ceil(M*D / 256), BH), 256 threads; one thread per output element.
-template <typename OutT>
+//
+// FROM_LSE = false: partials are (O_p unnormalised, mref_p log2-domain, l_p).
+// FROM_LSE = true:  partials are (O_p normalised, lse_p natural log) -- one
+//   token shard's softmax output and log-sum-exp; an empty shard has
+//   lse_p = -inf.  l_part is unused; mref_p = lse_p log2(e), l_p = 1.
+// lse_out (may be null) receives the natural-log log-sum-exp of the union,
+// ln(2^m* sum_p w_p l_p); a row with no tokens at all gets out = 0 and
+// lse_out = -inf.
+template <typename OutT, bool FROM_LSE>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ O_part,
                                                         const float* __restrict__ m_part,
                                                         const float* __restrict__ l_part, OutT* __restrict__ out,
-                                                        int P, int M, int D) {
+                                                        float* __restrict__ lse_out, MergeGeom g) {
+  constexpr float kLn2 = 0.6931471805599453f;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
-  if (idx >= M * D) return;
+  if (idx >= g.M * g.D) return;
   const int bh = blockIdx.y;
-  const int m = idx / D;
-  const int d = idx - m * D;
-  const size_t base = static_cast<size_t>(bh) * P;
+  const int m = idx / g.D;
+  const int d = idx - m * g.D;
+  const long long sbase = bh * g.s_head + m;
+  const long long obase = bh * g.o_head + static_cast<long long>(m) * g.D + d;
   float mx = -INFINITY;
-  for (int p = 0; p < P; ++p) {
-    const size_t row = (base + p) * M + m;
-    if (l_part[row] > 0.f) mx = fmaxf(mx, m_part[row]);
-  }
-  float num = 0.f, den = 0.f;
-  for (int p = 0; p < P; ++p) {
-    const size_t row = (base + p) * M + m;
-    const float l = l_part[row];
-    if (l > 0.f) {
-      const float w = exp2f(m_part[row] - mx);
-      den = fmaf(w, l, den);
-      num = fmaf(w, O_part[row * D + d], num);
+  for (int p = 0; p < g.P; ++p) {
+    const long long row = sbase + p * g.s_part;
+    if constexpr (FROM_LSE) {
+      mx = fmaxf(mx, m_part[row] * kLog2e);
+    } else {
+      if (l_part[row] > 0.f) mx = fmaxf(mx, m_part[row]);
     }
   }
-  out[(static_cast<size_t>(bh) * M + m) * D + d] = to_out<OutT>(num / den);
+  float num = 0.f, den = 0.f;
+  if (mx > -INFINITY) {
+    for (int p = 0; p < g.P; ++p) {
+      const long long row = sbase + p * g.s_part;
+      const float l = FROM_LSE ? (m_part[row] > -INFINITY ? 1.f : 0.f) : l_part[row];
+      if (l > 0.f) {
+        const float w = exp2f((FROM_LSE ? m_part[row] * kLog2e : m_part[row]) - mx);
+        den = fmaf(w, l, den);
+        num = fmaf(w, O_part[obase + p * g.o_part], num);
+      }
+    }
+  }
+  const size_t orow = static_cast<size_t>(bh) * g.M + m;
+  out[orow * g.D + d] = to_out<OutT>(den > 0.f ? num / den : 0.f);
+  if (lse_out && d == 0) lse_out[orow] = den > 0.f ? (mx + log2f(den)) * kLn2 : -INFINITY;
 }
 
 }  // namespace flare

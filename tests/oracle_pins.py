@@ -21,6 +21,10 @@ What pins what:
   those of W_encode W_decode ("Спектральный анализ").
 * invariants of the definition: row sums, K = 0, M = 1, N = 1, constant V,
   token permutation, key shift, convex hull.
+* token shards ("FLARE++" page, "Contributions Clés", context parallelism):
+  the shard results combined equal the pure-Python encode over all tokens;
+  each shard's log-sum-exp equals a scalar ``math.log(fsum(exp))`` and
+  scipy's ``logsumexp``; one-token and empty shards take their closed forms.
 """
 from __future__ import annotations
 
@@ -242,6 +246,44 @@ def pin_mix_layout(o):
     assert np.allclose(Yr, Y[1, 2][rows], atol=1e-14)
 
 
+# ---------------------------------------------------------------- token shards
+def _bf_lse(Q, K):
+    out = []
+    for q in Q:
+        logits = [sum(q[d] * k[d] for d in range(len(q))) for k in K]
+        top = max(logits)
+        out.append(top + math.log(math.fsum(math.exp(x - top) for x in logits)))
+    return out
+
+
+def pin_shard_combine(o):
+    from scipy.special import logsumexp
+
+    for seed, (N, M, D, cuts) in enumerate([(7, 3, 2, [0, 3, 3, 7]), (12, 4, 3, [0, 1, 5, 11, 12]),
+                                            (5, 2, 2, [0, 5]), (9, 1, 1, [0, 0, 4, 9, 9])]):
+        Q, K, V = _case(800 + seed, N, M, D, std=1.3)
+        parts = [o.encode_shard(Q, K[a:b], V[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+        for (Op, lp), a, b in zip(parts, cuts[:-1], cuts[1:]):
+            if b == a:  # empty shard: no tokens, no weight
+                assert np.all(Op == 0) and np.all(np.isneginf(lp)), ("empty", seed)
+                continue
+            assert np.allclose(lp, _bf_lse(Q.tolist(), K[a:b].tolist()), rtol=1e-13, atol=1e-13), ("lse", seed)
+            assert np.allclose(lp, logsumexp(Q @ K[a:b].T, axis=1), rtol=1e-13, atol=1e-13), ("lse", seed)
+            assert np.allclose(Op, _bf_encode(Q.tolist(), K[a:b].tolist(), V[a:b].tolist()), rtol=1e-12,
+                               atol=1e-13), ("O", seed)
+            if b - a == 1:  # one token: O is its value row, lse its logit
+                assert np.allclose(Op, np.broadcast_to(V[a], Op.shape), atol=1e-15)
+                assert np.allclose(lp, Q @ K[a], atol=1e-14)
+        out, L = o.combine_shards([p[0] for p in parts], [p[1] for p in parts])
+        assert np.allclose(out, _bf_encode(Q.tolist(), K.tolist(), V.tolist()), rtol=1e-12, atol=1e-13), seed
+        assert np.allclose(L, logsumexp(Q @ K.T, axis=1), rtol=1e-13, atol=1e-13), seed
+        rev, Lr = o.combine_shards([p[0] for p in parts[::-1]], [p[1] for p in parts[::-1]])
+        assert np.allclose(rev, out, atol=1e-14) and np.allclose(Lr, L, atol=1e-14), seed
+    # a latent with every shard empty
+    out, L = o.combine_shards([np.zeros((2, 3))] * 2, [np.full(2, -np.inf)] * 2)
+    assert np.all(out == 0) and np.all(np.isneginf(L))
+
+
 ALL_PINS = [
     pin_worked_examples,
     pin_torch_sdpa,
@@ -250,4 +292,5 @@ ALL_PINS = [
     pin_rank_and_spectrum,
     pin_invariants,
     pin_mix_layout,
+    pin_shard_combine,
 ]

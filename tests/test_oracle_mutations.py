@@ -41,6 +41,18 @@ MUTANTS = {
     "eig_wrong_product": ("ev = np.linalg.eigvals(W_enc @ W_dec)", "ev = np.linalg.eigvals(W_enc @ W_enc.T)"),
     # communication matrix built from transposed factors (still NxN)
     "comm_transposed_factors": ("return W_dec @ W_enc", "return W_enc.T @ W_dec.T"),
+    # shard log-sum-exp without its max term
+    "shard_lse_drops_max": ("return (E @ V) / tot[:, None], top[:, 0] + np.log(tot)",
+                            "return (E @ V) / tot[:, None], np.log(tot)"),
+    # shards combined as a plain average (statistics ignored)
+    "combine_unweighted": ('out[live] = np.einsum("rm,rmd->md", w[:, live], O[:, live]) / tot[live, None]',
+                           'out[live] = O[:, live].mean(axis=0)'),
+    # shard weights taken linearly in lse instead of exponentially
+    "combine_linear_weights": ("w[:, live] = np.exp(lse[:, live] - top[live])",
+                               "w[:, live] = 1.0 + lse[:, live] - top[live]"),
+    # shard output left unnormalised
+    "shard_unnormalised": ("return (E @ V) / tot[:, None], top[:, 0] + np.log(tot)",
+                           "return (E @ V), top[:, 0] + np.log(tot)"),
 }
 
 
