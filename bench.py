@@ -24,7 +24,12 @@ the data path.  Rank 0 prints one JSON line:
 * cpu_baseline: the fp64 oracle on a bounded sample, on the host cores;
 * flare_fixed_query: FLARE with the seeds as fixed latent queries (one
   encode, one decode) on the same inputs, and the FLARE++ : FLARE step-time
-  ratio.
+  ratio;
+* context_parallel: ONE million-token cloud sharded over the N ranks by
+  token ranges (strong scaling; rank r's range is drawn from its own cloud),
+  mixed by the token-sharded path: shard encodes, one NCCL all-gather of the
+  latent (O, lse) per encode, combine, local decode.  With N = 1 it is the
+  same cloud as the headline on one GPU, through the sharded path.
 
 --impl reference times the oracle (the reference arm of this comparison) on
 the host cores, rank 0 only, and prints the same line with "impl": "reference".
@@ -356,6 +361,34 @@ def run_native(args):
         raise RuntimeError(f"device status after the communication matrix: {st}")
     del wsc, Cm, Qd
 
+    # ---- context parallelism: one cloud of w.N tokens sharded over the ranks
+    from rank_latent_attention_b200 import context_parallel as cp
+
+    t0, t1 = cp.token_range(w.N, world, rank)
+    K_r, V_r = K_d[:, :, t0:t1].contiguous(), V_d[:, :, t0:t1].contiguous()
+    ws_cp = torch.empty(max(1, flare.flare_encode_lse_workspace_size(1, w.H, t1 - t0, w.M, w.D, 1)),
+                        dtype=torch.uint8, device=dev)
+    cp_ops = cp.LibraryOps(None, workspace=ws_cp)
+
+    def cp_step():
+        return cp.flarepp_mix_cp(s_d, K_r, V_r, ops=cp_ops)
+
+    ncp = max(1, min(args.steps, 50))
+    for _ in range(3):
+        cp_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(ncp):
+        cp_step()
+    ev1.record(stream)
+    barrier()
+    cp_ms = max_over_ranks(ev0.elapsed_time(ev1)) / ncp
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after the context-parallel steps: {st}")
+    cp_exchange = 2 * cp.exchange_floats(1, w.H, w.M, w.D) * 4
+    del K_r, V_r, ws_cp
+
     # ---- end to end: pinned host inputs, copies inside the timed region
     Y_host = torch.empty(K_h.shape, dtype=torch.bfloat16).pin_memory()
     ne = max(1, min(args.e2e_steps, args.steps))
@@ -439,6 +472,10 @@ def run_native(args):
         "clocks": clocks.summary(),
         "flare_fixed_query": {"ms_per_step": flare_ms, "tokens_per_s": ranks.job_tokens_per_s(w.N, env, flare_ms),
                               "flarepp_over_flare": ms / flare_ms, "steps": nf},
+        "context_parallel": {"ms_per_step": cp_ms, "tokens_per_s": w.N / (cp_ms * 1e-3), "ranks": world,
+                             "scaling": "strong", "tokens": w.N, "steps": ncp,
+                             "exchange_bytes_per_rank_per_step": cp_exchange,
+                             "collective": "all_gather_into_tensor (NCCL), 2 per step" if world > 1 else "none (1 rank)"},
         "communication_matrix": {"ms_per_call": comm_ms, "launches": comm_launches,
                                  "what": "C = softmax_N(Q_dyn K^T) softmax_M(K Q_dyn^T), M x M per head"},
         "e2e": {"value": ranks.job_tokens_per_s(w.N, env, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -63,8 +63,9 @@ class LibraryOps:
 
     exchange_dtype = "float32"  # what flare_encode_lse writes and flare_lse_combine reads
 
-    def __init__(self, group=None):
+    def __init__(self, group=None, workspace=None):
         self.group = group
+        self.workspace = workspace  # device scratch for flare_encode_lse (None: the library allocates)
 
     def encode_lse(self, Q, K, V, send):
         import rank_latent_attention_b200 as flare
@@ -72,7 +73,8 @@ class LibraryOps:
         B, H, _, D = K.shape
         M = Q.shape[-2]
         n = B * H * M * D
-        flare.flare_encode_lse(Q, K, V, O=send[:n].view(B, H, M, D), lse=send[n:].view(B, H, M))
+        flare.flare_encode_lse(Q, K, V, O=send[:n].view(B, H, M, D), lse=send[n:].view(B, H, M),
+                               workspace=self.workspace)
 
     def all_gather(self, send):
         return gather_rows(send, self.group)
