@@ -38,6 +38,11 @@ as the routing encode; Q_dyn is used as-is (no normalisation) both as the
 routing queries and as the decode keys; softmax is max-subtracted, which is
 the same function.
 
+The backward (``flarepp_head_backward``) is the chain rule through the same
+three steps, written out step by step; the pages train the mixer end to end
+("FLARE++" page, "Méthodologie : FLARE++": the routing is built from SDPA
+calls alone, so it is differentiable like any attention).
+
 Every function here is "pinned" by tests in ``tests/test_oracle.py`` against
 things other than itself: the hand-derived worked examples in
 ``tests/golden/``, a pure-Python brute force, torch's float64 SDPA, the dense
@@ -61,6 +66,8 @@ __all__ = [
     "communication_eigenvalues",
     "encode_shard",
     "combine_shards",
+    "flarepp_head_backward",
+    "flarepp_backward",
 ]
 
 
@@ -207,3 +214,76 @@ def combine_shards(O_parts, lse_parts):
     L = np.full(top.shape, -np.inf)
     L[live] = top[live] + np.log(tot[live])
     return out, L
+
+
+def _softmax_backward(A: np.ndarray, dA: np.ndarray, c: np.ndarray) -> np.ndarray:
+    """dS for rows A = softmax(S) given dA = dL/dA and each row's c = sum(A * dA)."""
+    return A * (dA - c[:, None])
+
+
+def flarepp_head_backward(seeds, K, V, dY, Q_dyn=None, Z=None):
+    """Gradients of L = sum(dY * Y) for one FLARE++ head: (d_seeds, dK, dV).
+
+    Forward (``flarepp_head``): S1 = Q~ K^T, A1 = softmax over tokens,
+    Q_dyn = A1 V; S2 = Q_dyn K^T, A2 = softmax over tokens, Z = A2 V;
+    S3 = K Q_dyn^T, P3 = softmax over latents, Y = P3 Z.  Backward, last step
+    first:
+
+      decode   dZ = P3^T dY;  dP3 = dY Z^T;  dS3 = P3 (dP3 - rowsum(dY * Y))
+               dK += dS3 Q_dyn;  dQ_dyn += dS3^T K
+      routing  dV += A2^T dZ;  dA2 = dZ V^T;  dS2 = A2 (dA2 - rowsum(dZ * Z))
+               dQ_dyn += dS2 K;  dK += dS2^T Q_dyn
+      seed     dV += A1^T dQ_dyn;  dA1 = dQ_dyn V^T;
+               dS1 = A1 (dA1 - rowsum(dQ_dyn * Q_dyn))
+               d_seeds = dS1 K;  dK += dS1^T Q~
+
+    Each rowsum(dO * O) is the softmax backward's sum(A * dA) written with
+    the step's output O = A X.  With Q_dyn / Z given (as a reduced-precision
+    forward stored them), those values are used wherever Q_dyn / Z appear:
+    in the logits S2 and S3, in Y = P3 Z and in the rowsums; A1 is still
+    softmax(Q~ K^T).  That is the gradient of the stored chain with each
+    rounding passed through as the identity.
+    """
+    seeds = np.asarray(seeds, dtype=np.float64)
+    K = np.asarray(K, dtype=np.float64)
+    V = np.asarray(V, dtype=np.float64)
+    dY = np.asarray(dY, dtype=np.float64)
+    A1 = attention_weights(seeds, K)  # M x N
+    Qd = A1 @ V if Q_dyn is None else np.asarray(Q_dyn, dtype=np.float64)
+    A2 = attention_weights(Qd, K)  # M x N
+    Zs = A2 @ V if Z is None else np.asarray(Z, dtype=np.float64)
+    P3 = attention_weights(K, Qd)  # N x M
+    Y = P3 @ Zs
+
+    dZ = P3.T @ dY
+    dS3 = _softmax_backward(P3, dY @ Zs.T, np.sum(dY * Y, axis=1))
+    dK = dS3 @ Qd
+    dQd = dS3.T @ K
+
+    dV = A2.T @ dZ
+    dS2 = _softmax_backward(A2, dZ @ V.T, np.sum(dZ * Zs, axis=1))
+    dQd = dQd + dS2 @ K
+    dK = dK + dS2.T @ Qd
+
+    dV = dV + A1.T @ dQd
+    dS1 = _softmax_backward(A1, dQd @ V.T, np.sum(dQd * Qd, axis=1))
+    d_seeds = dS1 @ K
+    dK = dK + dS1.T @ seeds
+    return d_seeds, dK, dV
+
+
+def flarepp_backward(seeds, K, V, dY, Q_dyn=None, Z=None):
+    """Batched backward: seeds [H,M,D], K, V, dY [B,H,N,D] -> (d_seeds [H,M,D],
+    dK, dV [B,H,N,D]); the seeds are shared by the batch, so their gradient
+    is summed over it.  Q_dyn / Z [B,H,M,D] optionally as stored."""
+    B, H, N, D = K.shape
+    d_seeds = np.zeros(np.shape(seeds))
+    dK = np.zeros((B, H, N, D))
+    dV = np.zeros((B, H, N, D))
+    for b in range(B):
+        for h in range(H):
+            g = flarepp_head_backward(seeds[h], K[b, h], V[b, h], dY[b, h],
+                                      None if Q_dyn is None else Q_dyn[b, h], None if Z is None else Z[b, h])
+            d_seeds[h] += g[0]
+            dK[b, h], dV[b, h] = g[1], g[2]
+    return d_seeds, dK, dV

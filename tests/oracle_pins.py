@@ -25,6 +25,12 @@ What pins what:
   the shard results combined equal the pure-Python encode over all tokens;
   each shard's log-sum-exp equals a scalar ``math.log(fsum(exp))`` and
   scipy's ``logsumexp``; one-token and empty shards take their closed forms.
+* backward: torch float64 autograd through three SDPA calls; central finite
+  differences of the oracle's own forward along random directions; closed
+  forms (N = 1: dV = dY, dK = 0, d_seeds = 0; K = 0: dV = mean of dY,
+  d_seeds = 0); the seeds' gradient summed over the batch; the
+  stored-intermediates form equal to the exact one when given the exact
+  intermediates.
 """
 from __future__ import annotations
 
@@ -284,6 +290,67 @@ def pin_shard_combine(o):
     assert np.all(out == 0) and np.all(np.isneginf(L))
 
 
+# ---------------------------------------------------------------- backward
+def _torch_chain_grads(seeds, K, V, dY):
+    import torch
+
+    F = torch.nn.functional.scaled_dot_product_attention
+    t = [torch.tensor(x, dtype=torch.float64, requires_grad=True) for x in (seeds, K, V)]
+    Qd = F(t[0][None], t[1][None], t[2][None], scale=1.0)[0]
+    Z = F(Qd[None], t[1][None], t[2][None], scale=1.0)[0]
+    Y = F(t[1][None], Qd[None], Z[None], scale=1.0)[0]
+    (Y * torch.tensor(dY, dtype=torch.float64)).sum().backward()
+    return [x.grad.numpy() for x in t]
+
+
+def pin_backward(o):
+    for seed, (N, M, D) in enumerate([(7, 3, 4), (12, 5, 2), (4, 4, 3), (9, 1, 2), (3, 6, 5)]):
+        S, K, V = _case(900 + seed, N, M, D, std=0.9)
+        dY = _rng(950 + seed).standard_normal((N, D))
+        got = o.flarepp_head_backward(S, K, V, dY)
+        for name, g, w in zip(("d_seeds", "dK", "dV"), got, _torch_chain_grads(S, K, V, dY)):
+            assert np.allclose(g, w, rtol=1e-10, atol=1e-12), ("autograd", name, N, M, D)
+        # directional finite differences of L = sum(dY * Y) through the forward
+        g = _rng(980 + seed)
+        U = [g.standard_normal(x.shape) for x in (S, K, V)]
+        eps = 1e-5
+
+        def L(t):
+            return float(np.sum(dY * o.flarepp_head(S + t * U[0], K + t * U[1], V + t * U[2])[2]))
+
+        fd = (L(eps) - L(-eps)) / (2 * eps)
+        an = sum(float(np.sum(gi * ui)) for gi, ui in zip(got, U))
+        assert abs(fd - an) <= 1e-6 * max(1.0, abs(an)), ("finite differences", fd, an)
+        # the stored-intermediates form, given the exact intermediates
+        Qd, Z, _ = o.flarepp_head(S, K, V)
+        again = o.flarepp_head_backward(S, K, V, dY, Q_dyn=Qd, Z=Z)
+        for a, b in zip(got, again):
+            assert np.allclose(a, b, rtol=1e-13, atol=1e-14)
+    # N = 1: Y = V whatever the seeds and keys
+    S, K, V = _case(990, 1, 3, 2)
+    dY = _rng(991).standard_normal((1, 2))
+    ds, dk, dv = o.flarepp_head_backward(S, K, V, dY)
+    assert np.allclose(ds, 0, atol=1e-15) and np.allclose(dk, 0, atol=1e-15) and np.allclose(dv, dY, atol=1e-15)
+    # K = 0: every softmax is uniform, Y = mean(V), the seeds have no effect
+    S, _, V = _case(992, 6, 3, 2)
+    dY = _rng(993).standard_normal((6, 2))
+    ds, dk, dv = o.flarepp_head_backward(S, np.zeros((6, 2)), V, dY)
+    assert np.allclose(dv, np.broadcast_to(dY.mean(axis=0), dv.shape), atol=1e-14)
+    assert np.allclose(ds, 0, atol=1e-15)
+    # batched form: seeds shared by the batch, their gradient summed over it
+    B, H, N, M, D = 2, 2, 5, 3, 2
+    g = _rng(994)
+    seeds = g.standard_normal((H, M, D))
+    K, V, dY = (g.standard_normal((B, H, N, D)) for _ in range(3))
+    ds, dk, dv = o.flarepp_backward(seeds, K, V, dY)
+    for h in range(H):
+        want = [_torch_chain_grads(seeds[h], K[b, h], V[b, h], dY[b, h]) for b in range(B)]
+        assert np.allclose(ds[h], want[0][0] + want[1][0], rtol=1e-10, atol=1e-12)
+        for b in range(B):
+            assert np.allclose(dk[b, h], want[b][1], rtol=1e-10, atol=1e-12)
+            assert np.allclose(dv[b, h], want[b][2], rtol=1e-10, atol=1e-12)
+
+
 ALL_PINS = [
     pin_worked_examples,
     pin_torch_sdpa,
@@ -293,4 +360,5 @@ ALL_PINS = [
     pin_invariants,
     pin_mix_layout,
     pin_shard_combine,
+    pin_backward,
 ]

@@ -53,6 +53,19 @@ MUTANTS = {
     # shard output left unnormalised
     "shard_unnormalised": ("return (E @ V) / tot[:, None], top[:, 0] + np.log(tot)",
                            "return (E @ V), top[:, 0] + np.log(tot)"),
+    # decode backward without the softmax's row term
+    "bwd_decode_drops_rowsum": ("dS3 = _softmax_backward(P3, dY @ Zs.T, np.sum(dY * Y, axis=1))",
+                                "dS3 = _softmax_backward(P3, dY @ Zs.T, 0 * np.sum(dY * Y, axis=1))"),
+    # the decode's contribution to dQ_dyn forgotten
+    "bwd_no_decode_dqdyn": ("dQd = dS3.T @ K", "dQd = 0 * (dS3.T @ K)"),
+    # seed-encode row term taken with Z instead of Q_dyn
+    "bwd_seed_rowsum_with_Z": ("np.sum(dQd * Qd, axis=1)", "np.sum(dQd * Zs, axis=1)"),
+    # routing-encode value gradient through the decode weights
+    "bwd_dv_wrong_weights": ("dV = A2.T @ dZ", "dV = P3 @ dZ"),
+    # the seeds' gradient not summed over the batch
+    "bwd_seeds_not_summed": ("d_seeds[h] += g[0]", "d_seeds[h] = g[0]"),
+    # the seed encode's key gradient taken with Q_dyn
+    "bwd_seed_dk_with_qdyn": ("dK = dK + dS1.T @ seeds", "dK = dK + dS1.T @ Qd"),
 }
 
 
