@@ -145,6 +145,36 @@ int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, voi
  * no workspace.  Sizes as flare_encode with N = 1.
  */
 size_t flare_encode_lse_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+
+/*
+ * FLARE++ mixer backward: the gradients of L = sum(dY * Y) with respect to
+ * the seeds, K and V, where Y = flarepp_mix(seeds, K, V).  The pages train
+ * the mixer end to end ("FLARE++: Low-rank attention with dynamic attention
+ * routing", "Méthodologie : FLARE++": the routing is SDPA calls alone);
+ * this is the chain rule through the three steps:
+ *   decode   dZ = P3^T dY,  dS3 = P3 (dY Z^T - rowsum(dY * Y))
+ *   routing  dS2 = A2 (dZ V^T - rowsum(dZ * Z)),
+ *            dQ_dyn = dS3^T K + dS2 K
+ *   seed     dS1 = A1 (dQ_dyn V^T - rowsum(dQ_dyn * Q_dyn))
+ *   d_seeds = sum_b dS1 K,  dK = (dS3 + dS2^T) Q_dyn + dS1^T seeds,
+ *   dV = A2^T dZ + A1^T dQ_dyn
+ * with A1, A2 the encode weights (softmax over tokens) and P3 the decode
+ * weights (softmax over latents).
+ *   seeds      [H][M][D]            K, V, dY   [B][H][N][D]
+ *   d_seeds    [H][M][D] output (summed over the batch, which shares the seeds)
+ *   dK, dV     [B][H][N][D] outputs
+ * The call recomputes the two encodes (Q_dyn and Z exactly as flarepp_mix
+ * stores them, bf16 on FLARE_BF16, with their log-sum-exps) and then runs
+ * eight fp32 CUDA-core kernels.  Stored values such as Q_dyn and Z are used
+ * as stored, so the result is the gradient of the computed chain with each
+ * rounding taken as the identity.  Everything after the loads is fp32; dK, dV
+ * and d_seeds are stored in dtype.  dtype FLARE_BF16 or FLARE_F32; the
+ * workspace comes from flarepp_mix_backward_workspace_size.
+ */
+size_t flarepp_mix_backward_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+int flarepp_mix_backward(const void* seeds, const void* K, const void* V, const void* dY, void* d_seeds, void* dK,
+                         void* dV, int B, int H, int64_t N, int M, int D, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream);
 int flare_encode_lse(const void* Q, int q_batched, const void* K, const void* V, float* O, float* lse, int B,
                      int H, int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes,
                      void* stream);
@@ -249,7 +279,8 @@ typedef enum {
   FLARE_KERNEL_MERGE = 2,       /* log-sum-exp merge of encode partials  */
   FLARE_KERNEL_DECODE_TC = 3,   /* tcgen05 decode                        */
   FLARE_KERNEL_ENCODE_F32 = 4,  /* fp32 CUDA-core encode (partials)      */
-  FLARE_KERNEL_DECODE_F32 = 5   /* fp32 CUDA-core decode                 */
+  FLARE_KERNEL_DECODE_F32 = 5,  /* fp32 CUDA-core decode                 */
+  FLARE_KERNEL_BACKWARD = 6     /* the backward's CUDA-core kernels, one record for all eight */
 } flare_kernel_kind_t;
 
 /*

@@ -31,6 +31,8 @@ __all__ = [
     "flare_encode_lse",
     "flare_encode_lse_workspace_size",
     "flare_lse_combine",
+    "flarepp_mix_backward",
+    "flarepp_mix_backward_workspace_size",
     "flarepp_workspace_size",
     "flarepp_mix_host",
     "flare_communication_matrix",
@@ -59,6 +61,8 @@ _SIGNATURES = {
     "flare_encode": (_c_int, [_vp, _c_int, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_decode": (_c_int, [_vp, _vp, _c_int, _vp, _vp, *_SIZES, _vp]),
     "flare_encode_lse_workspace_size": (_c_size, _SIZES),
+    "flarepp_mix_backward_workspace_size": (_c_size, _SIZES),
+    "flarepp_mix_backward": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_encode_lse": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_lse_combine": (_c_int, [_vp, _vp, _c_int, _c_i64, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                    _vp]),
@@ -77,7 +81,8 @@ _SIGNATURES = {
     "flare_profile_end": (_c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int), _c_int]),
 }
 
-KERNEL_NAMES = {1: "encode_tc", 2: "lse_merge", 3: "decode_tc", 4: "encode_f32", 5: "decode_f32"}
+KERNEL_NAMES = {1: "encode_tc", 2: "lse_merge", 3: "decode_tc", 4: "encode_f32", 5: "decode_f32",
+                6: "backward_simt"}
 
 _lib = None
 
@@ -241,6 +246,33 @@ def flare_lse_combine(O_parts, lse_parts, out=None, lse_out=None, *, dtype=None,
                                    _stream(stream)),
            "flare_lse_combine")
     return out
+
+
+def flarepp_mix_backward_workspace_size(B, H, N, M, D, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (BF16 if "bfloat16" in str(dtype) else F32)
+    return lib().flarepp_mix_backward_workspace_size(B, H, N, M, D, code)
+
+
+def flarepp_mix_backward(seeds, K, V, dY, d_seeds=None, dK=None, dV=None, *, workspace=None, stream=None):
+    """Gradients (d_seeds [H,M,D], dK, dV [B,H,N,D]) of sum(dY * Y) for
+    Y = flarepp_mix(seeds, K, V); all tensors share K's dtype."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = seeds.shape[-2]
+    if d_seeds is None:
+        d_seeds = torch.empty_like(seeds)
+    if dK is None:
+        dK = torch.empty_like(K)
+    if dV is None:
+        dV = torch.empty_like(V)
+    ws, wsb = _ws(workspace)
+    dt = K.dtype
+    _check(lib().flarepp_mix_backward(_ptr(seeds, "seeds", dt), _ptr(K, "K", dt), _ptr(V, "V", dt),
+                                      _ptr(dY, "dY", dt), _ptr(d_seeds, "d_seeds", dt), _ptr(dK, "dK", dt),
+                                      _ptr(dV, "dV", dt), B, H, N, M, D, _dtype_code(K), ws, wsb,
+                                      _stream(stream)),
+           "flarepp_mix_backward")
+    return d_seeds, dK, dV
 
 
 def flarepp_mix_host(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, stream=None):

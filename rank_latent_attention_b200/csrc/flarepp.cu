@@ -13,6 +13,7 @@
 #include <vector>
 
 #include "../../include/flarepp.h"
+#include "backward_simt.cuh"
 #include "decode_tc.cuh"
 #include "encode_tc.cuh"
 #include "merge.cuh"
@@ -280,7 +281,7 @@ cudaError_t launch_merge(const EncodeWs& w, void* out, float* lse_out, int BH, i
 // writes the natural-log log-sum-exp of each latent's logits ([B][H][M]).
 int run_encode(const void* Q, int q_batched, const void* K, const void* V, void* out, int B, int H, int64_t N,
                int M, int D, int dtype, char* ws, cudaStream_t st, int* launches, bool q_bf16 = false,
-               float* lse_out = nullptr) {
+               float* lse_out = nullptr, bool f32_out = false) {
   const int BH = B * H;
   const int splits = choose_splits(BH, N, kEncTile);
   const int P = partials(M, D, splits, dtype);
@@ -314,8 +315,8 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
     ProfScope prof(FLARE_KERNEL_MERGE, st);
-    e = lse_out ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st)
-                : launch_merge<__nv_bfloat16>(w, out, nullptr, BH, P, M, D, st);
+    e = f32_out ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st)
+                : launch_merge<__nv_bfloat16>(w, out, lse_out, BH, P, M, D, st);
   } else {
     EncodeF32Args a;
     a.N = static_cast<int>(N);
@@ -585,6 +586,139 @@ bool host_ptr(const void* p) {
   return attr.type == cudaMemoryTypeHost || attr.type == cudaMemoryTypeUnregistered;
 }
 
+// ------------------------------------------------------------------ backward
+// Workspace of flarepp_mix_backward, in order: the encode's own workspace,
+// Q_dyn and Z (dtype), lse1, lse2, c1, c2 ([BH][M] fp32), dZ, dQ_dyn
+// ([BH][M][D] fp32), lse3, delta ([BH][N] fp32), two partial blocks
+// [BH][S][M][D] fp32.
+struct BackwardWs {
+  char* enc;
+  void* Qd;
+  void* Z;
+  float *lse1, *lse2, *c1, *c2, *dZ, *dQd, *lse3, *delta, *part;
+  long long part_stride;
+  int S;
+  size_t bytes;
+};
+
+int backward_splits(int BH, int64_t N, int M) {
+  const int64_t tiles = ceil_div(N, kBwdChunk);
+  const int64_t chunks = ceil_div(M, kBwdChunk);
+  const int64_t want = ceil_div(int64_t(2) * sm_count(), int64_t(BH) * chunks);
+  return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, tiles)));
+}
+
+BackwardWs backward_ws_layout(char* base, int BH, int64_t N, int M, int D, int dtype) {
+  BackwardWs w;
+  const size_t esz = dtype == FLARE_BF16 ? 2 : 4;
+  const size_t lat = static_cast<size_t>(BH) * M;
+  w.S = backward_splits(BH, N, M);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* p = base ? base + off : nullptr;
+    off += align256(bytes);
+    return p;
+  };
+  w.enc = take(encode_ws_layout(nullptr, BH, N, M, D, dtype).bytes);
+  w.Qd = take(lat * D * esz);
+  w.Z = take(lat * D * esz);
+  w.lse1 = reinterpret_cast<float*>(take(lat * 4));
+  w.lse2 = reinterpret_cast<float*>(take(lat * 4));
+  w.c1 = reinterpret_cast<float*>(take(lat * 4));
+  w.c2 = reinterpret_cast<float*>(take(lat * 4));
+  w.dZ = reinterpret_cast<float*>(take(lat * D * 4));
+  w.dQd = reinterpret_cast<float*>(take(lat * D * 4));
+  w.lse3 = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * N * 4));
+  w.delta = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * N * 4));
+  w.part_stride = static_cast<long long>(BH) * w.S * M * D;
+  w.part = reinterpret_cast<float*>(take(2 * static_cast<size_t>(w.part_stride) * 4));
+  w.bytes = off;
+  return w;
+}
+
+template <typename K>
+cudaError_t launch_dyn(K kernel, dim3 grid, int smem, cudaStream_t st, const BwdArgs& a) {
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kernel<<<grid, kBwdThreads, smem, st>>>(a);
+  return cudaGetLastError();
+}
+
+template <int D, typename T>
+cudaError_t launch_backward_d(const BwdArgs& a, int B, int BH, cudaStream_t st) {
+  const unsigned tok_tiles = static_cast<unsigned>(ceil_div(static_cast<int64_t>(a.N), kBwdChunk));
+  const unsigned lat_chunks = static_cast<unsigned>(ceil_div(a.M, kBwdChunk));
+  const dim3 red(static_cast<unsigned>(ceil_div(a.M, 8)), BH);
+  cudaError_t e;
+  if ((e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a))) return e;
+  if ((e = launch_dyn(latent_grad_kernel<D, T, kBwdDec>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st, a)))
+    return e;
+  grad_reduce_kernel<D, T, kBwdDec><<<red, kBwdThreads, 0, st>>>(a, B);
+  if ((e = cudaGetLastError())) return e;
+  if ((e = launch_dyn(latent_grad_kernel<D, T, kBwdEncRouting>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st,
+                      a)))
+    return e;
+  grad_reduce_kernel<D, T, kBwdEncRouting><<<red, kBwdThreads, 0, st>>>(a, B);
+  if ((e = cudaGetLastError())) return e;
+  if ((e = launch_dyn(latent_grad_kernel<D, T, kBwdEncSeed>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st,
+                      a)))
+    return e;
+  grad_reduce_kernel<D, T, kBwdEncSeed><<<dim3(red.x, a.H), kBwdThreads, 0, st>>>(a, B);
+  if ((e = cudaGetLastError())) return e;
+  return launch_dyn(token_grad_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_grad<D>(), st, a);
+}
+
+template <typename T>
+cudaError_t launch_backward_t(int D, const BwdArgs& a, int B, int BH, cudaStream_t st) {
+  switch (D) {
+    case 16: return launch_backward_d<16, T>(a, B, BH, st);
+    case 32: return launch_backward_d<32, T>(a, B, BH, st);
+    case 64: return launch_backward_d<64, T>(a, B, BH, st);
+    default: return launch_backward_d<128, T>(a, B, BH, st);
+  }
+}
+
+int run_backward(const void* seeds, const void* K, const void* V, const void* dY, void* d_seeds, void* dK, void* dV,
+                 int B, int H, int64_t N, int M, int D, int dtype, char* ws, cudaStream_t st, int* launches) {
+  const int BH = B * H;
+  const BackwardWs w = backward_ws_layout(ws, BH, N, M, D, dtype);
+  // the forward's encodes again, for Q_dyn and Z as it stored them and their
+  // per-latent log-sum-exps
+  int rc = run_encode(seeds, 0, K, V, w.Qd, B, H, N, M, D, dtype, w.enc, st, launches, false, w.lse1);
+  if (rc) return rc;
+  rc = run_encode(w.Qd, 1, K, V, w.Z, B, H, N, M, D, dtype, w.enc, st, launches, false, w.lse2);
+  if (rc) return rc;
+  BwdArgs a;
+  a.N = static_cast<int>(N);
+  a.M = M;
+  a.H = H;
+  a.seeds = seeds;
+  a.K = K;
+  a.V = V;
+  a.dY = dY;
+  a.Qd = w.Qd;
+  a.Z = w.Z;
+  a.lse1 = w.lse1;
+  a.lse2 = w.lse2;
+  a.lse3 = w.lse3;
+  a.delta = w.delta;
+  a.dZ = w.dZ;
+  a.dQd = w.dQd;
+  a.c1 = w.c1;
+  a.c2 = w.c2;
+  a.part = w.part;
+  a.part_stride = w.part_stride;
+  a.S = w.S;
+  a.d_seeds = d_seeds;
+  a.dK = dK;
+  a.dV = dV;
+  ProfScope prof(FLARE_KERNEL_BACKWARD, st);
+  const cudaError_t e = dtype == FLARE_BF16 ? launch_backward_t<__nv_bfloat16>(D, a, B, BH, st)
+                                            : launch_backward_t<float>(D, a, B, BH, st);
+  *launches += 8;
+  return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
+}
+
 // fp32 tensor in device memory with 4-byte alignment (the per-latent
 // statistics of a slice of a gathered [R][B][H][M] array need no more).
 bool device_ptr_f32(const void* p) {
@@ -668,7 +802,7 @@ int flare_encode_lse(const void* Q, int q_batched, const void* K, const void* V,
   rc = get_scratch(workspace, workspace_bytes, encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes, st, &s);
   if (rc) return rc;
   int launches = 0;
-  rc = run_encode(Q, q_batched, K, V, O, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse);
+  rc = run_encode(Q, q_batched, K, V, O, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse, true);
   const int rc2 = release_scratch(s, st);
   if (!rc) {
     rc = rc2;
@@ -701,6 +835,35 @@ int flare_lse_combine(const float* O_parts, const float* lse_parts, int R, int64
   if (cudaGetLastError() != cudaSuccess) return FLARE_ERR_CUDA;
   t_last_launches = 1;
   return FLARE_OK;
+}
+
+size_t flarepp_mix_backward_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (check_sizes(B, H, N, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
+  return backward_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
+}
+
+int flarepp_mix_backward(const void* seeds, const void* K, const void* V, const void* dY, void* d_seeds, void* dK,
+                         void* dV, int B, int H, int64_t N, int M, int D, int dtype, void* workspace,
+                         size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  for (const void* p : {seeds, K, V, dY, static_cast<const void*>(d_seeds), static_cast<const void*>(dK),
+                        static_cast<const void*>(dV)})
+    if (!device_ptr(p)) return FLARE_ERR_INVALID_ARG;
+  if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch s;
+  rc = get_scratch(workspace, workspace_bytes, backward_ws_layout(nullptr, B * H, N, M, D, dtype).bytes, st, &s);
+  if (rc) return rc;
+  int launches = 0;
+  rc = run_backward(seeds, K, V, dY, d_seeds, dK, dV, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  const int rc2 = release_scratch(s, st);
+  if (!rc) {
+    rc = rc2;
+    t_last_launches = launches;
+  }
+  return rc;
 }
 
 int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N,

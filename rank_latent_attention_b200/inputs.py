@@ -37,7 +37,7 @@ import os
 
 import numpy as np
 
-__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_head", "make_seeds", "custom"]
+__all__ = ["Workload", "WORKLOADS", "make_inputs", "make_head", "make_seeds", "make_upstream", "custom"]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -84,7 +84,7 @@ WORKLOADS: dict[str, Workload] = {
     ]
 }
 
-_TENSOR_ID = {"seeds": 0, "K": 1, "V": 2, "outliers": 3, "mesh": 4}
+_TENSOR_ID = {"seeds": 0, "K": 1, "V": 2, "outliers": 3, "mesh": 4, "dY": 5}
 
 
 def custom(B, H, N, M, D, dtype="bf16", kind="gauss", seed_index=99, scale=None) -> Workload:
@@ -161,6 +161,16 @@ def make_head(w: Workload, b: int, h: int) -> tuple[np.ndarray, np.ndarray]:
             k[rows] *= np.float32(w.outlier_gain)
             v[rows] *= np.float32(w.outlier_gain)
     return _round(k, w.dtype), _round(v, w.dtype)
+
+
+def make_upstream(w: Workload) -> np.ndarray:
+    """An upstream gradient dY [B,H,N,D] for the backward: N(0,1) values,
+    float32 holding values exact in the workload dtype."""
+    dY = np.empty((w.B, w.H, w.N, w.D), dtype=np.float32)
+    for b in range(w.B):
+        for h in range(w.H):
+            dY[b, h] = _rng(w, "dY", b, h).standard_normal((w.N, w.D), dtype=np.float32)
+    return _round(dY, w.dtype)
 
 
 def make_inputs(w: Workload, threads: int | None = None):

@@ -1,0 +1,109 @@
+"""GPU parity of flarepp_mix_backward against the fp64 oracle's backward.
+
+Two references per case:
+* stored: oracle.flarepp_backward given the Q_dyn and Z the GPU forward
+  stored (flarepp_mix_debug) -- the gradient of the computed chain with each
+  rounding taken as the identity, which is what the library computes.  Only
+  fp32 accumulation and the encodes' log-sum-exps separate the two.
+* exact: the oracle's exact gradient.  On fp32 inputs it is the same as the
+  stored one; on bf16 the stored Q_dyn and Z sit one bf16 rounding away.
+Bars, per gradient g with reference r, on the excess
+max(|g - r| - rel |r|) / RMS(r), where rel = 2^-8 covers the bf16 store of
+g (one rounding, 2^-9 relative, with room for the fp32 arithmetic before
+it) and 0 for fp32:
+* stored reference: 1e-4 (measured at most ~1e-5: fp32 accumulation and the
+  encodes' log-sum-exps are all that differ);
+* exact reference, bf16: 3e-2 (measured up to 7.6e-3: the stored Q_dyn and
+  Z move every logit of the routing and decode steps by up to 2^-9 of its
+  size, and d_seeds, which sums over all tokens, moves the most).
+"""
+import numpy as np
+import pytest
+
+import oracle
+import rank_latent_attention_b200 as flare
+from gpu_common import require_cuda, rms, to_dev, to_host
+from rank_latent_attention_b200 import inputs
+
+pytestmark = pytest.mark.gpu
+
+NAMES = ("d_seeds", "dK", "dV")
+CASES = [
+    ("tiny_f32", None),
+    ("cloud", None),
+    ("custom", (2, 3, 333, 48, 32, "f32")),     # ragged tokens, M not a multiple of 32
+    ("custom", (1, 2, 517, 256, 128, "bf16")),  # largest M and D
+    ("custom", (3, 2, 1, 16, 16, "bf16")),      # N = 1: dV = dY, the rest 0
+    ("custom", (1, 1, 100, 1, 16, "f32")),      # M = 1
+    ("custom", (2, 2, 257, 64, 64, "bf16")),
+]
+
+
+def _workload(name, spec):
+    if name != "custom":
+        return inputs.WORKLOADS[name]
+    B, H, N, M, D, dt = spec
+    return inputs.custom(B, H, N, M, D, dtype=dt, seed_index=70 + N % 17)
+
+
+def _run(w):
+    seeds, K, V = inputs.make_inputs(w)
+    dY = inputs.make_upstream(w)
+    dev = [to_dev(x, w.dtype) for x in (seeds, K, V, dY)]
+    grads = flare.flarepp_mix_backward(*dev)
+    launches = flare.flare_last_launch_count()
+    _, Qd, Z = flare.flarepp_mix_debug(*dev[:3])
+    assert flare.flare_check_status() == (0, 0)
+    return (seeds, K, V, dY), [to_host(g) for g in grads], to_host(Qd), to_host(Z), launches
+
+
+def _excess(got, want, rel):
+    """max over elements of (|got - want| - rel |want|) / RMS(want), per gradient."""
+    return [float(np.max(np.abs(g - r) - rel * np.abs(r))) / max(rms(r), 1e-30) for g, r in zip(got, want)]
+
+
+@pytest.mark.parametrize("name,spec", CASES, ids=lambda x: str(x))
+def test_backward_matches_oracle(name, spec):
+    require_cuda()
+    w = _workload(name, spec)
+    (seeds, K, V, dY), got, Qd, Z, launches = _run(w)
+    assert launches == 12  # two encodes (4) + eight backward kernels
+    args = [x.astype(np.float64) for x in (seeds, K, V, dY)]
+    stored = oracle.flarepp_backward(*args, Q_dyn=Qd, Z=Z)
+    exact = stored if w.dtype == "f32" else oracle.flarepp_backward(*args)
+    rel = 0.0 if w.dtype == "f32" else 2.0 ** -8  # the bf16 store of each gradient
+    e_stored, e_exact = _excess(got, stored, rel), _excess(got, exact, rel)
+    print(f"{w.name}: stored {e_stored} exact {e_exact}")
+    for g in got:
+        assert np.all(np.isfinite(g))
+    if w.N == 1:  # Y = V: dV = dY (up to its bf16 store), nothing else moves Y
+        assert np.allclose(got[2], dY, rtol=2.0 ** -8, atol=1e-6)
+        assert np.max(np.abs(got[0])) <= 1e-4 and np.max(np.abs(got[1])) <= 1e-4
+        return
+    for n, e in zip(NAMES, e_stored):
+        assert e <= 1e-4, (w.name, n, "stored", e)
+    if w.dtype == "bf16":
+        for n, e in zip(NAMES, e_exact):
+            assert e <= 3e-2, (w.name, n, "exact", e)
+
+
+def test_workspace_and_stream():
+    import torch
+
+    require_cuda()
+    w = inputs.custom(1, 2, 300, 32, 32, dtype="bf16", seed_index=77)
+    seeds, K, V = inputs.make_inputs(w)
+    dY = inputs.make_upstream(w)
+    dev = [to_dev(x, "bf16") for x in (seeds, K, V, dY)]
+    nbytes = flare.flarepp_mix_backward_workspace_size(1, 2, 300, 32, 32, torch.bfloat16)
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        g1 = flare.flarepp_mix_backward(*dev, workspace=ws, stream=s)
+    s.synchronize()
+    g2 = flare.flarepp_mix_backward(*dev)
+    for a, b in zip(g1, g2):
+        assert torch.equal(a, b)  # same kernels, same order: the same bits
+    small = torch.empty(nbytes - 256, dtype=torch.uint8, device="cuda")
+    with pytest.raises(flare.FlareError):
+        flare.flarepp_mix_backward(*dev, workspace=small)
