@@ -95,6 +95,8 @@ struct BwdArgs {
   float* dQd;         // [BH][M][D]
   float* c1;          // [BH][M]
   float* c2;          // [BH][M]
+  __nv_bfloat16* dZ16;   // [BH][M][D] bf16 copies of dZ and dQ_dyn for tensor-core
+  __nv_bfloat16* dQd16;  // operands (null when the CUDA-core token kernel runs)
   float* part;        // [BH][S][M][D] x 2 (second block at part + part_stride)
   long long part_stride;
   int S;              // token splits of the latent-row kernels
@@ -318,10 +320,12 @@ __global__ void __launch_bounds__(kBwdThreads) grad_reduce_kernel(const BwdArgs 
       if constexpr (MODE == kBwdDec) {
         a.dQd[o] = v;
         a.dZ[o] = v0;
+        if (a.dZ16) a.dZ16[o] = __float2bfloat16_rn(v0);
         dot = fmaf(v0, ld_f32(static_cast<const T*>(a.Z) + o), dot);
       } else {
         v += a.dQd[o];
         a.dQd[o] = v;
+        if (a.dQd16) a.dQd16[o] = __float2bfloat16_rn(v);
         dot = fmaf(v, ld_f32(static_cast<const T*>(a.Qd) + o), dot);
       }
     }

@@ -14,6 +14,7 @@
 
 #include "../../include/flarepp.h"
 #include "backward_simt.cuh"
+#include "backward_tc.cuh"
 #include "decode_tc.cuh"
 #include "encode_tc.cuh"
 #include "merge.cuh"
@@ -596,6 +597,7 @@ struct BackwardWs {
   void* Qd;
   void* Z;
   float *lse1, *lse2, *c1, *c2, *dZ, *dQd, *lse3, *delta, *part;
+  __nv_bfloat16 *dZ16, *dQd16;
   long long part_stride;
   int S;
   size_t bytes;
@@ -628,6 +630,8 @@ BackwardWs backward_ws_layout(char* base, int BH, int64_t N, int M, int D, int d
   w.c2 = reinterpret_cast<float*>(take(lat * 4));
   w.dZ = reinterpret_cast<float*>(take(lat * D * 4));
   w.dQd = reinterpret_cast<float*>(take(lat * D * 4));
+  w.dZ16 = reinterpret_cast<__nv_bfloat16*>(take(lat * D * 2));
+  w.dQd16 = reinterpret_cast<__nv_bfloat16*>(take(lat * D * 2));
   w.lse3 = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * N * 4));
   w.delta = reinterpret_cast<float*>(take(static_cast<size_t>(BH) * N * 4));
   w.part_stride = static_cast<long long>(BH) * w.S * M * D;
@@ -644,8 +648,47 @@ cudaError_t launch_dyn(K kernel, dim3 grid, int smem, cudaStream_t st, const Bwd
   return cudaGetLastError();
 }
 
+// The token-side kernel on the tensor cores: bf16, D <= 64.
+bool backward_token_tc(int D, int dtype) { return dtype == FLARE_BF16 && D <= 64; }
+
+template <int D>
+cudaError_t launch_token_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH, cudaStream_t st) {
+  using C = BtcCfg<D>;
+  CUtensorMap mQd, mZ, mdZ, mS, mdQ, mK, mdY, mV;
+  const int64_t N = a.N;
+  if (!make_map(&mQd, w.Qd, D, a.M, BH, 64) || !make_map(&mZ, w.Z, D, a.M, BH, 64) ||
+      !make_map(&mdZ, w.dZ16, D, a.M, BH, 64) || !make_map(&mS, a.seeds, D, a.M, a.H, 64) ||
+      !make_map(&mdQ, w.dQd16, D, a.M, BH, 64) || !make_map(&mK, a.K, D, N, BH, kBtcTile) ||
+      !make_map(&mdY, a.dY, D, N, BH, kBtcTile) || !make_map(&mV, a.V, D, N, BH, kBtcTile))
+    return cudaErrorInvalidValue;
+  BwdTcArgs t;
+  t.N = a.N;
+  t.M = a.M;
+  t.H = a.H;
+  t.tiles = static_cast<int>(ceil_div(N, kBtcTile));
+  t.splits = choose_splits(BH, N, kBtcTile);
+  t.lse1 = a.lse1;
+  t.lse2 = a.lse2;
+  t.c1 = a.c1;
+  t.c2 = a.c2;
+  t.lse3 = a.lse3;
+  t.delta = a.delta;
+  t.dK = static_cast<__nv_bfloat16*>(a.dK);
+  t.dV = static_cast<__nv_bfloat16*>(a.dV);
+  t.status = status_ptr();
+  t.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+  // at least 120 KB of shared memory: one CTA per SM, so two CTAs never
+  // contend for the 512 TMEM columns each allocates
+  const int smem = C::kSmemBytes > 120 * 1024 ? C::kSmemBytes : 120 * 1024;
+  auto kern = token_grad_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(t.splits, BH), C::kThreads, smem, st>>>(mQd, mZ, mdZ, mS, mdQ, mK, mdY, mV, t);
+  return cudaGetLastError();
+}
+
 template <int D, typename T>
-cudaError_t launch_backward_d(const BwdArgs& a, int B, int BH, cudaStream_t st) {
+cudaError_t launch_backward_d(const BwdArgs& a, const BackwardWs& w, int B, int BH, int dtype, cudaStream_t st) {
   const unsigned tok_tiles = static_cast<unsigned>(ceil_div(static_cast<int64_t>(a.N), kBwdChunk));
   const unsigned lat_chunks = static_cast<unsigned>(ceil_div(a.M, kBwdChunk));
   const dim3 red(static_cast<unsigned>(ceil_div(a.M, 8)), BH);
@@ -665,16 +708,20 @@ cudaError_t launch_backward_d(const BwdArgs& a, int B, int BH, cudaStream_t st) 
     return e;
   grad_reduce_kernel<D, T, kBwdEncSeed><<<dim3(red.x, a.H), kBwdThreads, 0, st>>>(a, B);
   if ((e = cudaGetLastError())) return e;
+  if constexpr (D <= 64) {
+    if (backward_token_tc(D, dtype)) return launch_token_grad_tc<D>(a, w, BH, st);
+  }
   return launch_dyn(token_grad_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_grad<D>(), st, a);
 }
 
 template <typename T>
-cudaError_t launch_backward_t(int D, const BwdArgs& a, int B, int BH, cudaStream_t st) {
+cudaError_t launch_backward_t(int D, const BwdArgs& a, const BackwardWs& w, int B, int BH, int dtype,
+                              cudaStream_t st) {
   switch (D) {
-    case 16: return launch_backward_d<16, T>(a, B, BH, st);
-    case 32: return launch_backward_d<32, T>(a, B, BH, st);
-    case 64: return launch_backward_d<64, T>(a, B, BH, st);
-    default: return launch_backward_d<128, T>(a, B, BH, st);
+    case 16: return launch_backward_d<16, T>(a, w, B, BH, dtype, st);
+    case 32: return launch_backward_d<32, T>(a, w, B, BH, dtype, st);
+    case 64: return launch_backward_d<64, T>(a, w, B, BH, dtype, st);
+    default: return launch_backward_d<128, T>(a, w, B, BH, dtype, st);
   }
 }
 
@@ -706,6 +753,9 @@ int run_backward(const void* seeds, const void* K, const void* V, const void* dY
   a.dQd = w.dQd;
   a.c1 = w.c1;
   a.c2 = w.c2;
+  const bool tc = backward_token_tc(D, dtype);
+  a.dZ16 = tc ? w.dZ16 : nullptr;
+  a.dQd16 = tc ? w.dQd16 : nullptr;
   a.part = w.part;
   a.part_stride = w.part_stride;
   a.S = w.S;
@@ -713,8 +763,8 @@ int run_backward(const void* seeds, const void* K, const void* V, const void* dY
   a.dK = dK;
   a.dV = dV;
   ProfScope prof(FLARE_KERNEL_BACKWARD, st);
-  const cudaError_t e = dtype == FLARE_BF16 ? launch_backward_t<__nv_bfloat16>(D, a, B, BH, st)
-                                            : launch_backward_t<float>(D, a, B, BH, st);
+  const cudaError_t e = dtype == FLARE_BF16 ? launch_backward_t<__nv_bfloat16>(D, a, w, B, BH, dtype, st)
+                                            : launch_backward_t<float>(D, a, w, B, BH, dtype, st);
   *launches += 8;
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
 }

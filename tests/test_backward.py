@@ -11,8 +11,15 @@ Bars, per gradient g with reference r, on the excess
 max(|g - r| - rel |r|) / RMS(r), where rel = 2^-8 covers the bf16 store of
 g (one rounding, 2^-9 relative, with room for the fp32 arithmetic before
 it) and 0 for fp32:
-* stored reference: 1e-4 (measured at most ~1e-5: fp32 accumulation and the
-  encodes' log-sum-exps are all that differ);
+* stored reference, CUDA-core kernels (fp32, or D = 128): 1e-4 (measured at
+  most ~1e-5: fp32 accumulation and the encodes' log-sum-exps are all that
+  differ);
+* stored reference, tensor-core kernels (bf16, D <= 64): 3e-2 (measured up
+  to 1e-2).  Their MMA operands are bf16: the softmax-gradient weights and
+  the copies of dZ and dQ_dyn each carry a 2^-9 relative rounding.  A
+  gradient row sums M such terms, whose rounding errors add in quadrature
+  while the terms themselves partly cancel.  The same holds for flash
+  attention's bf16 dS;
 * exact reference, bf16: 3e-2 (measured up to 7.6e-3: the stored Q_dyn and
   Z move every logit of the routing and decode steps by up to 2^-9 of its
   size, and d_seeds, which sums over all tokens, moves the most).
@@ -80,8 +87,9 @@ def test_backward_matches_oracle(name, spec):
         assert np.allclose(got[2], dY, rtol=2.0 ** -8, atol=1e-6)
         assert np.max(np.abs(got[0])) <= 1e-4 and np.max(np.abs(got[1])) <= 1e-4
         return
+    tensor_cores = w.dtype == "bf16" and w.D <= 64
     for n, e in zip(NAMES, e_stored):
-        assert e <= 1e-4, (w.name, n, "stored", e)
+        assert e <= (3e-2 if tensor_cores else 1e-4), (w.name, n, "stored", e)
     if w.dtype == "bf16":
         for n, e in zip(NAMES, e_exact):
             assert e <= 3e-2, (w.name, n, "exact", e)
