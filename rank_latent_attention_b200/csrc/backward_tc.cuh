@@ -318,4 +318,282 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Latent side of the backward on the tensor cores: per 128 latents of one head
+// (MMA rows) over a token range in tiles of 64 (MMA N of the logits):
+//   DEC   S = Q_dyn K_t^T, G = Z dY_t^T   e = exp(S - lse3_t), w = e (G - delta_t)
+//         dZ += e dY_t,  dQ_dyn += w K_t          (decode part of dQ_dyn)
+//   ENC   S = A K_t^T,   G = B V_t^T      e = exp(S - lse_m),  w = e (G - c_m)
+//         out += w K_t   with (A, B, lse, c, out) = (Q_dyn, dZ, lse2, c2, dQ_dyn)
+//         for the routing encode, (Q~, dQ_dyn, lse1, c1, d_seeds) for the seed encode
+// The partial sums of the CTA's token range go to the same [BH][S][M][D] fp32
+// blocks as latent_grad_kernel's, summed by grad_reduce_kernel.
+//
+// Warps 0-3: one latent row per thread.  Warp 4: TMA (two token stages) and
+// MMAs.  TMEM: S [0,64), G [64,128); e and w (bf16 pairs) are written over
+// the first half of S and of G once read; out0 [128, 128+D) (dZ, DEC only),
+// out1 [128+D, 128+2D).
+constexpr int kBltcTok = 64;
+
+struct BltcArgs {
+  int N, M, S, tiles;
+  const float* lse_row;  // ENC: [BH][M] lse of the encode (natural log)
+  const float* c_row;    // ENC: [BH][M]
+  const float* lse3;     // DEC: [BH][N]
+  const float* delta;    // DEC: [BH][N]
+  float* part;           // [BH][S][M][D] (out1), out0 at part + part_stride
+  long long part_stride;
+  int* status;
+  unsigned long long wait_ns;
+};
+
+template <int D>
+struct BltcCfg {
+  using G = TileGeom<D>;
+  static constexpr int kThreads = 160;
+  static constexpr int kIssuerWarp = 4;
+  static constexpr int kLatBytes = G::bytes(128);
+  static constexpr int kTokBytes = G::bytes(kBltcTok);
+  static constexpr int kOffLat = 0;                              // A, B [128][D]
+  static constexpr int kOffTok = 2 * kLatBytes;                  // stage s: K, X
+  static constexpr int kOffStat = kOffTok + 4 * kTokBytes;       // [2 buffers][2][64] floats
+  static constexpr int kOffBars = kOffStat + 2 * 2 * kBltcTok * 4;
+  static constexpr int kNumBars = 10;
+  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr uint32_t kColOut0 = 128;
+  static constexpr uint32_t kColOut1 = 128 + D;
+  static_assert(kColOut1 + D <= 256, "TMEM budget (256 columns per CTA)");
+  static constexpr uint32_t kIdescLogit = ptx::idesc_bf16(128, kBltcTok, 0, 0);
+  static constexpr uint32_t kIdescAcc = ptx::idesc_bf16(128, D, 0, 1);
+};
+
+enum { kSiteBwdLatIssuer = 9, kSiteBwdLatWeights = 10 };
+
+template <int D, int MODE>
+__global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
+    latent_grad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                          const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmX,
+                          const BltcArgs args, int a_per_batch_head, int H) {
+  using C = BltcCfg<D>;
+  using G = typename C::G;
+  constexpr bool kDec = MODE == 0;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
+  uint64_t* bar_lat = bars + 0;
+  uint64_t* full = bars + 1;   // [2] token stage landed
+  uint64_t* empty = bars + 3;  // [2] token stage consumed by the accumulation MMAs
+  uint64_t* bar_S = bars + 5;
+  uint64_t* bar_W = bars + 6;
+  uint64_t* bar_fin = bars + 7;
+  uint64_t* drain = bars + 8;
+  float* sTok = reinterpret_cast<float*>(smem + C::kOffStat);
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, bh = blockIdx.y, m0 = blockIdx.z * 128;
+  const int tile0 = static_cast<int>((static_cast<long long>(split) * args.tiles) / args.S);
+  const int tile1 = static_cast<int>((static_cast<long long>(split + 1) * args.tiles) / args.S);
+  const int T = tile1 - tile0;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar_lat, 1);
+    for (int i = 0; i < 2; ++i) {
+      ptx::mbar_init(&full[i], 1);
+      ptx::mbar_init(&empty[i], 1);
+    }
+    ptx::mbar_init(bar_S, 1);
+    ptx::mbar_init(bar_W, 4);
+    ptx::mbar_init(bar_fin, 1);
+    ptx::mbar_init(drain, 32);
+    *s_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == C::kIssuerWarp) {
+    ptx::tmem_alloc(s_tmem, 256);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t sbase = ptx::smem_u32(smem);
+
+  if (warp == C::kIssuerWarp) {
+    // ---------------------------------------------------------------- loads + MMAs
+    const int planeA = a_per_batch_head ? bh : bh % H;
+    auto load_tile = [&](int i) {
+      const int st = i & 1;
+      const int tok = (tile0 + i) * kBltcTok;
+      ptx::mbar_arrive_expect_tx(&full[st], 2 * C::kTokBytes);
+      ptx::tma_load_3d(smem + C::kOffTok + st * 2 * C::kTokBytes, &tmK, &full[st], 0, tok, bh);
+      ptx::tma_load_3d(smem + C::kOffTok + st * 2 * C::kTokBytes + C::kTokBytes, &tmX, &full[st], 0, tok, bh);
+    };
+    int loaded = 0;
+    if (ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(bar_lat, 2 * C::kLatBytes);
+      ptx::tma_load_3d(smem + C::kOffLat, &tmA, bar_lat, 0, m0, planeA);
+      ptx::tma_load_3d(smem + C::kOffLat + C::kLatBytes, &tmB, bar_lat, 0, m0, bh);
+      for (int i = 0; i < 2 && i < T; ++i) load_tile(i);
+    }
+    __syncwarp();
+    loaded = T < 2 ? T : 2;
+    bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_lat, 0, s_abort, args.wait_ns));
+    const uint32_t aA = sbase + C::kOffLat, aB = aA + C::kLatBytes;
+    for (int i = 0; ok && i < T; ++i) {
+      const int st = i & 1;
+      const uint32_t aK = sbase + C::kOffTok + st * 2 * C::kTokBytes, aX = aK + C::kTokBytes;
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[st], (i >> 1) & 1, s_abort, args.wait_ns));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t acc = k > 0 ? 1u : 0u;
+          ptx::mma_ss(tmem + 0, G::kmajor(aA, 128, k), G::kmajor(aK, kBltcTok, k), C::kIdescLogit, acc);
+          ptx::mma_ss(tmem + 64, G::kmajor(aB, 128, k), G::kmajor(aX, kBltcTok, k), C::kIdescLogit, acc);
+        }
+        ptx::mma_commit(bar_S);
+      }
+      __syncwarp();
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_W, i & 1, s_abort, args.wait_ns));
+      if (!ok) break;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < kBltcTok / 16; ++kk) {
+          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          if constexpr (kDec)
+            ptx::mma_ts(tmem + C::kColOut0, tmem + 0 + kk * 8, G::mnmajor(aX, kBltcTok, kk), C::kIdescAcc, acc);
+          ptx::mma_ts(tmem + C::kColOut1, tmem + 64 + kk * 8, G::mnmajor(aK, kBltcTok, kk), C::kIdescAcc, acc);
+        }
+        ptx::mma_commit(&empty[st]);
+        if (i == T - 1) ptx::mma_commit(bar_fin);
+      }
+      __syncwarp();
+      if (i + 2 < T) {
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&empty[st], (i >> 1) & 1, s_abort, args.wait_ns));
+        if (!ok) break;
+        if (ptx::elect_one()) load_tile(i + 2);
+        __syncwarp();
+        loaded = i + 3;
+      }
+    }
+    if (!ok) {
+      if (lane == 0) record_error(args.status, kErrTimeout, kSiteBwdLatIssuer);
+      *s_abort = 1;
+    }
+    ptx::mma_commit(drain);
+    ptx::mbar_wait_drain(drain, 0);
+    for (int t = (loaded > 2 ? loaded - 2 : 0); t < loaded; ++t) ptx::mbar_wait_drain(&full[t & 1], (t >> 1) & 1);
+    ptx::mbar_wait_drain(bar_lat, 0);
+  } else {
+    // ---------------------------------------------------------------- weights
+    constexpr float kL2e = 1.4426950408889634f;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const int m = m0 + warp * 32 + lane;
+    const bool live_m = m < args.M;
+    const size_t lat_row = static_cast<size_t>(bh) * args.M + (live_m ? m : 0);
+    float Lm = 0.f, cm = 0.f;
+    if constexpr (!kDec) {
+      Lm = live_m ? args.lse_row[lat_row] * kL2e : INFINITY;
+      cm = live_m ? args.c_row[lat_row] : 0.f;
+    }
+    const size_t tok_base = static_cast<size_t>(bh) * args.N;
+    bool ok = true;
+    for (int i = 0; ok && i < T; ++i) {
+      const long long t0 = static_cast<long long>(tile0 + i) * kBltcTok;
+      const int live_cols = static_cast<int>(args.N - t0 < kBltcTok ? args.N - t0 : kBltcTok);
+      float* stat = sTok + (i & 1) * 2 * kBltcTok;
+      if constexpr (kDec) {
+        // lse3 (log2 domain) and delta of the tile's tokens, shared by the 128 rows
+        const int j = threadIdx.x & (kBltcTok - 1);
+        const bool live = j < live_cols;
+        stat[threadIdx.x] = threadIdx.x < kBltcTok ? (live ? args.lse3[tok_base + t0 + j] * kL2e : 0.f)
+                                                   : (live ? args.delta[tok_base + t0 + j] : 0.f);
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+      }
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_S, i & 1, s_abort, args.wait_ns));
+      if (!ok) break;
+      ptx::tc_fence_after();
+#pragma unroll
+      for (int p = 0; p < 4; ++p) {
+        float sv[16], gv[16];
+        ptx::tmem_ld16(trow + 0 + 16 * p, sv);
+        ptx::tmem_ld16(trow + 64 + 16 * p, gv);
+        ptx::tmem_wait_ld();
+        uint32_t pe[8], pw[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          float e[2], w[2];
+#pragma unroll
+          for (int q = 0; q < 2; ++q) {
+            const int j = 16 * p + 2 * u + q;
+            float ee, ww;
+            if constexpr (kDec) {
+              ee = ptx::ex2(fmaf(sv[2 * u + q], kL2e, -stat[j]));
+              ww = ee * (gv[2 * u + q] - stat[kBltcTok + j]);
+            } else {
+              ee = ptx::ex2(fmaf(sv[2 * u + q], kL2e, -Lm));
+              ww = ee * (gv[2 * u + q] - cm);
+            }
+            const bool live = j < live_cols;
+            e[q] = live ? ee : 0.f;
+            w[q] = live ? ww : 0.f;
+          }
+          pe[u] = ptx::pack_bf16(e[0], e[1]);
+          pw[u] = ptx::pack_bf16(w[0], w[1]);
+        }
+        // over columns of S and G this thread has already read
+        ptx::tmem_st8(trow + 0 + 8 * p, pe);
+        ptx::tmem_st8(trow + 64 + 8 * p, pw);
+      }
+      ptx::tmem_wait_st();
+      ptx::tc_fence_before();
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(bar_W);
+    }
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_fin, 0, s_abort, args.wait_ns));
+      if (ok) {
+        ptx::tc_fence_after();
+        const size_t row = (static_cast<size_t>(bh) * args.S + split) * args.M + (live_m ? m : 0);
+#pragma unroll
+        for (int which = kDec ? 0 : 1; which < 2; ++which) {
+          float* dst = args.part + (which == 0 ? args.part_stride : 0) + row * D;
+          const uint32_t col = which == 0 ? C::kColOut0 : C::kColOut1;
+#pragma unroll
+          for (int d0 = 0; d0 < D; d0 += 16) {
+            float v[16];
+            ptx::tmem_ld16(trow + col + d0, v);
+            ptx::tmem_wait_ld();
+            if (live_m) {
+              float4* o = reinterpret_cast<float4*>(dst + d0);
+#pragma unroll
+              for (int z = 0; z < 4; ++z) o[z] = make_float4(v[4 * z], v[4 * z + 1], v[4 * z + 2], v[4 * z + 3]);
+            }
+          }
+        }
+      }
+    } else if (ok && live_m) {
+      // no tokens in this split: its partial is zero
+      const size_t row = (static_cast<size_t>(bh) * args.S + split) * args.M + m;
+      for (int which = kDec ? 0 : 1; which < 2; ++which)
+        for (int d = 0; d < D; ++d) args.part[(which == 0 ? args.part_stride : 0) + row * D + d] = 0.f;
+    }
+    if (!ok) {
+      if (lane == 0) record_error(args.status, kErrTimeout, kSiteBwdLatWeights);
+      *s_abort = 1;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::kIssuerWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 256);
+  }
+}
+
 }  // namespace flare

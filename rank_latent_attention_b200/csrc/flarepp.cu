@@ -12,6 +12,8 @@
 #include <mutex>
 #include <vector>
 
+#include <type_traits>
+
 #include "../../include/flarepp.h"
 #include "backward_simt.cuh"
 #include "backward_tc.cuh"
@@ -610,11 +612,20 @@ int backward_splits(int BH, int64_t N, int M) {
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(want, tiles)));
 }
 
+// The backward's tensor-core kernels: bf16, D <= 64.
+bool backward_tc(int D, int dtype) { return dtype == FLARE_BF16 && D <= 64; }
+
+// Token splits of the latent-side kernels (the partial blocks' S).
+int backward_latent_splits(int BH, int64_t N, int M, int D, int dtype) {
+  if (backward_tc(D, dtype)) return choose_splits(BH * static_cast<int>(ceil_div(M, 128)), N, kBltcTok);
+  return backward_splits(BH, N, M);
+}
+
 BackwardWs backward_ws_layout(char* base, int BH, int64_t N, int M, int D, int dtype) {
   BackwardWs w;
   const size_t esz = dtype == FLARE_BF16 ? 2 : 4;
   const size_t lat = static_cast<size_t>(BH) * M;
-  w.S = backward_splits(BH, N, M);
+  w.S = backward_latent_splits(BH, N, M, D, dtype);
   size_t off = 0;
   auto take = [&](size_t bytes) {
     char* p = base ? base + off : nullptr;
@@ -648,8 +659,40 @@ cudaError_t launch_dyn(K kernel, dim3 grid, int smem, cudaStream_t st, const Bwd
   return cudaGetLastError();
 }
 
-// The token-side kernel on the tensor cores: bf16, D <= 64.
-bool backward_token_tc(int D, int dtype) { return dtype == FLARE_BF16 && D <= 64; }
+template <int D, int MODE>
+cudaError_t launch_latent_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH, cudaStream_t st) {
+  using C = BltcCfg<D>;
+  CUtensorMap mA, mB, mK, mX;
+  const int64_t N = a.N;
+  const void* A = MODE == kBwdEncSeed ? a.seeds : w.Qd;
+  const void* Bm = MODE == kBwdDec ? w.Z : (MODE == kBwdEncRouting ? static_cast<const void*>(w.dZ16) : w.dQd16);
+  const void* X = MODE == kBwdDec ? a.dY : a.V;
+  if (!make_map(&mA, A, D, a.M, MODE == kBwdEncSeed ? a.H : BH, 128) || !make_map(&mB, Bm, D, a.M, BH, 128) ||
+      !make_map(&mK, a.K, D, N, BH, kBltcTok) || !make_map(&mX, X, D, N, BH, kBltcTok))
+    return cudaErrorInvalidValue;
+  BltcArgs t;
+  t.N = a.N;
+  t.M = a.M;
+  t.S = a.S;
+  t.tiles = static_cast<int>(ceil_div(N, kBltcTok));
+  t.lse_row = MODE == kBwdEncSeed ? a.lse1 : a.lse2;
+  t.c_row = MODE == kBwdEncSeed ? a.c1 : a.c2;
+  t.lse3 = a.lse3;
+  t.delta = a.delta;
+  t.part = a.part;
+  t.part_stride = a.part_stride;
+  t.status = status_ptr();
+  t.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+  // at least 80 KB of shared memory: at most two CTAs per SM, each with 256 TMEM columns
+  const int smem = C::kSmemBytes > 80 * 1024 ? C::kSmemBytes : 80 * 1024;
+  constexpr int kMode = MODE == kBwdDec ? 0 : 1;
+  auto kern = latent_grad_tc_kernel<D, kMode>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(a.S, BH, static_cast<unsigned>(ceil_div(a.M, 128))), C::kThreads, smem, st>>>(
+      mA, mB, mK, mX, t, MODE == kBwdEncSeed ? 0 : 1, a.H);
+  return cudaGetLastError();
+}
 
 template <int D>
 cudaError_t launch_token_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH, cudaStream_t st) {
@@ -693,23 +736,27 @@ cudaError_t launch_backward_d(const BwdArgs& a, const BackwardWs& w, int B, int 
   const unsigned lat_chunks = static_cast<unsigned>(ceil_div(a.M, kBwdChunk));
   const dim3 red(static_cast<unsigned>(ceil_div(a.M, 8)), BH);
   cudaError_t e;
+  const bool tc = D <= 64 && backward_tc(D, dtype);
+  // one latent-side pass: the tensor-core kernel or the CUDA-core one
+  auto latent = [&](auto mode) -> cudaError_t {
+    constexpr int kMode = decltype(mode)::value;
+    if constexpr (D <= 64) {
+      if (tc) return launch_latent_grad_tc<D, kMode>(a, w, BH, st);
+    }
+    return launch_dyn(latent_grad_kernel<D, T, kMode>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st, a);
+  };
   if ((e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a))) return e;
-  if ((e = launch_dyn(latent_grad_kernel<D, T, kBwdDec>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st, a)))
-    return e;
+  if ((e = latent(std::integral_constant<int, kBwdDec>{}))) return e;
   grad_reduce_kernel<D, T, kBwdDec><<<red, kBwdThreads, 0, st>>>(a, B);
   if ((e = cudaGetLastError())) return e;
-  if ((e = launch_dyn(latent_grad_kernel<D, T, kBwdEncRouting>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st,
-                      a)))
-    return e;
+  if ((e = latent(std::integral_constant<int, kBwdEncRouting>{}))) return e;
   grad_reduce_kernel<D, T, kBwdEncRouting><<<red, kBwdThreads, 0, st>>>(a, B);
   if ((e = cudaGetLastError())) return e;
-  if ((e = launch_dyn(latent_grad_kernel<D, T, kBwdEncSeed>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st,
-                      a)))
-    return e;
+  if ((e = latent(std::integral_constant<int, kBwdEncSeed>{}))) return e;
   grad_reduce_kernel<D, T, kBwdEncSeed><<<dim3(red.x, a.H), kBwdThreads, 0, st>>>(a, B);
   if ((e = cudaGetLastError())) return e;
   if constexpr (D <= 64) {
-    if (backward_token_tc(D, dtype)) return launch_token_grad_tc<D>(a, w, BH, st);
+    if (tc) return launch_token_grad_tc<D>(a, w, BH, st);
   }
   return launch_dyn(token_grad_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_grad<D>(), st, a);
 }
@@ -753,7 +800,7 @@ int run_backward(const void* seeds, const void* K, const void* V, const void* dY
   a.dQd = w.dQd;
   a.c1 = w.c1;
   a.c2 = w.c2;
-  const bool tc = backward_token_tc(D, dtype);
+  const bool tc = backward_tc(D, dtype);
   a.dZ16 = tc ? w.dZ16 : nullptr;
   a.dQd16 = tc ? w.dQd16 : nullptr;
   a.part = w.part;
