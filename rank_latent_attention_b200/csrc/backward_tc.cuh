@@ -596,4 +596,210 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
   }
 }
 
+// ---------------------------------------------------------------------------
+// Per-token statistics of the decode on the tensor cores: for 128 tokens of
+// one head (MMA rows) and the latents in chunks of 64,
+//   S3 = K_t Q_dyn^T,  dP3 = dY_t Z^T      (tcgen05, fp32 in TMEM)
+// and, online over the chunks (log2 domain), one thread per token:
+//   lse3_t  = log-sum-exp over the latents of S3,
+//   delta_t = sum_m softmax(S3)_m dP3_m    (= dY_t . Y_t).
+// Q_dyn and Z of the head stay in shared memory; logits are double-buffered
+// in TMEM (buffer b: S3 at 128 b, dP3 at 128 b + 64).
+constexpr int kBstChunk = 64;
+
+struct BstArgs {
+  int N, M, splits, tiles;
+  float* lse3;  // [BH][N]
+  float* delta;
+  int* status;
+  unsigned long long wait_ns;
+};
+
+template <int D>
+struct BstCfg {
+  using G = TileGeom<D>;
+  static constexpr int kThreads = 160;
+  static constexpr int kIssuerWarp = 4;
+  static constexpr int kLatBytes = G::bytes(256);
+  static constexpr int kTokBytes = G::bytes(128);
+  static constexpr int kOffLat = 0;                  // Q_dyn, Z [256][D]
+  static constexpr int kOffTok = 2 * kLatBytes;      // K, dY [128][D]
+  static constexpr int kOffBars = kOffTok + 2 * kTokBytes;
+  static constexpr int kNumBars = 8;
+  static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
+  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr uint32_t kIdesc = ptx::idesc_bf16(128, kBstChunk, 0, 0);
+};
+
+enum { kSiteBwdStatIssuer = 11, kSiteBwdStatRows = 12 };
+
+template <int D>
+__global__ void __launch_bounds__(BstCfg<D>::kThreads, 1)
+    token_stats_tc_kernel(const __grid_constant__ CUtensorMap tmQd, const __grid_constant__ CUtensorMap tmZ,
+                          const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmdY,
+                          const BstArgs args) {
+  using C = BstCfg<D>;
+  using G = typename C::G;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
+  uint64_t* bar_lat = bars + 0;
+  uint64_t* bar_tok = bars + 1;
+  uint64_t* bar_S = bars + 2;    // [2] logits of a chunk in buffer b
+  uint64_t* bar_rel = bars + 4;  // [2] buffer b read by the 4 row warps
+  uint64_t* bar_tdone = bars + 6;  // every MMA of a tile done (token tiles free)
+  uint64_t* drain = bars + 7;
+  uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
+  volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int split = blockIdx.x, bh = blockIdx.y;
+  const int tile0 = static_cast<int>((static_cast<long long>(split) * args.tiles) / args.splits);
+  const int tile1 = static_cast<int>((static_cast<long long>(split + 1) * args.tiles) / args.splits);
+  const int T = tile1 - tile0;
+  const int nC = (args.M + kBstChunk - 1) / kBstChunk;
+
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(bar_lat, 1);
+    ptx::mbar_init(bar_tok, 1);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&bar_S[b], 1);
+      ptx::mbar_init(&bar_rel[b], 4);
+    }
+    ptx::mbar_init(bar_tdone, 1);
+    ptx::mbar_init(drain, 32);
+    *s_abort = 0;
+    ptx::fence_mbar_init();
+  }
+  if (warp == C::kIssuerWarp) {
+    ptx::tmem_alloc(s_tmem, 256);
+    ptx::tmem_relinquish();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
+  const uint32_t tmem = *s_tmem;
+  const uint32_t sbase = ptx::smem_u32(smem);
+
+  if (warp == C::kIssuerWarp) {
+    const int boxes = (args.M + 63) / 64;
+    if (ptx::elect_one()) {
+      ptx::mbar_arrive_expect_tx(bar_lat, 2 * boxes * 64 * D * 2);
+      for (int bx = 0; bx < boxes; ++bx) {
+        ptx::tma_load_3d(smem + C::kOffLat + bx * 64 * G::kRowBytes, &tmQd, bar_lat, 0, bx * 64, bh);
+        ptx::tma_load_3d(smem + C::kOffLat + C::kLatBytes + bx * 64 * G::kRowBytes, &tmZ, bar_lat, 0, bx * 64, bh);
+      }
+    }
+    __syncwarp();
+    bool ok = true;
+    int tok_issued = -1;
+    int kc = 0;  // chunks issued (buffer kc & 1, its (kc >> 1)-th use)
+    const uint32_t aQ = sbase + C::kOffLat, aZ = aQ + C::kLatBytes;
+    const uint32_t aK = sbase + C::kOffTok, adY = aK + C::kTokBytes;
+    for (int i = 0; ok && i < T; ++i) {
+      if (i > 0) ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_tdone, (i - 1) & 1, s_abort, args.wait_ns));
+      if (!ok) break;
+      if (ptx::elect_one()) {
+        const int tok = (tile0 + i) * 128;
+        ptx::mbar_arrive_expect_tx(bar_tok, 2 * C::kTokBytes);
+        ptx::tma_load_3d(smem + C::kOffTok, &tmK, bar_tok, 0, tok, bh);
+        ptx::tma_load_3d(smem + C::kOffTok + C::kTokBytes, &tmdY, bar_tok, 0, tok, bh);
+      }
+      __syncwarp();
+      tok_issued = i;
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_tok, i & 1, s_abort, args.wait_ns) &&
+                                       (i > 0 || ptx::mbar_wait(bar_lat, 0, s_abort, args.wait_ns)));
+      for (int c = 0; ok && c < nC; ++c, ++kc) {
+        const int b = kc & 1;
+        // the buffer's previous chunk has been read by the row warps
+        if (kc >= 2) ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_rel[b], ((kc >> 1) - 1) & 1, s_abort, args.wait_ns));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
+          const uint32_t off = static_cast<uint32_t>(c * kBstChunk * G::kRowBytes);
+#pragma unroll
+          for (int k = 0; k < D / 16; ++k) {
+            const uint32_t acc = k > 0 ? 1u : 0u;
+            ptx::mma_ss(tmem + 128 * b, G::kmajor(aK, 128, k), G::kmajor(aQ + off, 256, k), C::kIdesc, acc);
+            ptx::mma_ss(tmem + 128 * b + 64, G::kmajor(adY, 128, k), G::kmajor(aZ + off, 256, k), C::kIdesc, acc);
+          }
+          ptx::mma_commit(&bar_S[b]);
+          if (c == nC - 1) ptx::mma_commit(bar_tdone);
+        }
+        __syncwarp();
+      }
+    }
+    if (!ok) {
+      if (lane == 0) record_error(args.status, kErrTimeout, kSiteBwdStatIssuer);
+      *s_abort = 1;
+    }
+    ptx::mma_commit(drain);
+    ptx::mbar_wait_drain(drain, 0);
+    if (tok_issued >= 0) ptx::mbar_wait_drain(bar_tok, tok_issued & 1);
+    ptx::mbar_wait_drain(bar_lat, 0);
+  } else {
+    constexpr float kL2e = 1.4426950408889634f;
+    constexpr float kLn2 = 0.6931471805599453f;
+    const uint32_t trow = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const size_t tok_base = static_cast<size_t>(bh) * args.N;
+    bool ok = true;
+    int kc = 0;
+    for (int i = 0; ok && i < T; ++i) {
+      float mx = -INFINITY, l = 0.f, acc = 0.f;
+      for (int c = 0; c < nC; ++c, ++kc) {
+        const int b = kc & 1;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_S[b], (kc >> 1) & 1, s_abort, args.wait_ns));
+        if (!ok) break;
+        ptx::tc_fence_after();
+#pragma unroll
+        for (int p = 0; p < kBstChunk / 16; ++p) {
+          float sv[16], gv[16];
+          ptx::tmem_ld16(trow + 128 * b + 16 * p, sv);
+          ptx::tmem_ld16(trow + 128 * b + 64 + 16 * p, gv);
+          ptx::tmem_wait_ld();
+          const int mbase = c * kBstChunk + 16 * p;
+          float cm = -INFINITY;
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            sv[j] = mbase + j < args.M ? sv[j] * kL2e : -INFINITY;
+            cm = fmaxf(cm, sv[j]);
+          }
+          const float nm = fmaxf(mx, cm);
+          if (nm > mx) {
+            const float sc = mx == -INFINITY ? 0.f : ptx::ex2(mx - nm);
+            l *= sc;
+            acc *= sc;
+            mx = nm;
+          }
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const float e = ptx::ex2(sv[j] - mx);  // 0 for masked latents
+            l += e;
+            acc = fmaf(e, gv[j], acc);
+          }
+        }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bar_rel[b]);
+      }
+      if (!ok) break;
+      const long long n = static_cast<long long>(tile0 + i) * 128 + warp * 32 + lane;
+      if (n < args.N) {
+        args.lse3[tok_base + n] = (mx + __log2f(l)) * kLn2;
+        args.delta[tok_base + n] = acc / l;
+      }
+    }
+    if (!ok) {
+      if (lane == 0) record_error(args.status, kErrTimeout, kSiteBwdStatRows);
+      *s_abort = 1;
+    }
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  if (warp == C::kIssuerWarp) {
+    ptx::tc_fence_after();
+    ptx::tmem_dealloc(tmem, 256);
+  }
+}
+
 }  // namespace flare

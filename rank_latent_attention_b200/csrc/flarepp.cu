@@ -695,6 +695,32 @@ cudaError_t launch_latent_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH,
 }
 
 template <int D>
+cudaError_t launch_token_stats_tc(const BwdArgs& a, const BackwardWs& w, int BH, cudaStream_t st) {
+  using C = BstCfg<D>;
+  CUtensorMap mQd, mZ, mK, mdY;
+  const int64_t N = a.N;
+  if (!make_map(&mQd, w.Qd, D, a.M, BH, 64) || !make_map(&mZ, w.Z, D, a.M, BH, 64) ||
+      !make_map(&mK, a.K, D, N, BH, 128) || !make_map(&mdY, a.dY, D, N, BH, 128))
+    return cudaErrorInvalidValue;
+  BstArgs t;
+  t.N = a.N;
+  t.M = a.M;
+  t.tiles = static_cast<int>(ceil_div(N, 128));
+  t.splits = choose_splits(BH, N, 128);
+  t.lse3 = a.lse3;
+  t.delta = a.delta;
+  t.status = status_ptr();
+  t.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+  // at least 80 KB of shared memory: at most two CTAs per SM, each with 256 TMEM columns
+  const int smem = C::kSmemBytes > 80 * 1024 ? C::kSmemBytes : 80 * 1024;
+  auto kern = token_stats_tc_kernel<D>;
+  cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kern<<<dim3(t.splits, BH), C::kThreads, smem, st>>>(mQd, mZ, mK, mdY, t);
+  return cudaGetLastError();
+}
+
+template <int D>
 cudaError_t launch_token_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH, cudaStream_t st) {
   using C = BtcCfg<D>;
   CUtensorMap mQd, mZ, mdZ, mS, mdQ, mK, mdY, mV;
@@ -745,7 +771,12 @@ cudaError_t launch_backward_d(const BwdArgs& a, const BackwardWs& w, int B, int 
     }
     return launch_dyn(latent_grad_kernel<D, T, kMode>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st, a);
   };
-  if ((e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a))) return e;
+  e = cudaSuccess;
+  if constexpr (D <= 64) {
+    if (tc) e = launch_token_stats_tc<D>(a, w, BH, st);
+  }
+  if (!tc) e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a);
+  if (e) return e;
   if ((e = latent(std::integral_constant<int, kBwdDec>{}))) return e;
   grad_reduce_kernel<D, T, kBwdDec><<<red, kBwdThreads, 0, st>>>(a, B);
   if ((e = cudaGetLastError())) return e;
