@@ -29,7 +29,9 @@ the data path.  Rank 0 prints one JSON line:
   token ranges (strong scaling; rank r's range is drawn from its own cloud),
   mixed by the token-sharded path: shard encodes, one NCCL all-gather of the
   latent (O, lse) per encode, combine, local decode.  With N = 1 it is the
-  same cloud as the headline on one GPU, through the sharded path.
+  same cloud as the headline on one GPU, through the sharded path;
+* backward: flarepp_mix_backward (gradients of the seeds, K and V for a
+  seeded N(0,1) dY) on the same inputs, with its per-kernel split.
 
 --impl reference times the oracle (the reference arm of this comparison) on
 the host cores, rank 0 only, and prints the same line with "impl": "reference".
@@ -389,6 +391,37 @@ def run_native(args):
     cp_exchange = 2 * cp.exchange_floats(1, w.H, w.M, w.D) * 4
     del K_r, V_r, ws_cp
 
+    # ---- backward: gradients of sum(dY * Y) for the seeds, K and V
+    gdy = torch.Generator(device=dev).manual_seed(5)
+    dY = torch.randn(K_d.shape, device=dev, generator=gdy).to(torch.bfloat16)
+    grads = (torch.empty_like(s_d), torch.empty_like(K_d), torch.empty_like(V_d))
+    wsb = torch.empty(flare.flarepp_mix_backward_workspace_size(1, w.H, w.N, w.M, w.D, 1), dtype=torch.uint8,
+                      device=dev)
+
+    def bwd_step():
+        flare.flarepp_mix_backward(s_d, K_d, V_d, dY, *grads, workspace=wsb)
+
+    for _ in range(2):
+        bwd_step()
+    bwd_launches = flare.flare_last_launch_count()
+    nb = max(1, min(args.steps, 20))
+    barrier()
+    ev0.record(stream)
+    for _ in range(nb):
+        bwd_step()
+    ev1.record(stream)
+    barrier()
+    bwd_ms = max_over_ranks(ev0.elapsed_time(ev1)) / nb
+    flare.flare_profile_begin(64)
+    bwd_step()
+    bwd_split = {}
+    for name, t in flare.flare_profile_end():
+        bwd_split[name] = bwd_split.get(name, 0.0) + t
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after the backward steps: {st}")
+    del dY, grads, wsb
+
     # ---- end to end: pinned host inputs, copies inside the timed region
     Y_host = torch.empty(K_h.shape, dtype=torch.bfloat16).pin_memory()
     ne = max(1, min(args.e2e_steps, args.steps))
@@ -476,6 +509,10 @@ def run_native(args):
                              "scaling": "strong", "tokens": w.N, "steps": ncp,
                              "exchange_bytes_per_rank_per_step": cp_exchange,
                              "collective": "all_gather_into_tensor (NCCL), 2 per step" if world > 1 else "none (1 rank)"},
+        "backward": {"ms_per_step": bwd_ms, "tokens_per_s": ranks.job_tokens_per_s(w.N, env, bwd_ms), "steps": nb,
+                     "launches": bwd_launches, "kernel_ms": bwd_split,
+                     "executed_gemm_tflops": 25 * 2.0 * w.N * w.M * w.D * w.H / (bwd_ms * 1e-3) / 1e12,
+                     "what": "d_seeds, dK, dV of sum(dY * Y); two recomputed encodes + eight kernels"},
         "communication_matrix": {"ms_per_call": comm_ms, "launches": comm_launches,
                                  "what": "C = softmax_N(Q_dyn K^T) softmax_M(K Q_dyn^T), M x M per head"},
         "e2e": {"value": ranks.job_tokens_per_s(w.N, env, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

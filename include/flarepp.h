@@ -165,7 +165,9 @@ size_t flare_encode_lse_workspace_size(int B, int H, int64_t N, int M, int D, in
  *   dK, dV     [B][H][N][D] outputs
  * The call recomputes the two encodes (Q_dyn and Z exactly as flarepp_mix
  * stores them, bf16 on FLARE_BF16, with their log-sum-exps) and then runs
- * eight fp32 CUDA-core kernels.  Stored values such as Q_dyn and Z are used
+ * eight kernels: on FLARE_BF16 with D <= 64 the five token/latent passes are
+ * tcgen05 tensor-core kernels (bf16 operands, fp32 accumulation), otherwise
+ * fp32 CUDA-core kernels; the three partial-sum reductions are fp32.  Stored values such as Q_dyn and Z are used
  * as stored, so the result is the gradient of the computed chain with each
  * rounding taken as the identity.  Everything after the loads is fp32; dK, dV
  * and d_seeds are stored in dtype.  dtype FLARE_BF16 or FLARE_F32; the
@@ -279,8 +281,11 @@ typedef enum {
   FLARE_KERNEL_MERGE = 2,       /* log-sum-exp merge of encode partials  */
   FLARE_KERNEL_DECODE_TC = 3,   /* tcgen05 decode                        */
   FLARE_KERNEL_ENCODE_F32 = 4,  /* fp32 CUDA-core encode (partials)      */
-  FLARE_KERNEL_DECODE_F32 = 5,  /* fp32 CUDA-core decode                 */
-  FLARE_KERNEL_BACKWARD = 6     /* the backward's CUDA-core kernels, one record for all eight */
+  FLARE_KERNEL_DECODE_F32 = 5,       /* fp32 CUDA-core decode                 */
+  FLARE_KERNEL_BWD_TOKEN_STATS = 6,  /* backward: per-token lse3, delta       */
+  FLARE_KERNEL_BWD_LATENT = 7,       /* backward: latent-side partials        */
+  FLARE_KERNEL_BWD_REDUCE = 8,       /* backward: sums of those partials      */
+  FLARE_KERNEL_BWD_TOKEN_GRAD = 9    /* backward: dK, dV                      */
 } flare_kernel_kind_t;
 
 /*

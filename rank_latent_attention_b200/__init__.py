@@ -82,7 +82,7 @@ _SIGNATURES = {
 }
 
 KERNEL_NAMES = {1: "encode_tc", 2: "lse_merge", 3: "decode_tc", 4: "encode_f32", 5: "decode_f32",
-                6: "backward_simt"}
+                6: "bwd_token_stats", 7: "bwd_latent", 8: "bwd_reduce", 9: "bwd_token_grad"}
 
 _lib = None
 

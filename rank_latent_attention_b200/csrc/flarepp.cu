@@ -766,26 +766,36 @@ cudaError_t launch_backward_d(const BwdArgs& a, const BackwardWs& w, int B, int 
   // one latent-side pass: the tensor-core kernel or the CUDA-core one
   auto latent = [&](auto mode) -> cudaError_t {
     constexpr int kMode = decltype(mode)::value;
+    ProfScope prof(FLARE_KERNEL_BWD_LATENT, st);
     if constexpr (D <= 64) {
       if (tc) return launch_latent_grad_tc<D, kMode>(a, w, BH, st);
     }
     return launch_dyn(latent_grad_kernel<D, T, kMode>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st, a);
   };
-  e = cudaSuccess;
-  if constexpr (D <= 64) {
-    if (tc) e = launch_token_stats_tc<D>(a, w, BH, st);
+  {
+    ProfScope prof(FLARE_KERNEL_BWD_TOKEN_STATS, st);
+    e = cudaSuccess;
+    if constexpr (D <= 64) {
+      if (tc) e = launch_token_stats_tc<D>(a, w, BH, st);
+    }
+    if (!tc) e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a);
   }
-  if (!tc) e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a);
   if (e) return e;
-  if ((e = latent(std::integral_constant<int, kBwdDec>{}))) return e;
-  grad_reduce_kernel<D, T, kBwdDec><<<red, kBwdThreads, 0, st>>>(a, B);
-  if ((e = cudaGetLastError())) return e;
-  if ((e = latent(std::integral_constant<int, kBwdEncRouting>{}))) return e;
-  grad_reduce_kernel<D, T, kBwdEncRouting><<<red, kBwdThreads, 0, st>>>(a, B);
-  if ((e = cudaGetLastError())) return e;
-  if ((e = latent(std::integral_constant<int, kBwdEncSeed>{}))) return e;
-  grad_reduce_kernel<D, T, kBwdEncSeed><<<dim3(red.x, a.H), kBwdThreads, 0, st>>>(a, B);
-  if ((e = cudaGetLastError())) return e;
+  auto reduce = [&](auto mode, dim3 grid) -> cudaError_t {
+    ProfScope prof(FLARE_KERNEL_BWD_REDUCE, st);
+    grad_reduce_kernel<D, T, decltype(mode)::value><<<grid, kBwdThreads, 0, st>>>(a, B);
+    return cudaGetLastError();
+  };
+  using Dec = std::integral_constant<int, kBwdDec>;
+  using Rout = std::integral_constant<int, kBwdEncRouting>;
+  using Seed = std::integral_constant<int, kBwdEncSeed>;
+  if ((e = latent(Dec{}))) return e;
+  if ((e = reduce(Dec{}, red))) return e;
+  if ((e = latent(Rout{}))) return e;
+  if ((e = reduce(Rout{}, red))) return e;
+  if ((e = latent(Seed{}))) return e;
+  if ((e = reduce(Seed{}, dim3(red.x, a.H)))) return e;
+  ProfScope prof(FLARE_KERNEL_BWD_TOKEN_GRAD, st);
   if constexpr (D <= 64) {
     if (tc) return launch_token_grad_tc<D>(a, w, BH, st);
   }
@@ -840,7 +850,6 @@ int run_backward(const void* seeds, const void* K, const void* V, const void* dY
   a.d_seeds = d_seeds;
   a.dK = dK;
   a.dV = dV;
-  ProfScope prof(FLARE_KERNEL_BACKWARD, st);
   const cudaError_t e = dtype == FLARE_BF16 ? launch_backward_t<__nv_bfloat16>(D, a, w, B, BH, dtype, st)
                                             : launch_backward_t<float>(D, a, w, B, BH, dtype, st);
   *launches += 8;
