@@ -17,11 +17,13 @@
 // head stay in shared memory for the whole range (TMA, loaded once), the
 // token tiles K, dY, V come in by TMA per tile.  Warps 0-3 own TMEM lanes
 // 0-127 (one token row per thread); warp 4 issues the TMA loads and the MMAs.
-// The schedule is serial: logits, weights, accumulation, chunk after chunk.
+// Logits are double-buffered: the MMAs of chunk g + 1 run while the rows
+// turn chunk g into weights.
 //
-// TMEM columns: S3 [0,32) dP3 [32,64) dA2 [64,96) S1 [96,128) dA1 [128,160),
-// weights wQ [160,176) wS [176,192) wZ [192,208) wD [208,224) (bf16 pairs),
-// dK [224, 224+D), dV [224+D, 224+2D).
+// TMEM columns, logit buffer b at 160 b: S3 [0,32) dP3 [32,64) dA2 [64,96)
+// S1 [96,128) dA1 [128,160); the weights (bf16 pairs) wQ, wS, wZ, wD go over
+// the first 16 columns of S3, dP3, dA2 and S1 once read; dK [320, 320+D),
+// dV [320+D, 320+2D).
 #pragma once
 
 #include <cuda.h>
@@ -61,13 +63,16 @@ struct BtcCfg {
   static constexpr int kOffTok = 5 * kLatBytes;            // K, dY, V
   static constexpr int kOffStats = kOffTok + 3 * kTokBytes;  // L1, L2, C1, C2 [kMPad]
   static constexpr int kOffBars = kOffStats + 4 * kMPad * 4;
-  static constexpr int kNumBars = 8;
+  static constexpr int kNumBars = 10;
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  static constexpr uint32_t kColW = 160;
-  static constexpr uint32_t kColDK = 224;
-  static constexpr uint32_t kColDV = 224 + D;
+  // logit buffer b at kBufCols * b; the weights overwrite the first 16
+  // columns of four of its logit tiles once their rows have read them
+  static constexpr uint32_t kBufCols = 160;
+  static constexpr uint32_t kOffWQ = 0, kOffWS = 32, kOffWZ = 64, kOffWD = 96;
+  static constexpr uint32_t kColDK = 2 * kBufCols;
+  static constexpr uint32_t kColDV = 2 * kBufCols + D;
   static_assert(kColDV + D <= 512, "TMEM budget");
   static constexpr uint32_t kIdescLogit = ptx::idesc_bf16(kBtcTile, kBtcChunk, 0, 0);
   static constexpr uint32_t kIdescAcc = ptx::idesc_bf16(kBtcTile, D, 0, 1);
@@ -89,11 +94,11 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* bar_lat = bars + 0;   // latent matrices landed
   uint64_t* bar_tok = bars + 1;   // token tile landed
-  uint64_t* bar_S = bars + 2;     // logits of a chunk computed
-  uint64_t* bar_W = bars + 3;     // weights of a chunk stored (4 warps)
-  uint64_t* bar_acc = bars + 4;   // last accumulation of a tile done
-  uint64_t* bar_free = bars + 5;  // dK, dV of a tile read out (4 warps)
-  uint64_t* drain = bars + 6;
+  uint64_t* bar_S = bars + 2;     // [2] logits of a chunk computed, per buffer
+  uint64_t* bar_W = bars + 4;     // [2] weights of a chunk stored (4 warps), per buffer
+  uint64_t* bar_acc = bars + 6;   // last accumulation of a tile done
+  uint64_t* bar_free = bars + 7;  // dK, dV of a tile read out (4 warps)
+  uint64_t* drain = bars + 8;
   float* sL1 = reinterpret_cast<float*>(smem + C::kOffStats);
   float* sL2 = sL1 + C::kMPad;
   float* sC1 = sL2 + C::kMPad;
@@ -112,8 +117,10 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_lat, 1);
     ptx::mbar_init(bar_tok, 1);
-    ptx::mbar_init(bar_S, 1);
-    ptx::mbar_init(bar_W, 4);
+    for (int b = 0; b < 2; ++b) {
+      ptx::mbar_init(&bar_S[b], 1);
+      ptx::mbar_init(&bar_W[b], 4);
+    }
     ptx::mbar_init(bar_acc, 1);
     ptx::mbar_init(bar_free, 4);
     ptx::mbar_init(drain, 32);
@@ -158,10 +165,8 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       }
     }
     __syncwarp();
-    int kc = 0;  // chunks issued so far (parity of bar_S / bar_W)
-    for (int i = 0; ok && i < T; ++i) {
-      if (i > 0) ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, (i - 1) & 1, s_abort, args.wait_ns));
-      if (!ok) break;
+    const int nG = T * nC;  // chunks of the CTA, in order; chunk g uses logit buffer g & 1
+    auto load_tokens = [&](int i) {
       if (ptx::elect_one()) {
         const int tok = (tile0 + i) * kBtcTile;
         ptx::mbar_arrive_expect_tx(bar_tok, 3 * C::kTokBytes);
@@ -171,46 +176,75 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       }
       __syncwarp();
       tok_issued = i;
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_tok, i & 1, s_abort, args.wait_ns) &&
-                                       (i > 0 || ptx::mbar_wait(bar_lat, 0, s_abort, args.wait_ns)));
-      for (int c = 0; ok && c < nC; ++c, ++kc) {
-        ptx::tc_fence_after();
-        if (ptx::elect_one()) {
-          const uint32_t lat_off = static_cast<uint32_t>(c * kBtcChunk * G::kRowBytes);
+    };
+    auto issue_logits = [&](int g) {
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+        const uint32_t buf = tmem + C::kBufCols * (g & 1);
+        const uint32_t lat_off = static_cast<uint32_t>((g % nC) * kBtcChunk * G::kRowBytes);
 #pragma unroll
-          for (int k = 0; k < D / 16; ++k) {
-            const uint64_t dKt = G::kmajor(aTok, kBtcTile, k);
-            const uint64_t ddY = G::kmajor(aTok + C::kTokBytes, kBtcTile, k);
-            const uint64_t dVt = G::kmajor(aTok + 2 * C::kTokBytes, kBtcTile, k);
-            const uint32_t acc = k > 0 ? 1u : 0u;
-            ptx::mma_ss(tmem + 0, dKt, G::kmajor(aLat + 0 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-            ptx::mma_ss(tmem + 32, ddY, G::kmajor(aLat + 1 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-            ptx::mma_ss(tmem + 64, dVt, G::kmajor(aLat + 2 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-            ptx::mma_ss(tmem + 96, dKt, G::kmajor(aLat + 3 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-            ptx::mma_ss(tmem + 128, dVt, G::kmajor(aLat + 4 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit,
-                        acc);
-          }
-          ptx::mma_commit(bar_S);
+        for (int k = 0; k < D / 16; ++k) {
+          const uint64_t dKt = G::kmajor(aTok, kBtcTile, k);
+          const uint64_t ddY = G::kmajor(aTok + C::kTokBytes, kBtcTile, k);
+          const uint64_t dVt = G::kmajor(aTok + 2 * C::kTokBytes, kBtcTile, k);
+          const uint32_t acc = k > 0 ? 1u : 0u;
+          ptx::mma_ss(buf + 0, dKt, G::kmajor(aLat + 0 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
+          ptx::mma_ss(buf + 32, ddY, G::kmajor(aLat + 1 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
+          ptx::mma_ss(buf + 64, dVt, G::kmajor(aLat + 2 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
+          ptx::mma_ss(buf + 96, dKt, G::kmajor(aLat + 3 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
+          ptx::mma_ss(buf + 128, dVt, G::kmajor(aLat + 4 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit,
+                      acc);
         }
-        __syncwarp();
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_W, kc & 1, s_abort, args.wait_ns) &&
-                                         (c > 0 || i == 0 || ptx::mbar_wait(bar_free, (i - 1) & 1, s_abort, args.wait_ns)));
-        if (!ok) break;
-        ptx::tc_fence_after();
-        if (ptx::elect_one()) {
-          const uint32_t lat_off = static_cast<uint32_t>(c * kBtcChunk * G::kRowBytes);
+        ptx::mma_commit(&bar_S[g & 1]);
+      }
+      __syncwarp();
+    };
+    // accumulation of chunk g; false on a timed-out wait
+    auto issue_acc = [&](int g) -> bool {
+      const int i = g / nC, c = g % nC;
+      bool w = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_W[g & 1], (g >> 1) & 1, s_abort, args.wait_ns) &&
+                                           (c > 0 || i == 0 || ptx::mbar_wait(bar_free, (i - 1) & 1, s_abort, args.wait_ns)));
+      if (!w) return false;
+      ptx::tc_fence_after();
+      if (ptx::elect_one()) {
+        const uint32_t buf = tmem + C::kBufCols * (g & 1);
+        const uint32_t lat_off = static_cast<uint32_t>(c * kBtcChunk * G::kRowBytes);
 #pragma unroll
-          for (int kk = 0; kk < kBtcChunk / 16; ++kk) {
-            const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
-            auto mn = [&](int j) { return G::mnmajor(aLat + j * C::kLatBytes + lat_off, C::kMPad, kk); };
-            ptx::mma_ts(tmem + C::kColDK, tmem + C::kColW + 0 + kk * 8, mn(0), C::kIdescAcc, first);
-            ptx::mma_ts(tmem + C::kColDK, tmem + C::kColW + 16 + kk * 8, mn(3), C::kIdescAcc, 1u);
-            ptx::mma_ts(tmem + C::kColDV, tmem + C::kColW + 32 + kk * 8, mn(2), C::kIdescAcc, first);
-            ptx::mma_ts(tmem + C::kColDV, tmem + C::kColW + 48 + kk * 8, mn(4), C::kIdescAcc, 1u);
-          }
-          if (c == nC - 1) ptx::mma_commit(bar_acc);
+        for (int kk = 0; kk < kBtcChunk / 16; ++kk) {
+          const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
+          auto mn = [&](int j) { return G::mnmajor(aLat + j * C::kLatBytes + lat_off, C::kMPad, kk); };
+          ptx::mma_ts(tmem + C::kColDK, buf + C::kOffWQ + kk * 8, mn(0), C::kIdescAcc, first);
+          ptx::mma_ts(tmem + C::kColDK, buf + C::kOffWS + kk * 8, mn(3), C::kIdescAcc, 1u);
+          ptx::mma_ts(tmem + C::kColDV, buf + C::kOffWZ + kk * 8, mn(2), C::kIdescAcc, first);
+          ptx::mma_ts(tmem + C::kColDV, buf + C::kOffWD + kk * 8, mn(4), C::kIdescAcc, 1u);
         }
-        __syncwarp();
+        if (c == nC - 1) ptx::mma_commit(bar_acc);
+      }
+      __syncwarp();
+      return true;
+    };
+    if (nG > 0) {
+      load_tokens(0);
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_tok, 0, s_abort, args.wait_ns) &&
+                                       ptx::mbar_wait(bar_lat, 0, s_abort, args.wait_ns));
+      if (ok) issue_logits(0);
+    }
+    for (int g = 0; ok && g < nG; ++g) {
+      const bool more = g + 1 < nG;
+      const bool new_tile = more && (g + 1) % nC == 0;
+      // the next chunk's logits go into the other buffer while this chunk's
+      // weights are computed (its rows read that buffer two chunks ago)
+      if (more && !new_tile) issue_logits(g + 1);
+      ok = issue_acc(g);
+      if (ok && new_tile) {
+        const int i = g / nC;
+        // every MMA of tile i done: the token tiles may be overwritten
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, i & 1, s_abort, args.wait_ns));
+        if (ok) {
+          load_tokens(i + 1);
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_tok, (i + 1) & 1, s_abort, args.wait_ns));
+        }
+        if (ok) issue_logits(g + 1);
       }
     }
     if (!ok) {
@@ -235,17 +269,19 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       const float L3 = live_tok ? args.lse3[tok_base + n] * kL2e : 0.f;
       const float dl = live_tok ? args.delta[tok_base + n] : 0.f;
       for (int c = 0; c < nC; ++c, ++kc) {
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_S, kc & 1, s_abort, args.wait_ns));
+        const int b = kc & 1;
+        const uint32_t buf = trow + C::kBufCols * b;
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_S[b], (kc >> 1) & 1, s_abort, args.wait_ns));
         if (!ok) break;
         ptx::tc_fence_after();
 #pragma unroll
         for (int hh = 0; hh < 2; ++hh) {
           float s3[16], dp[16], da2[16], s1[16], da1[16];
-          ptx::tmem_ld16(trow + 0 + hh * 16, s3);
-          ptx::tmem_ld16(trow + 32 + hh * 16, dp);
-          ptx::tmem_ld16(trow + 64 + hh * 16, da2);
-          ptx::tmem_ld16(trow + 96 + hh * 16, s1);
-          ptx::tmem_ld16(trow + 128 + hh * 16, da1);
+          ptx::tmem_ld16(buf + 0 + hh * 16, s3);
+          ptx::tmem_ld16(buf + 32 + hh * 16, dp);
+          ptx::tmem_ld16(buf + 64 + hh * 16, da2);
+          ptx::tmem_ld16(buf + 96 + hh * 16, s1);
+          ptx::tmem_ld16(buf + 128 + hh * 16, da1);
           ptx::tmem_wait_ld();
           uint32_t wq[8], ws[8], wz[8], wd[8];
 #pragma unroll
@@ -268,15 +304,16 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
             wz[u] = ptx::pack_bf16(z[0], z[1]);
             wd[u] = ptx::pack_bf16(dq[0], dq[1]);
           }
-          ptx::tmem_st8(trow + C::kColW + 0 + hh * 8, wq);
-          ptx::tmem_st8(trow + C::kColW + 16 + hh * 8, ws);
-          ptx::tmem_st8(trow + C::kColW + 32 + hh * 8, wz);
-          ptx::tmem_st8(trow + C::kColW + 48 + hh * 8, wd);
+          // into columns [8 hh, 8 hh + 8) of four logit tiles, read in piece 0
+          ptx::tmem_st8(buf + C::kOffWQ + hh * 8, wq);
+          ptx::tmem_st8(buf + C::kOffWS + hh * 8, ws);
+          ptx::tmem_st8(buf + C::kOffWZ + hh * 8, wz);
+          ptx::tmem_st8(buf + C::kOffWD + hh * 8, wd);
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(bar_W);
+        if (lane == 0) ptx::mbar_arrive(&bar_W[b]);
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, i & 1, s_abort, args.wait_ns));
