@@ -15,15 +15,16 @@
 //
 // One CTA per (token range, head); the five [M][D] latent matrices of the
 // head stay in shared memory for the whole range (TMA, loaded once), the
-// token tiles K, dY, V come in by TMA per tile.  Warps 0-3 own TMEM lanes
-// 0-127 (one token row per thread); warp 4 issues the TMA loads and the MMAs.
+// token tiles K, dY, V come in by TMA per tile.  Warps 0-7 turn logits into
+// weights, two per TMEM lane quarter (one token row per thread, one half of
+// a chunk's latents per warp); warp 8 issues the TMA loads and the MMAs.
 // Logits are double-buffered: the MMAs of chunk g + 1 run while the rows
 // turn chunk g into weights.
 //
-// TMEM columns, logit buffer b at 160 b: S3 [0,32) dP3 [32,64) dA2 [64,96)
-// S1 [96,128) dA1 [128,160); the weights (bf16 pairs) wQ, wS, wZ, wD go over
-// the first 16 columns of S3, dP3, dA2 and S1 once read; dK [320, 320+D),
-// dV [320+D, 320+2D).
+// TMEM columns, logit buffer b at 160 b: S3 [0,32) S1 [32,64) dA2 [64,96)
+// dA1 [96,128) dP3 [128,160) (S3 | S1 and dA2 | dA1 are one MMA each); the
+// weights (bf16 pairs) go over S3 and S1 once read (BtcCfg::w_col);
+// dK [320, 320+D), dV [320+D, 320+2D).
 #pragma once
 
 #include <cuda.h>
@@ -54,10 +55,17 @@ struct BwdTcArgs {
 template <int D>
 struct BtcCfg {
   using G = TileGeom<D>;
-  static constexpr int kThreads = 160;
-  static constexpr int kIssuerWarp = 4;
+  static constexpr int kThreads = 288;
+  static constexpr int kIssuerWarp = 8;  // warps 0-7: two per TMEM lane quarter
   static constexpr int kMPad = 256;  // latent rows reserved per matrix (M <= 256)
   static constexpr int kLatBytes = G::bytes(kMPad);
+  // Latent rows in shared memory, chunk by chunk: block c holds the 32 rows
+  // of chunk c of Q_dyn, Q~, dZ, dQ_dyn, Z in that order, so that (Q_dyn; Q~)
+  // and (dZ; dQ_dyn) are 64-row B operands: one MMA each against K_t and V_t.
+  static constexpr int kChunkRows = 5 * kBtcChunk;
+  __host__ __device__ static constexpr uint32_t lat_row(int c, int pos) {
+    return static_cast<uint32_t>((c * 5 + pos) * kBtcChunk);
+  }
   static constexpr int kTokBytes = G::bytes(kBtcTile);
   static constexpr int kOffLat = 0;                        // Q_dyn, Z, dZ, Q~, dQ_dyn
   static constexpr int kOffTok = 5 * kLatBytes;            // K, dY, V
@@ -67,14 +75,20 @@ struct BtcCfg {
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  // logit buffer b at kBufCols * b; the weights overwrite the first 16
-  // columns of four of its logit tiles once their rows have read them
+  // logit buffer b at kBufCols * b: S3 [0,32) S1 [32,64) dA2 [64,96)
+  // dA1 [96,128) dP3 [128,160).  The weights of latents [16 hh, 16 hh + 16)
+  // (K step hh of the accumulation) overwrite columns [16 hh, 16 hh + 16) of
+  // S3 (wQ, then wS) and of S1 (wZ, then wD): the columns that the warp
+  // handling those latents has itself just read.
   static constexpr uint32_t kBufCols = 160;
-  static constexpr uint32_t kOffWQ = 0, kOffWS = 32, kOffWZ = 64, kOffWD = 96;
+  __host__ __device__ static constexpr uint32_t w_col(int which, int hh) {
+    return (which >> 1) * 32 + hh * 16 + (which & 1) * 8;  // which: 0 wQ, 1 wS, 2 wZ, 3 wD
+  }
   static constexpr uint32_t kColDK = 2 * kBufCols;
   static constexpr uint32_t kColDV = 2 * kBufCols + D;
   static_assert(kColDV + D <= 512, "TMEM budget");
   static constexpr uint32_t kIdescLogit = ptx::idesc_bf16(kBtcTile, kBtcChunk, 0, 0);
+  static constexpr uint32_t kIdescLogit2 = ptx::idesc_bf16(kBtcTile, 2 * kBtcChunk, 0, 0);
   static constexpr uint32_t kIdescAcc = ptx::idesc_bf16(kBtcTile, D, 0, 1);
 };
 
@@ -119,10 +133,10 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
     ptx::mbar_init(bar_tok, 1);
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&bar_S[b], 1);
-      ptx::mbar_init(&bar_W[b], 4);
+      ptx::mbar_init(&bar_W[b], 8);
     }
     ptx::mbar_init(bar_acc, 1);
-    ptx::mbar_init(bar_free, 4);
+    ptx::mbar_init(bar_free, 8);
     ptx::mbar_init(drain, 32);
     *s_abort = 0;
     ptx::fence_mbar_init();
@@ -151,18 +165,15 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
     // ---------------------------------------------------------------- loads + MMAs
     const uint32_t aLat = sbase + C::kOffLat;  // matrix j at aLat + j * kLatBytes
     const uint32_t aTok = sbase + C::kOffTok;  // K, dY, V
-    const int boxes = (args.M + 63) / 64;
     bool ok = true;
     int tok_issued = -1;
     if (ptx::elect_one()) {
-      ptx::mbar_arrive_expect_tx(bar_lat, 5 * boxes * 64 * D * 2);
-      const CUtensorMap* maps[5] = {&tmQd, &tmZ, &tmdZ, &tmS, &tmdQ};
-      for (int j = 0; j < 5; ++j) {
-        const int plane = j == 3 ? h : bh;
-        for (int bx = 0; bx < boxes; ++bx)
-          ptx::tma_load_3d(smem + C::kOffLat + j * C::kLatBytes + bx * 64 * G::kRowBytes, maps[j], bar_lat, 0,
-                           bx * 64, plane);
-      }
+      ptx::mbar_arrive_expect_tx(bar_lat, 5 * nC * kBtcChunk * D * 2);
+      const CUtensorMap* maps[5] = {&tmQd, &tmS, &tmdZ, &tmdQ, &tmZ};  // block order
+      for (int c = 0; c < nC; ++c)
+        for (int j = 0; j < 5; ++j)
+          ptx::tma_load_3d(smem + C::kOffLat + C::lat_row(c, j) * G::kRowBytes, maps[j], bar_lat, 0, c * kBtcChunk,
+                           j == 1 ? h : bh);
     }
     __syncwarp();
     const int nG = T * nC;  // chunks of the CTA, in order; chunk g uses logit buffer g & 1
@@ -181,19 +192,17 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
         const uint32_t buf = tmem + C::kBufCols * (g & 1);
-        const uint32_t lat_off = static_cast<uint32_t>((g % nC) * kBtcChunk * G::kRowBytes);
+        const int c = g % nC;
+        auto lat = [&](int pos) { return aLat + C::lat_row(c, pos) * G::kRowBytes; };
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint64_t dKt = G::kmajor(aTok, kBtcTile, k);
           const uint64_t ddY = G::kmajor(aTok + C::kTokBytes, kBtcTile, k);
           const uint64_t dVt = G::kmajor(aTok + 2 * C::kTokBytes, kBtcTile, k);
           const uint32_t acc = k > 0 ? 1u : 0u;
-          ptx::mma_ss(buf + 0, dKt, G::kmajor(aLat + 0 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-          ptx::mma_ss(buf + 32, ddY, G::kmajor(aLat + 1 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-          ptx::mma_ss(buf + 64, dVt, G::kmajor(aLat + 2 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-          ptx::mma_ss(buf + 96, dKt, G::kmajor(aLat + 3 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit, acc);
-          ptx::mma_ss(buf + 128, dVt, G::kmajor(aLat + 4 * C::kLatBytes + lat_off, C::kMPad, k), C::kIdescLogit,
-                      acc);
+          ptx::mma_ss(buf + 0, dKt, G::kmajor(lat(0), 2 * kBtcChunk, k), C::kIdescLogit2, acc);   // S3 | S1
+          ptx::mma_ss(buf + 64, dVt, G::kmajor(lat(2), 2 * kBtcChunk, k), C::kIdescLogit2, acc);  // dA2 | dA1
+          ptx::mma_ss(buf + 128, ddY, G::kmajor(lat(4), kBtcChunk, k), C::kIdescLogit, acc);      // dP3
         }
         ptx::mma_commit(&bar_S[g & 1]);
       }
@@ -208,15 +217,16 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
         const uint32_t buf = tmem + C::kBufCols * (g & 1);
-        const uint32_t lat_off = static_cast<uint32_t>(c * kBtcChunk * G::kRowBytes);
 #pragma unroll
         for (int kk = 0; kk < kBtcChunk / 16; ++kk) {
           const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
-          auto mn = [&](int j) { return G::mnmajor(aLat + j * C::kLatBytes + lat_off, C::kMPad, kk); };
-          ptx::mma_ts(tmem + C::kColDK, buf + C::kOffWQ + kk * 8, mn(0), C::kIdescAcc, first);
-          ptx::mma_ts(tmem + C::kColDK, buf + C::kOffWS + kk * 8, mn(3), C::kIdescAcc, 1u);
-          ptx::mma_ts(tmem + C::kColDV, buf + C::kOffWZ + kk * 8, mn(2), C::kIdescAcc, first);
-          ptx::mma_ts(tmem + C::kColDV, buf + C::kOffWD + kk * 8, mn(4), C::kIdescAcc, 1u);
+          auto mn = [&](int pos) {
+            return G::mnmajor(aLat + C::lat_row(c, pos) * G::kRowBytes, C::kChunkRows, kk);
+          };
+          ptx::mma_ts(tmem + C::kColDK, buf + C::w_col(0, kk), mn(0), C::kIdescAcc, first);  // wQ Q_dyn
+          ptx::mma_ts(tmem + C::kColDK, buf + C::w_col(1, kk), mn(1), C::kIdescAcc, 1u);     // wS Q~
+          ptx::mma_ts(tmem + C::kColDV, buf + C::w_col(2, kk), mn(2), C::kIdescAcc, first);  // wZ dZ
+          ptx::mma_ts(tmem + C::kColDV, buf + C::w_col(3, kk), mn(3), C::kIdescAcc, 1u);     // wD dQ_dyn
         }
         if (c == nC - 1) ptx::mma_commit(bar_acc);
       }
@@ -258,13 +268,14 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
     ptx::mbar_wait_drain(bar_lat, 0);
   } else {
     // ---------------------------------------------------------------- weights
-    const uint32_t lane_off = static_cast<uint32_t>(warp * 32) << 16;
+    const int quarter = warp & 3, hh = warp >> 2;  // TMEM lanes 32 quarter.., latents 16 hh.. of a chunk
+    const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t trow = tmem + lane_off;
     const size_t tok_base = static_cast<size_t>(bh) * args.N;
     bool ok = true;
     int kc = 0;
     for (int i = 0; ok && i < T; ++i) {
-      const long long n = static_cast<long long>(tile0 + i) * kBtcTile + warp * 32 + lane;
+      const long long n = static_cast<long long>(tile0 + i) * kBtcTile + quarter * 32 + lane;
       const bool live_tok = n < args.N;
       const float L3 = live_tok ? args.lse3[tok_base + n] * kL2e : 0.f;
       const float dl = live_tok ? args.delta[tok_base + n] : 0.f;
@@ -274,14 +285,13 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_S[b], (kc >> 1) & 1, s_abort, args.wait_ns));
         if (!ok) break;
         ptx::tc_fence_after();
-#pragma unroll
-        for (int hh = 0; hh < 2; ++hh) {
+        {
           float s3[16], dp[16], da2[16], s1[16], da1[16];
           ptx::tmem_ld16(buf + 0 + hh * 16, s3);
-          ptx::tmem_ld16(buf + 32 + hh * 16, dp);
+          ptx::tmem_ld16(buf + 32 + hh * 16, s1);
           ptx::tmem_ld16(buf + 64 + hh * 16, da2);
-          ptx::tmem_ld16(buf + 96 + hh * 16, s1);
-          ptx::tmem_ld16(buf + 128 + hh * 16, da1);
+          ptx::tmem_ld16(buf + 96 + hh * 16, da1);
+          ptx::tmem_ld16(buf + 128 + hh * 16, dp);
           ptx::tmem_wait_ld();
           uint32_t wq[8], ws[8], wz[8], wd[8];
 #pragma unroll
@@ -304,11 +314,10 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
             wz[u] = ptx::pack_bf16(z[0], z[1]);
             wd[u] = ptx::pack_bf16(dq[0], dq[1]);
           }
-          // into columns [8 hh, 8 hh + 8) of four logit tiles, read in piece 0
-          ptx::tmem_st8(buf + C::kOffWQ + hh * 8, wq);
-          ptx::tmem_st8(buf + C::kOffWS + hh * 8, ws);
-          ptx::tmem_st8(buf + C::kOffWZ + hh * 8, wz);
-          ptx::tmem_st8(buf + C::kOffWD + hh * 8, wd);
+          ptx::tmem_st8(buf + C::w_col(0, hh), wq);
+          ptx::tmem_st8(buf + C::w_col(1, hh), ws);
+          ptx::tmem_st8(buf + C::w_col(2, hh), wz);
+          ptx::tmem_st8(buf + C::w_col(3, hh), wd);
         }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
@@ -319,8 +328,8 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, i & 1, s_abort, args.wait_ns));
       if (!ok) break;
       ptx::tc_fence_after();
-#pragma unroll
-      for (int which = 0; which < 2; ++which) {
+      {
+        const int which = hh;  // warps 0-3 store dK, warps 4-7 dV
         __nv_bfloat16* dst = (which == 0 ? args.dK : args.dV) + (tok_base + (live_tok ? n : 0)) * D;
         const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
 #pragma unroll

@@ -725,9 +725,9 @@ cudaError_t launch_token_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH, 
   using C = BtcCfg<D>;
   CUtensorMap mQd, mZ, mdZ, mS, mdQ, mK, mdY, mV;
   const int64_t N = a.N;
-  if (!make_map(&mQd, w.Qd, D, a.M, BH, 64) || !make_map(&mZ, w.Z, D, a.M, BH, 64) ||
-      !make_map(&mdZ, w.dZ16, D, a.M, BH, 64) || !make_map(&mS, a.seeds, D, a.M, a.H, 64) ||
-      !make_map(&mdQ, w.dQd16, D, a.M, BH, 64) || !make_map(&mK, a.K, D, N, BH, kBtcTile) ||
+  if (!make_map(&mQd, w.Qd, D, a.M, BH, kBtcChunk) || !make_map(&mZ, w.Z, D, a.M, BH, kBtcChunk) ||
+      !make_map(&mdZ, w.dZ16, D, a.M, BH, kBtcChunk) || !make_map(&mS, a.seeds, D, a.M, a.H, kBtcChunk) ||
+      !make_map(&mdQ, w.dQd16, D, a.M, BH, kBtcChunk) || !make_map(&mK, a.K, D, N, BH, kBtcTile) ||
       !make_map(&mdY, a.dY, D, N, BH, kBtcTile) || !make_map(&mV, a.V, D, N, BH, kBtcTile))
     return cudaErrorInvalidValue;
   BwdTcArgs t;
