@@ -69,7 +69,7 @@ struct BtcCfg {
   static constexpr int kTokBytes = G::bytes(kBtcTile);
   static constexpr int kOffLat = 0;                        // Q_dyn, Z, dZ, Q~, dQ_dyn
   static constexpr int kOffTok = 5 * kLatBytes;            // K, dY, V
-  static constexpr int kOffStats = kOffTok + 3 * kTokBytes;  // L1, L2, C1, C2 [kMPad]
+  static constexpr int kOffStats = kOffTok + 3 * kTokBytes;  // float4 {L1, L2, c1, c2} [kMPad]
   static constexpr int kOffBars = kOffStats + 4 * kMPad * 4;
   static constexpr int kNumBars = 10;
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
@@ -113,10 +113,7 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
   uint64_t* bar_acc = bars + 6;   // last accumulation of a tile done
   uint64_t* bar_free = bars + 7;  // dK, dV of a tile read out (4 warps)
   uint64_t* drain = bars + 8;
-  float* sL1 = reinterpret_cast<float*>(smem + C::kOffStats);
-  float* sL2 = sL1 + C::kMPad;
-  float* sC1 = sL2 + C::kMPad;
-  float* sC2 = sC1 + C::kMPad;
+  float4* sStat = reinterpret_cast<float4*>(smem + C::kOffStats);  // per latent {L1, L2, c1, c2}
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
 
@@ -146,10 +143,9 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
   constexpr float kL2e = 1.4426950408889634f;
   for (int m = threadIdx.x; m < C::kMPad; m += blockDim.x) {
     const bool live = m < args.M;
-    sL1[m] = live ? args.lse1[lat_base + m] * kL2e : INFINITY;
-    sL2[m] = live ? args.lse2[lat_base + m] * kL2e : INFINITY;
-    sC1[m] = live ? args.c1[lat_base + m] : 0.f;
-    sC2[m] = live ? args.c2[lat_base + m] : 0.f;
+    sStat[m] = live ? make_float4(args.lse1[lat_base + m] * kL2e, args.lse2[lat_base + m] * kL2e, args.c1[lat_base + m],
+                                  args.c2[lat_base + m])
+                    : make_float4(INFINITY, INFINITY, 0.f, 0.f);
   }
   if (warp == C::kIssuerWarp) {
     ptx::tmem_alloc(s_tmem, 512);
@@ -301,11 +297,12 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
             for (int e = 0; e < 2; ++e) {
               const int j = 2 * u + e;
               const int m = c * kBtcChunk + hh * 16 + j;
+              const float4 st = sStat[m];
               const float p3 = m < args.M ? ptx::ex2(fmaf(s3[j], kL2e, -L3)) : 0.f;
-              const float a2 = ptx::ex2(fmaf(s3[j], kL2e, -sL2[m]));
-              const float a1 = ptx::ex2(fmaf(s1[j], kL2e, -sL1[m]));
-              q[e] = fmaf(p3, dp[j] - dl, a2 * (da2[j] - sC2[m]));
-              sd[e] = a1 * (da1[j] - sC1[m]);
+              const float a2 = ptx::ex2(fmaf(s3[j], kL2e, -st.y));
+              const float a1 = ptx::ex2(fmaf(s1[j], kL2e, -st.x));
+              q[e] = fmaf(p3, dp[j] - dl, a2 * (da2[j] - st.w));
+              sd[e] = a1 * (da1[j] - st.z);
               z[e] = a2;
               dq[e] = a1;
             }
@@ -552,13 +549,15 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
     for (int i = 0; ok && i < T; ++i) {
       const long long t0 = static_cast<long long>(tile0 + i) * kBltcTok;
       const int live_cols = static_cast<int>(args.N - t0 < kBltcTok ? args.N - t0 : kBltcTok);
-      float* stat = sTok + (i & 1) * 2 * kBltcTok;
+      float2* stat = reinterpret_cast<float2*>(sTok) + (i & 1) * kBltcTok;  // {lse3 log2 domain, delta}
       if constexpr (kDec) {
-        // lse3 (log2 domain) and delta of the tile's tokens, shared by the 128 rows
-        const int j = threadIdx.x & (kBltcTok - 1);
-        const bool live = j < live_cols;
-        stat[threadIdx.x] = threadIdx.x < kBltcTok ? (live ? args.lse3[tok_base + t0 + j] * kL2e : 0.f)
-                                                   : (live ? args.delta[tok_base + t0 + j] : 0.f);
+        // the tile's token statistics, shared by the 128 rows
+        if (threadIdx.x < kBltcTok) {
+          const int j = threadIdx.x;
+          const bool live = j < live_cols;
+          stat[j] = live ? make_float2(args.lse3[tok_base + t0 + j] * kL2e, args.delta[tok_base + t0 + j])
+                         : make_float2(0.f, 0.f);
+        }
         asm volatile("bar.sync 1, 128;" ::: "memory");
       }
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_S, i & 1, s_abort, args.wait_ns));
@@ -579,8 +578,9 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
             const int j = 16 * p + 2 * u + q;
             float ee, ww;
             if constexpr (kDec) {
-              ee = ptx::ex2(fmaf(sv[2 * u + q], kL2e, -stat[j]));
-              ww = ee * (gv[2 * u + q] - stat[kBltcTok + j]);
+              const float2 tj = stat[j];
+              ee = ptx::ex2(fmaf(sv[2 * u + q], kL2e, -tj.x));
+              ww = ee * (gv[2 * u + q] - tj.y);
             } else {
               ee = ptx::ex2(fmaf(sv[2 * u + q], kL2e, -Lm));
               ww = ee * (gv[2 * u + q] - cm);
