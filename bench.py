@@ -52,7 +52,7 @@ sys.path.insert(0, ROOT)
 
 METRIC = "FLARE++ mixer fwd tokens/s & TFLOP/s (bf16) at N=1M, M=256; % of roofline"
 WORKLOAD = "million"
-CPU_SAMPLE_TOKENS = 1 << 18  # cpu_baseline sample: one head, its first 262144 tokens (~10 s)
+CPU_SAMPLE_TOKENS = 1 << 20  # cpu_baseline sample: one whole head, 1,048,576 tokens (~8 s on 16 cores)
 REFERENCE_BUDGET_S = 150.0   # the reference arm's K + W steps together
 
 
