@@ -479,6 +479,18 @@ def run_native(args):
     roof["kernel"] = "encode_tc"
     roof["ms_per_launch"] = enc_ms
     roof["peak_source"] = f"{peak_kind} (sustained bf16 GEMM / STREAM copy)"
+    # The exponential unit binds in practice: one 2^x per score, N*M per head
+    # per encode launch, at 16 results per clock per SM (MUFU ex2) on 148 SMs.
+    # Peak at the maximum SM clock; frac_at_clock uses the median SM clock
+    # sampled under load (the kernels run power-capped).
+    clk = clocks.summary()
+    exps = float(w.N) * w.M * w.H
+    alu_peak = 16.0 * 148 * (clk["sm_max_mhz"] or 1965.0) * 1e6  # 1965 MHz: the B200's clocks.max.sm
+    alu_at_clock = 16.0 * 148 * clk["sm_mhz"] * 1e6 if clk.get("sm_mhz") else None
+    alu_roof = {"bound": "alu", "kernel": "encode_tc", "unit": "exp/s", "achieved": exps / (enc_ms * 1e-3),
+                "peak": alu_peak, "frac": exps / (enc_ms * 1e-3) / alu_peak,
+                "frac_at_clock": exps / (enc_ms * 1e-3) / alu_at_clock if alu_at_clock else None,
+                "per_launch": exps, "what": "exponentials of the encode (1/16 of them on the FMA pipe)"}
     line = {
         "metric": METRIC,
         "value": value,
@@ -499,6 +511,7 @@ def run_native(args):
         "step_roofline": {"t_roofline_ms": max(t_tensor, t_hbm) * 1e3, "bound": "tensor" if t_tensor >= t_hbm else "hbm",
                           "frac": max(t_tensor, t_hbm) * 1e3 / ms, "peaks": peak_kind},
         "roofline": roof,
+        "alu_roofline": alu_roof,
         "kernel_ms_per_step": step_kernel_ms,
         "decode_ms_per_launch": dec_ms,
         "gpu_launches": launches_per_step * args.steps,
