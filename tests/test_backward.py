@@ -43,6 +43,9 @@ CASES = [
     ("custom", (3, 2, 1, 16, 16, "bf16")),      # N = 1: dV = dY, the rest 0
     ("custom", (1, 1, 100, 1, 16, "f32")),      # M = 1
     ("custom", (2, 2, 257, 64, 64, "bf16")),
+    ("custom", (2, 2, 300, 48, 32, "bf16")),    # tensor cores, M not a multiple of 32
+    ("custom", (1, 3, 1000, 16, 64, "bf16")),   # one 16-latent chunk
+    ("custom", (1, 2, 700, 256, 64, "bf16")),   # both latent halves, the benchmark's M and D
 ]
 
 
