@@ -287,3 +287,4 @@ def flarepp_backward(seeds, K, V, dY, Q_dyn=None, Z=None):
             d_seeds[h] += g[0]
             dK[b, h], dV[b, h] = g[1], g[2]
     return d_seeds, dK, dV
+

@@ -317,15 +317,28 @@ __global__ void __launch_bounds__(kBwdThreads) grad_reduce_kernel(const BwdArgs 
         if constexpr (MODE == kBwdDec) v0 += a.part[a.part_stride + i];
       }
       const size_t o = (static_cast<size_t>(head) * a.M + m) * D + d;
+      // With bf16 copies (the tensor-core kernels take dZ V^T and dQ_dyn V^T
+      // from them), the row terms c2 = dZ . Z and c1 = dQ_dyn . Q_dyn use the
+      // same rounded values: then each softmax-gradient row still sums to
+      // zero (sum_n A (dA - c) = 0 when c = sum_n A dA), and the rounding of
+      // dZ and dQ_dyn is not amplified by the cancellation between dA and c.
       if constexpr (MODE == kBwdDec) {
         a.dQd[o] = v;
         a.dZ[o] = v0;
-        if (a.dZ16) a.dZ16[o] = __float2bfloat16_rn(v0);
+        if (a.dZ16) {
+          const __nv_bfloat16 r = __float2bfloat16_rn(v0);
+          a.dZ16[o] = r;
+          v0 = __bfloat162float(r);
+        }
         dot = fmaf(v0, ld_f32(static_cast<const T*>(a.Z) + o), dot);
       } else {
         v += a.dQd[o];
         a.dQd[o] = v;
-        if (a.dQd16) a.dQd16[o] = __float2bfloat16_rn(v);
+        if (a.dQd16) {
+          const __nv_bfloat16 r = __float2bfloat16_rn(v);
+          a.dQd16[o] = r;
+          v = __bfloat162float(r);
+        }
         dot = fmaf(v, ld_f32(static_cast<const T*>(a.Qd) + o), dot);
       }
     }
