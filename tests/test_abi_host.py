@@ -16,7 +16,7 @@ def L():
     return flare.lib()
 
 
-def test_header_declares_the_north_star_calls():
+def test_header_declares_the_mixer_calls():
     names = flare.header_functions()
     for n in ("flare_encode", "flare_decode", "flarepp_mix"):
         assert n in names
