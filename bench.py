@@ -31,7 +31,9 @@ the data path.  Rank 0 prints one JSON line:
   latent (O, lse) per encode, combine, local decode.  With N = 1 it is the
   same cloud as the headline on one GPU, through the sharded path;
 * backward: flarepp_mix_backward (gradients of the seeds, K and V for a
-  seeded N(0,1) dY) on the same inputs, with its per-kernel split.
+  seeded N(0,1) dY) on the same inputs, with its per-kernel split, and
+  the same backward reading the state flarepp_mix_save kept
+  (saved_state_ms_per_step).
 
 --impl reference times the oracle (the reference arm of this comparison) on
 the host cores, rank 0 only, and prints the same line with "impl": "reference".
@@ -420,7 +422,26 @@ def run_native(args):
     st = flare.flare_check_status()
     if st != (0, 0):
         raise RuntimeError(f"device status after the backward steps: {st}")
-    del dY, grads, wsb
+    # the training-step form: the forward keeps Q_dyn, Z and the encodes'
+    # log-sum-exps, and the backward reads them instead of recomputing
+    _, saved = flare.flarepp_mix_save(s_d, K_d, V_d, Y_d)
+
+    def bwd_saved_step():
+        flare.flarepp_mix_backward_saved(s_d, K_d, V_d, dY, saved, *grads, workspace=wsb)
+
+    for _ in range(2):
+        bwd_saved_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(nb):
+        bwd_saved_step()
+    ev1.record(stream)
+    barrier()
+    bwd_saved_ms = max_over_ranks(ev0.elapsed_time(ev1)) / nb
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after the saved-state backward steps: {st}")
+    del dY, grads, wsb, saved
 
     # ---- end to end: pinned host inputs, copies inside the timed region
     Y_host = torch.empty(K_h.shape, dtype=torch.bfloat16).pin_memory()
@@ -525,7 +546,8 @@ def run_native(args):
         "backward": {"ms_per_step": bwd_ms, "tokens_per_s": ranks.job_tokens_per_s(w.N, env, bwd_ms), "steps": nb,
                      "launches": bwd_launches, "kernel_ms": bwd_split,
                      "executed_gemm_tflops": 25 * 2.0 * w.N * w.M * w.D * w.H / (bwd_ms * 1e-3) / 1e12,
-                     "what": "d_seeds, dK, dV of sum(dY * Y); two recomputed encodes + eight kernels"},
+                     "what": "d_seeds, dK, dV of sum(dY * Y); two recomputed encodes + eight kernels",
+                     "saved_state_ms_per_step": bwd_saved_ms},
         "communication_matrix": {"ms_per_call": comm_ms, "launches": comm_launches,
                                  "what": "C = softmax_N(Q_dyn K^T) softmax_M(K Q_dyn^T), M x M per head"},
         "e2e": {"value": ranks.job_tokens_per_s(w.N, env, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,

@@ -174,6 +174,27 @@ size_t flare_encode_lse_workspace_size(int B, int H, int64_t N, int M, int D, in
  * workspace comes from flarepp_mix_backward_workspace_size.
  */
 size_t flarepp_mix_backward_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+
+/*
+ * Forward and backward with saved state, as a training step runs them:
+ * flarepp_mix_save is flarepp_mix that also keeps what the backward needs,
+ * and flarepp_mix_backward_saved is flarepp_mix_backward without its two
+ * recomputed encodes (it reads that state instead).
+ *   saved      device buffer of flarepp_saved_bytes(B, H, M, D, dtype) bytes,
+ *              256-byte aligned, owned by the caller; holds, each region
+ *              256-byte aligned: Q_dyn and Z [B][H][M][D] (dtype) as the
+ *              forward stored them, then lse1 and lse2 [B][H][M] fp32 (the
+ *              seed and routing encodes' log-sum-exps, natural log).
+ * The gradients equal flarepp_mix_backward's bit for bit when the forward
+ * ran on the same inputs.  dtype FLARE_BF16 or FLARE_F32; workspaces as
+ * flarepp_mix and flarepp_mix_backward.
+ */
+size_t flarepp_saved_bytes(int B, int H, int M, int D, int dtype);
+int flarepp_mix_save(const void* seeds, const void* K, const void* V, void* Y, void* saved, int B, int H, int64_t N,
+                     int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream);
+int flarepp_mix_backward_saved(const void* seeds, const void* K, const void* V, const void* dY, const void* saved,
+                               void* d_seeds, void* dK, void* dV, int B, int H, int64_t N, int M, int D, int dtype,
+                               void* workspace, size_t workspace_bytes, void* stream);
 int flarepp_mix_backward(const void* seeds, const void* K, const void* V, const void* dY, void* d_seeds, void* dK,
                          void* dV, int B, int H, int64_t N, int M, int D, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream);

@@ -33,6 +33,9 @@ __all__ = [
     "flare_lse_combine",
     "flarepp_mix_backward",
     "flarepp_mix_backward_workspace_size",
+    "flarepp_mix_save",
+    "flarepp_mix_backward_saved",
+    "flarepp_saved_bytes",
     "flarepp_workspace_size",
     "flarepp_mix_host",
     "flare_communication_matrix",
@@ -63,6 +66,9 @@ _SIGNATURES = {
     "flare_encode_lse_workspace_size": (_c_size, _SIZES),
     "flarepp_mix_backward_workspace_size": (_c_size, _SIZES),
     "flarepp_mix_backward": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
+    "flarepp_saved_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
+    "flarepp_mix_save": (_c_int, [_vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
+    "flarepp_mix_backward_saved": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_encode_lse": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_lse_combine": (_c_int, [_vp, _vp, _c_int, _c_i64, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                    _vp]),
@@ -272,6 +278,51 @@ def flarepp_mix_backward(seeds, K, V, dY, d_seeds=None, dK=None, dV=None, *, wor
                                       _ptr(dV, "dV", dt), B, H, N, M, D, _dtype_code(K), ws, wsb,
                                       _stream(stream)),
            "flarepp_mix_backward")
+    return d_seeds, dK, dV
+
+
+def flarepp_saved_bytes(B, H, M, D, dtype) -> int:
+    code = dtype if isinstance(dtype, int) else (BF16 if "bfloat16" in str(dtype) else F32)
+    return lib().flarepp_saved_bytes(B, H, M, D, code)
+
+
+def flarepp_mix_save(seeds, K, V, Y=None, saved=None, *, workspace=None, stream=None):
+    """flarepp_mix that also keeps the backward's state (Q_dyn, Z and the two
+    encodes' log-sum-exps) in `saved`, a uint8 CUDA tensor of
+    flarepp_saved_bytes bytes.  Returns (Y, saved)."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = seeds.shape[-2]
+    if Y is None:
+        Y = torch.empty_like(K)
+    if saved is None:
+        saved = torch.empty(flarepp_saved_bytes(B, H, M, D, K.dtype), dtype=torch.uint8, device=K.device)
+    ws, wsb = _ws(workspace)
+    dt = K.dtype
+    _check(lib().flarepp_mix_save(_ptr(seeds, "seeds", dt), _ptr(K, "K", dt), _ptr(V, "V", dt), _ptr(Y, "Y", dt),
+                                  _ptr(saved, "saved", torch.uint8), B, H, N, M, D, _dtype_code(K), ws, wsb,
+                                  _stream(stream)),
+           "flarepp_mix_save")
+    return Y, saved
+
+
+def flarepp_mix_backward_saved(seeds, K, V, dY, saved, d_seeds=None, dK=None, dV=None, *, workspace=None,
+                               stream=None):
+    """flarepp_mix_backward reading Q_dyn, Z and the log-sum-exps that
+    flarepp_mix_save kept instead of recomputing the two encodes."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = seeds.shape[-2]
+    d_seeds = torch.empty_like(seeds) if d_seeds is None else d_seeds
+    dK = torch.empty_like(K) if dK is None else dK
+    dV = torch.empty_like(V) if dV is None else dV
+    ws, wsb = _ws(workspace)
+    dt = K.dtype
+    _check(lib().flarepp_mix_backward_saved(_ptr(seeds, "seeds", dt), _ptr(K, "K", dt), _ptr(V, "V", dt),
+                                            _ptr(dY, "dY", dt), _ptr(saved, "saved", torch.uint8),
+                                            _ptr(d_seeds, "d_seeds", dt), _ptr(dK, "dK", dt), _ptr(dV, "dV", dt),
+                                            B, H, N, M, D, _dtype_code(K), ws, wsb, _stream(stream)),
+           "flarepp_mix_backward_saved")
     return d_seeds, dK, dV
 
 

@@ -425,7 +425,8 @@ int release_scratch(const Scratch& s, cudaStream_t st) {
 }
 
 int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_out, void* Z_out, int B, int H,
-             int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+             int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream,
+             float* lse1_out = nullptr, float* lse2_out = nullptr) {
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (!device_ptr(seeds) || !device_ptr(K) || !device_ptr(V) || !device_ptr(Y)) return FLARE_ERR_INVALID_ARG;
@@ -441,8 +442,8 @@ int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_
   void* Qd = Qd_out ? Qd_out : s.ptr + enc;
   void* Z = Z_out ? Z_out : s.ptr + enc + lat;
   int launches = 0;
-  rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, /*q_bf16=*/true);
-  if (!rc) rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, /*q_bf16=*/true, lse1_out);
+  if (!rc) rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out);
   if (!rc) rc = run_decode(K, Qd, 1, Z, Y, B, H, N, M, D, dtype, st, &launches);
   const int rc2 = release_scratch(s, st);
   if (!rc) {
@@ -813,16 +814,56 @@ cudaError_t launch_backward_t(int D, const BwdArgs& a, const BackwardWs& w, int 
   }
 }
 
+// What flarepp_mix_save keeps for the backward, in order, each region
+// 256-byte aligned: Q_dyn [B][H][M][D] and Z (dtype), lse1 and lse2
+// [B][H][M] fp32 (the two encodes' log-sum-exps, natural log).
+struct SavedLayout {
+  void* Qd;
+  void* Z;
+  float* lse1;
+  float* lse2;
+  size_t bytes;
+};
+
+SavedLayout saved_layout(void* base, int BH, int M, int D, int dtype) {
+  SavedLayout l;
+  const size_t lat = static_cast<size_t>(BH) * M;
+  const size_t esz = dtype == FLARE_BF16 ? 2 : 4;
+  char* p = static_cast<char*>(base);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    char* q = p ? p + off : nullptr;
+    off += align256(bytes);
+    return q;
+  };
+  l.Qd = take(lat * D * esz);
+  l.Z = take(lat * D * esz);
+  l.lse1 = reinterpret_cast<float*>(take(lat * 4));
+  l.lse2 = reinterpret_cast<float*>(take(lat * 4));
+  l.bytes = off;
+  return l;
+}
+
 int run_backward(const void* seeds, const void* K, const void* V, const void* dY, void* d_seeds, void* dK, void* dV,
-                 int B, int H, int64_t N, int M, int D, int dtype, char* ws, cudaStream_t st, int* launches) {
+                 int B, int H, int64_t N, int M, int D, int dtype, char* ws, cudaStream_t st, int* launches,
+                 void* saved = nullptr) {
   const int BH = B * H;
-  const BackwardWs w = backward_ws_layout(ws, BH, N, M, D, dtype);
-  // the forward's encodes again, for Q_dyn and Z as it stored them and their
-  // per-latent log-sum-exps
-  int rc = run_encode(seeds, 0, K, V, w.Qd, B, H, N, M, D, dtype, w.enc, st, launches, false, w.lse1);
-  if (rc) return rc;
-  rc = run_encode(w.Qd, 1, K, V, w.Z, B, H, N, M, D, dtype, w.enc, st, launches, false, w.lse2);
-  if (rc) return rc;
+  BackwardWs w = backward_ws_layout(ws, BH, N, M, D, dtype);
+  if (saved) {
+    // Q_dyn, Z and the encodes' log-sum-exps as flarepp_mix_save kept them
+    const SavedLayout l = saved_layout(saved, BH, M, D, dtype);
+    w.Qd = l.Qd;
+    w.Z = l.Z;
+    w.lse1 = l.lse1;
+    w.lse2 = l.lse2;
+  } else {
+    // the forward's encodes again, for Q_dyn and Z as it stored them and
+    // their per-latent log-sum-exps
+    int rc = run_encode(seeds, 0, K, V, w.Qd, B, H, N, M, D, dtype, w.enc, st, launches, false, w.lse1);
+    if (rc) return rc;
+    rc = run_encode(w.Qd, 1, K, V, w.Z, B, H, N, M, D, dtype, w.enc, st, launches, false, w.lse2);
+    if (rc) return rc;
+  }
   BwdArgs a;
   a.N = static_cast<int>(N);
   a.M = M;
@@ -995,6 +1036,46 @@ int flarepp_mix_backward(const void* seeds, const void* K, const void* V, const 
   if (rc) return rc;
   int launches = 0;
   rc = run_backward(seeds, K, V, dY, d_seeds, dK, dV, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  const int rc2 = release_scratch(s, st);
+  if (!rc) {
+    rc = rc2;
+    t_last_launches = launches;
+  }
+  return rc;
+}
+
+size_t flarepp_saved_bytes(int B, int H, int M, int D, int dtype) {
+  if (check_sizes(B, H, 1, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
+  return saved_layout(nullptr, B * H, M, D, dtype).bytes;
+}
+
+int flarepp_mix_save(const void* seeds, const void* K, const void* V, void* Y, void* saved, int B, int H, int64_t N,
+                     int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  if (!device_ptr(saved)) return FLARE_ERR_INVALID_ARG;
+  const SavedLayout l = saved_layout(saved, B * H, M, D, dtype);
+  return mix_impl(seeds, K, V, Y, l.Qd, l.Z, B, H, N, M, D, dtype, workspace, workspace_bytes, stream, l.lse1, l.lse2);
+}
+
+int flarepp_mix_backward_saved(const void* seeds, const void* K, const void* V, const void* dY, const void* saved,
+                               void* d_seeds, void* dK, void* dV, int B, int H, int64_t N, int M, int D, int dtype,
+                               void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_sizes(B, H, N, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  for (const void* p : {seeds, K, V, dY, saved, static_cast<const void*>(d_seeds), static_cast<const void*>(dK),
+                        static_cast<const void*>(dV)})
+    if (!device_ptr(p)) return FLARE_ERR_INVALID_ARG;
+  if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  Scratch s;
+  rc = get_scratch(workspace, workspace_bytes, backward_ws_layout(nullptr, B * H, N, M, D, dtype).bytes, st, &s);
+  if (rc) return rc;
+  int launches = 0;
+  rc = run_backward(seeds, K, V, dY, d_seeds, dK, dV, B, H, N, M, D, dtype, s.ptr, st, &launches,
+                    const_cast<void*>(saved));
   const int rc2 = release_scratch(s, st);
   if (!rc) {
     rc = rc2;

@@ -118,3 +118,35 @@ def test_workspace_and_stream():
     small = torch.empty(nbytes - 256, dtype=torch.uint8, device="cuda")
     with pytest.raises(flare.FlareError):
         flare.flarepp_mix_backward(*dev, workspace=small)
+
+
+@pytest.mark.parametrize("dtype,sizes", [("bf16", (2, 2, 300, 48, 32)), ("bf16", (1, 2, 700, 256, 64)),
+                                         ("f32", (1, 2, 333, 30, 16)), ("bf16", (1, 1, 200, 64, 128))])
+def test_saved_state_matches_recompute(dtype, sizes):
+    """flarepp_mix_save + flarepp_mix_backward_saved: the same Y as flarepp_mix,
+    the same Q_dyn and Z as flarepp_mix_debug, and the same gradients as
+    flarepp_mix_backward, bit for bit; two fewer launches."""
+    import torch
+
+    require_cuda()
+    B, H, N, M, D = sizes
+    w = inputs.custom(B, H, N, M, D, dtype=dtype, seed_index=80 + M)
+    seeds, K, V = inputs.make_inputs(w)
+    dY = inputs.make_upstream(w)
+    dev = [to_dev(x, dtype) for x in (seeds, K, V, dY)]
+    Y, saved = flare.flarepp_mix_save(*dev[:3])
+    assert saved.numel() == flare.flarepp_saved_bytes(B, H, M, D, dev[1].dtype)
+    assert torch.equal(Y, flare.flarepp_mix(*dev[:3]))
+    Yd, Qd, Z = flare.flarepp_mix_debug(*dev[:3])
+    esz = 2 if dtype == "bf16" else 4
+    n = B * H * M * D * esz
+    region = (n + 255) // 256 * 256
+    assert torch.equal(saved[:n], Qd.reshape(-1).view(torch.uint8))
+    assert torch.equal(saved[region:region + n], Z.reshape(-1).view(torch.uint8))
+    g_saved = flare.flarepp_mix_backward_saved(*dev, saved)
+    launches_saved = flare.flare_last_launch_count()
+    g_full = flare.flarepp_mix_backward(*dev)
+    assert flare.flare_last_launch_count() == launches_saved + 4  # two encodes and their merges
+    for a, b in zip(g_saved, g_full):
+        assert torch.equal(a, b)
+    assert flare.flare_check_status() == (0, 0)
