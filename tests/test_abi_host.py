@@ -75,6 +75,25 @@ def test_workspace_sizes(L):
     assert a - b >= 2 * 16 * 256 * 64 * 2
 
 
+def test_backward_and_shard_sizes(L):
+    # saved state: Q_dyn and Z (dtype) then two fp32 log-sum-exps, each region 256-byte aligned
+    def r(x):
+        return (x + 255) // 256 * 256
+    BH, M, D = 16, 256, 64
+    assert L.flarepp_saved_bytes(1, 16, M, D, BF16) == 2 * r(BH * M * D * 2) + 2 * r(BH * M * 4)
+    assert L.flarepp_saved_bytes(1, 16, M, D, F32) == 2 * r(BH * M * D * 4) + 2 * r(BH * M * 4)
+    assert L.flarepp_saved_bytes(1, 1, 17, 64, BF16) == 0          # bf16 needs M % 16 == 0
+    assert L.flarepp_saved_bytes(1, 1, 16, 64, 2) == 0             # fp32-output mode has no backward
+    wb = L.flarepp_mix_backward_workspace_size(1, 16, 1 << 20, M, D, BF16)
+    # it holds the encode workspace, the per-token statistics (8 bytes a token) and more
+    assert wb % 256 == 0 and wb > L.flare_encode_workspace_size(1, 16, 1 << 20, M, D, BF16) + 8 * BH * (1 << 20)
+    assert L.flarepp_mix_backward_workspace_size(1, 1, 0, 16, 16, BF16) == 0
+    # a token shard with no tokens needs no workspace; otherwise as the encode
+    assert L.flare_encode_lse_workspace_size(1, 2, 0, 64, 32, BF16) == 0
+    assert L.flare_encode_lse_workspace_size(1, 2, 5000, 64, 32, BF16) == L.flare_encode_workspace_size(
+        1, 2, 5000, 64, 32, BF16)
+
+
 def test_option_hooks_round_trip(L):
     old = L.flare_set_split_override(5)
     assert L.flare_set_split_override(old) == 5
