@@ -190,6 +190,33 @@ size_t flarepp_mix_backward_workspace_size(int B, int H, int64_t N, int M, int D
  * flarepp_mix and flarepp_mix_backward.
  */
 size_t flarepp_saved_bytes(int B, int H, int M, int D, int dtype);
+
+/*
+ * Token-sharded backward (training with the tokens of one cloud spread over
+ * ranks, as in the FLARE++ page's context-parallel item, "Contributions
+ * Clés").  Each rank holds its tokens' K, V, dY and the replicated state of
+ * the sharded forward (`saved`: Q_dyn, Z, lse1, lse2 of the whole cloud, as
+ * flarepp_mix_save lays them out).  The backward's token reductions (dZ,
+ * dQ_dyn, d_seeds) need every rank's tokens, so it runs in four phases;
+ * between phases the caller sums `exchange` over the ranks (an all-reduce):
+ *   phase 0: statistics and the decode pass; exchange = [dZ | dQ_dyn decode
+ *            part], 2 x [B][H][M][D] fp32
+ *   phase 1: routing pass; exchange = dQ_dyn routing part, [B][H][M][D]
+ *   phase 2: seed pass; exchange = d_seeds, [H][M][D] fp32
+ *   phase 3: d_seeds (dtype, the summed value) and this rank's dK, dV
+ * N is this rank's token count (0 allowed: the rank contributes zeros).
+ * The workspace (flarepp_backward_shard_workspace_size bytes) must be the
+ * same buffer in all four calls and is required; exchange holds at least
+ * flarepp_backward_shard_exchange_floats floats.  With one rank and no
+ * exchange between phases the result equals flarepp_mix_backward_saved's
+ * bit for bit.
+ */
+size_t flarepp_backward_shard_exchange_floats(int B, int H, int M, int D);
+size_t flarepp_backward_shard_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
+int flarepp_mix_backward_shard(int phase, const void* seeds, const void* K, const void* V, const void* dY,
+                               const void* saved, float* exchange, void* d_seeds, void* dK, void* dV, int B, int H,
+                               int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes,
+                               void* stream);
 int flarepp_mix_save(const void* seeds, const void* K, const void* V, void* Y, void* saved, int B, int H, int64_t N,
                      int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream);
 int flarepp_mix_backward_saved(const void* seeds, const void* K, const void* V, const void* dY, const void* saved,

@@ -36,6 +36,7 @@ __all__ = [
     "flarepp_mix_save",
     "flarepp_mix_backward_saved",
     "flarepp_saved_bytes",
+    "flarepp_mix_backward_shard",
     "flarepp_workspace_size",
     "flarepp_mix_host",
     "flare_communication_matrix",
@@ -69,6 +70,10 @@ _SIGNATURES = {
     "flarepp_saved_bytes": (_c_size, [_c_int, _c_int, _c_int, _c_int, _c_int]),
     "flarepp_mix_save": (_c_int, [_vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flarepp_mix_backward_saved": (_c_int, [_vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
+    "flarepp_backward_shard_exchange_floats": (_c_size, [_c_int, _c_int, _c_int, _c_int]),
+    "flarepp_backward_shard_workspace_size": (_c_size, _SIZES),
+    "flarepp_mix_backward_shard": (_c_int, [_c_int, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, _vp, *_SIZES, _vp,
+                                            _c_size, _vp]),
     "flare_encode_lse": (_c_int, [_vp, _c_int, _vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_lse_combine": (_c_int, [_vp, _vp, _c_int, _c_i64, _vp, _vp, _c_int, _c_int, _c_int, _c_int, _c_int,
                                    _vp]),
@@ -324,6 +329,27 @@ def flarepp_mix_backward_saved(seeds, K, V, dY, saved, d_seeds=None, dK=None, dV
                                             B, H, N, M, D, _dtype_code(K), ws, wsb, _stream(stream)),
            "flarepp_mix_backward_saved")
     return d_seeds, dK, dV
+
+
+def flarepp_mix_backward_shard(phase, seeds, K, V, dY, saved, exchange, d_seeds, dK, dV, workspace, *,
+                               stream=None):
+    """One phase (0-3) of the token-sharded backward for this rank's tokens
+    K, V, dY [B,H,N_r,D] (N_r may be 0).  `saved` is the whole cloud's state
+    (uint8, flarepp_mix_save's layout), `exchange` an fp32 buffer the caller
+    sums over the ranks between phases, `workspace` a uint8 buffer kept for
+    all four phases.  d_seeds is written in phase 3, dK and dV too."""
+    torch = _torch()
+    B, H, N, D = K.shape
+    M = seeds.shape[-2]
+    dt = seeds.dtype
+    kv = (None,) * 5 if N == 0 else (_ptr(K, "K", dt), _ptr(V, "V", dt), _ptr(dY, "dY", dt), _ptr(dK, "dK", dt),
+                                     _ptr(dV, "dV", dt))
+    _check(lib().flarepp_mix_backward_shard(phase, _ptr(seeds, "seeds", dt), kv[0], kv[1], kv[2],
+                                            _ptr(saved, "saved", torch.uint8), _ptr(exchange, "exchange", torch.float32),
+                                            _ptr(d_seeds, "d_seeds", dt), kv[3], kv[4], B, H, N, M, D,
+                                            _dtype_code(seeds), ctypes.c_void_p(workspace.data_ptr()),
+                                            workspace.numel(), _stream(stream)),
+           "flarepp_mix_backward_shard")
 
 
 def flarepp_mix_host(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, stream=None):

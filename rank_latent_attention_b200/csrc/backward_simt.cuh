@@ -98,6 +98,8 @@ struct BwdArgs {
   __nv_bfloat16* dZ16;   // [BH][M][D] bf16 copies of dZ and dQ_dyn for tensor-core
   __nv_bfloat16* dQd16;  // operands (null when the CUDA-core token kernel runs)
   float* part;        // [BH][S][M][D] x 2 (second block at part + part_stride)
+  float* exch;        // token-sharded backward: the sums each rank contributes, summed over ranks
+                      // between phases ([BH][M][D] x 2 after the decode pass, then x 1, then [H][M][D])
   long long part_stride;
   int S;              // token splits of the latent-row kernels
   void* d_seeds;      // [H][M][D]
@@ -294,7 +296,13 @@ __global__ void __launch_bounds__(kBwdThreads) latent_grad_kernel(const BwdArgs 
 //                         c2 = dZ . Z
 //   ROUTING (heads = BH): dQ_dyn += sum_s part1, c1 = dQ_dyn . Q_dyn
 //   SEED    (heads = H):  d_seeds[h] = sum_b sum_s part1   (stored as T)
-template <int D, typename T, int MODE>
+// STAGE 0 does it in one go.  A token-sharded backward splits it around the
+// sum over ranks: STAGE 1 writes this rank's sums to the exchange buffer
+// (DEC: dZ then dQ_dyn), and after the caller has summed that buffer over the
+// ranks, STAGE 2 takes the sums from it and does the rest.
+enum BwdStage { kStageFused = 0, kStageLocal = 1, kStageFinish = 2 };
+
+template <int D, typename T, int MODE, int STAGE>
 __global__ void __launch_bounds__(kBwdThreads) grad_reduce_kernel(const BwdArgs a, int B) {
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int m = blockIdx.x * 8 + warp;
@@ -304,19 +312,46 @@ __global__ void __launch_bounds__(kBwdThreads) grad_reduce_kernel(const BwdArgs 
   for (int d = lane; d < D; d += 32) {
     float v = 0.f, v0 = 0.f;
     if constexpr (MODE == kBwdEncSeed) {
-      for (int b = 0; b < B; ++b) {
-        const size_t row0 = (static_cast<size_t>(b * a.H + head) * a.S) * a.M + m;
-        for (int s = 0; s < a.S; ++s) v += a.part[(row0 + static_cast<size_t>(s) * a.M) * D + d];
-      }
-      st_from_f32(static_cast<T*>(a.d_seeds) + (static_cast<size_t>(head) * a.M + m) * D + d, v);
-    } else {
-      const size_t row0 = static_cast<size_t>(head) * a.S * a.M + m;
-      for (int s = 0; s < a.S; ++s) {
-        const size_t i = (row0 + static_cast<size_t>(s) * a.M) * D + d;
-        v += a.part[i];
-        if constexpr (MODE == kBwdDec) v0 += a.part[a.part_stride + i];
-      }
       const size_t o = (static_cast<size_t>(head) * a.M + m) * D + d;
+      if constexpr (STAGE == kStageFinish) {
+        v = a.exch[o];
+      } else {
+        for (int b = 0; b < B; ++b) {
+          const size_t row0 = (static_cast<size_t>(b * a.H + head) * a.S) * a.M + m;
+          for (int s = 0; s < a.S; ++s) v += a.part[(row0 + static_cast<size_t>(s) * a.M) * D + d];
+        }
+      }
+      if constexpr (STAGE == kStageLocal)
+        a.exch[o] = v;
+      else
+        st_from_f32(static_cast<T*>(a.d_seeds) + o, v);
+    } else {
+      const size_t o = (static_cast<size_t>(head) * a.M + m) * D + d;
+      const size_t L = static_cast<size_t>(gridDim.y) * a.M * D;  // one [BH][M][D] block
+      if constexpr (STAGE == kStageFinish) {
+        if constexpr (MODE == kBwdDec) {
+          v0 = a.exch[o];
+          v = a.exch[L + o];
+        } else {
+          v = a.exch[o];
+        }
+      } else {
+        const size_t row0 = static_cast<size_t>(head) * a.S * a.M + m;
+        for (int s = 0; s < a.S; ++s) {
+          const size_t i = (row0 + static_cast<size_t>(s) * a.M) * D + d;
+          v += a.part[i];
+          if constexpr (MODE == kBwdDec) v0 += a.part[a.part_stride + i];
+        }
+      }
+      if constexpr (STAGE == kStageLocal) {
+        if constexpr (MODE == kBwdDec) {
+          a.exch[o] = v0;
+          a.exch[L + o] = v;
+        } else {
+          a.exch[o] = v;
+        }
+        continue;
+      }
       // With bf16 copies (the tensor-core kernels take dZ V^T and dQ_dyn V^T
       // from them), the row terms c2 = dZ . Z and c1 = dQ_dyn . Q_dyn use the
       // same rounded values: then each softmax-gradient row still sums to
@@ -343,7 +378,7 @@ __global__ void __launch_bounds__(kBwdThreads) grad_reduce_kernel(const BwdArgs 
       }
     }
   }
-  if constexpr (MODE != kBwdEncSeed) {
+  if constexpr (MODE != kBwdEncSeed && STAGE != kStageLocal) {
     dot = warp_sum(dot);
     if (lane == 0) (MODE == kBwdDec ? a.c2 : a.c1)[static_cast<size_t>(head) * a.M + m] = dot;
   }

@@ -757,12 +757,20 @@ cudaError_t launch_token_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH, 
   return cudaGetLastError();
 }
 
+// phase < 0: the whole backward, each reduction in one kernel.  phase 0..3:
+// one phase of a token-sharded backward; between phases the caller sums
+// a.exch over the ranks (phase 0 leaves dZ and the decode part of dQ_dyn
+// there, phase 1 the routing part of dQ_dyn, phase 2 d_seeds in fp32).  A
+// shard without tokens (a.N == 0) contributes zeros.
 template <int D, typename T>
-cudaError_t launch_backward_d(const BwdArgs& a, const BackwardWs& w, int B, int BH, int dtype, cudaStream_t st) {
+cudaError_t launch_backward_d(const BwdArgs& a, const BackwardWs& w, int B, int BH, int dtype, cudaStream_t st,
+                              int phase = -1) {
   const unsigned tok_tiles = static_cast<unsigned>(ceil_div(static_cast<int64_t>(a.N), kBwdChunk));
   const unsigned lat_chunks = static_cast<unsigned>(ceil_div(a.M, kBwdChunk));
   const dim3 red(static_cast<unsigned>(ceil_div(a.M, 8)), BH);
-  cudaError_t e;
+  const bool all = phase < 0;
+  const bool tokens = a.N > 0;
+  cudaError_t e = cudaSuccess;
   const bool tc = D <= 64 && backward_tc(D, dtype);
   // one latent-side pass: the tensor-core kernel or the CUDA-core one
   auto latent = [&](auto mode) -> cudaError_t {
@@ -773,44 +781,65 @@ cudaError_t launch_backward_d(const BwdArgs& a, const BackwardWs& w, int B, int 
     }
     return launch_dyn(latent_grad_kernel<D, T, kMode>, dim3(a.S, BH, lat_chunks), bwd_smem_latent<D>(), st, a);
   };
-  {
-    ProfScope prof(FLARE_KERNEL_BWD_TOKEN_STATS, st);
-    e = cudaSuccess;
-    if constexpr (D <= 64) {
-      if (tc) e = launch_token_stats_tc<D>(a, w, BH, st);
-    }
-    if (!tc) e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a);
-  }
-  if (e) return e;
-  auto reduce = [&](auto mode, dim3 grid) -> cudaError_t {
+  auto reduce = [&](auto mode, auto stage, dim3 grid) -> cudaError_t {
     ProfScope prof(FLARE_KERNEL_BWD_REDUCE, st);
-    grad_reduce_kernel<D, T, decltype(mode)::value><<<grid, kBwdThreads, 0, st>>>(a, B);
+    grad_reduce_kernel<D, T, decltype(mode)::value, decltype(stage)::value><<<grid, kBwdThreads, 0, st>>>(a, B);
     return cudaGetLastError();
+  };
+  // this rank's sums: the reduction of its partials, or zeros without tokens
+  auto local = [&](auto mode, dim3 grid, size_t floats) -> cudaError_t {
+    if (!tokens) return cudaMemsetAsync(a.exch, 0, floats * sizeof(float), st);
+    return reduce(mode, std::integral_constant<int, kStageLocal>{}, grid);
   };
   using Dec = std::integral_constant<int, kBwdDec>;
   using Rout = std::integral_constant<int, kBwdEncRouting>;
   using Seed = std::integral_constant<int, kBwdEncSeed>;
-  if ((e = latent(Dec{}))) return e;
-  if ((e = reduce(Dec{}, red))) return e;
-  if ((e = latent(Rout{}))) return e;
-  if ((e = reduce(Rout{}, red))) return e;
-  if ((e = latent(Seed{}))) return e;
-  if ((e = reduce(Seed{}, dim3(red.x, a.H)))) return e;
-  ProfScope prof(FLARE_KERNEL_BWD_TOKEN_GRAD, st);
-  if constexpr (D <= 64) {
-    if (tc) return launch_token_grad_tc<D>(a, w, BH, st);
+  using Fused = std::integral_constant<int, kStageFused>;
+  using Finish = std::integral_constant<int, kStageFinish>;
+  const size_t L = static_cast<size_t>(BH) * a.M * D;
+  if (all || phase == 0) {
+    if (tokens) {
+      ProfScope prof(FLARE_KERNEL_BWD_TOKEN_STATS, st);
+      if constexpr (D <= 64) {
+        if (tc) e = launch_token_stats_tc<D>(a, w, BH, st);
+      }
+      if (!tc) e = launch_dyn(token_stats_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_stats<D>(), st, a);
+    }
+    if (e) return e;
+    if (tokens && (e = latent(Dec{}))) return e;
+    if ((e = all ? reduce(Dec{}, Fused{}, red) : local(Dec{}, red, 2 * L))) return e;
   }
-  return launch_dyn(token_grad_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_grad<D>(), st, a);
+  if (all || phase == 1) {
+    if (!all && (e = reduce(Dec{}, Finish{}, red))) return e;
+    if (tokens && (e = latent(Rout{}))) return e;
+    if ((e = all ? reduce(Rout{}, Fused{}, red) : local(Rout{}, red, L))) return e;
+  }
+  if (all || phase == 2) {
+    if (!all && (e = reduce(Rout{}, Finish{}, red))) return e;
+    if (tokens && (e = latent(Seed{}))) return e;
+    const dim3 sred(red.x, a.H);
+    if ((e = all ? reduce(Seed{}, Fused{}, sred) : local(Seed{}, sred, static_cast<size_t>(a.H) * a.M * D))) return e;
+  }
+  if (all || phase == 3) {
+    if (!all && (e = reduce(Seed{}, Finish{}, dim3(red.x, a.H)))) return e;
+    if (!tokens) return cudaSuccess;
+    ProfScope prof(FLARE_KERNEL_BWD_TOKEN_GRAD, st);
+    if constexpr (D <= 64) {
+      if (tc) return launch_token_grad_tc<D>(a, w, BH, st);
+    }
+    return launch_dyn(token_grad_kernel<D, T>, dim3(tok_tiles, BH), bwd_smem_token_grad<D>(), st, a);
+  }
+  return cudaSuccess;
 }
 
 template <typename T>
 cudaError_t launch_backward_t(int D, const BwdArgs& a, const BackwardWs& w, int B, int BH, int dtype,
-                              cudaStream_t st) {
+                              cudaStream_t st, int phase) {
   switch (D) {
-    case 16: return launch_backward_d<16, T>(a, w, B, BH, dtype, st);
-    case 32: return launch_backward_d<32, T>(a, w, B, BH, dtype, st);
-    case 64: return launch_backward_d<64, T>(a, w, B, BH, dtype, st);
-    default: return launch_backward_d<128, T>(a, w, B, BH, dtype, st);
+    case 16: return launch_backward_d<16, T>(a, w, B, BH, dtype, st, phase);
+    case 32: return launch_backward_d<32, T>(a, w, B, BH, dtype, st, phase);
+    case 64: return launch_backward_d<64, T>(a, w, B, BH, dtype, st, phase);
+    default: return launch_backward_d<128, T>(a, w, B, BH, dtype, st, phase);
   }
 }
 
@@ -846,7 +875,7 @@ SavedLayout saved_layout(void* base, int BH, int M, int D, int dtype) {
 
 int run_backward(const void* seeds, const void* K, const void* V, const void* dY, void* d_seeds, void* dK, void* dV,
                  int B, int H, int64_t N, int M, int D, int dtype, char* ws, cudaStream_t st, int* launches,
-                 void* saved = nullptr) {
+                 void* saved = nullptr, int phase = -1, float* exch = nullptr) {
   const int BH = B * H;
   BackwardWs w = backward_ws_layout(ws, BH, N, M, D, dtype);
   if (saved) {
@@ -891,9 +920,10 @@ int run_backward(const void* seeds, const void* K, const void* V, const void* dY
   a.d_seeds = d_seeds;
   a.dK = dK;
   a.dV = dV;
-  const cudaError_t e = dtype == FLARE_BF16 ? launch_backward_t<__nv_bfloat16>(D, a, w, B, BH, dtype, st)
-                                            : launch_backward_t<float>(D, a, w, B, BH, dtype, st);
-  *launches += 8;
+  a.exch = exch;
+  const cudaError_t e = dtype == FLARE_BF16 ? launch_backward_t<__nv_bfloat16>(D, a, w, B, BH, dtype, st, phase)
+                                            : launch_backward_t<float>(D, a, w, B, BH, dtype, st, phase);
+  *launches += phase < 0 ? 8 : 3;
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
 }
 
@@ -1081,6 +1111,39 @@ int flarepp_mix_backward_saved(const void* seeds, const void* K, const void* V, 
     rc = rc2;
     t_last_launches = launches;
   }
+  return rc;
+}
+
+size_t flarepp_backward_shard_exchange_floats(int B, int H, int M, int D) {
+  if (B < 1 || H < 1 || M < 1 || D < 1) return 0;
+  return 2 * static_cast<size_t>(B) * H * M * D;
+}
+
+size_t flarepp_backward_shard_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  if (N < 0 || check_sizes(B, H, N == 0 ? 1 : N, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
+  return backward_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
+}
+
+int flarepp_mix_backward_shard(int phase, const void* seeds, const void* K, const void* V, const void* dY,
+                               const void* saved, float* exchange, void* d_seeds, void* dK, void* dV, int B, int H,
+                               int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes,
+                               void* stream) {
+  if (phase < 0 || phase > 3 || N < 0) return FLARE_ERR_INVALID_ARG;
+  int rc = check_sizes(B, H, N == 0 ? 1 : N, M, D, dtype);
+  if (rc) return rc;
+  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  if (!device_ptr(seeds) || !device_ptr(saved) || !device_ptr(exchange) || !device_ptr(d_seeds))
+    return FLARE_ERR_INVALID_ARG;
+  if (N > 0 && (!device_ptr(K) || !device_ptr(V) || !device_ptr(dY) || !device_ptr(dK) || !device_ptr(dV)))
+    return FLARE_ERR_INVALID_ARG;
+  // the workspace carries the state between the four phases: it is the caller's
+  if (!device_ptr(workspace) ||
+      workspace_bytes < backward_ws_layout(nullptr, B * H, N, M, D, dtype).bytes)
+    return FLARE_ERR_INVALID_ARG;
+  int launches = 0;
+  rc = run_backward(seeds, K, V, dY, d_seeds, dK, dV, B, H, N, M, D, dtype, static_cast<char*>(workspace),
+                    static_cast<cudaStream_t>(stream), &launches, const_cast<void*>(saved), phase, exchange);
+  if (!rc) t_last_launches = launches;
   return rc;
 }
 

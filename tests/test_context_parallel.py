@@ -21,7 +21,7 @@ import pytest
 
 import oracle
 import rank_latent_attention_b200 as flare
-from gpu_common import assert_bf16_storage, assert_stated, require_cuda, to_dev, to_host
+from gpu_common import assert_backward_bar, assert_bf16_storage, assert_stated, require_cuda, to_dev, to_host
 from rank_latent_attention_b200 import context_parallel as cp
 from rank_latent_attention_b200 import inputs
 
@@ -197,3 +197,137 @@ def test_invalid_arguments():
                               vp(L.data_ptr()), 1, 1, -1, 16, 16, 0, None, 0, None)
     assert rc == 1
     torch.cuda.synchronize()
+
+
+# ---------------------------------------------------------------- sharded backward
+def _emulate_save(s_d, K_d, V_d, R):
+    """The sharded forward with save=True, R ranks emulated in turn: Q_dyn, Z
+    and their log-sum-exps combined from all shards into one saved state."""
+    import torch
+
+    B, H, N, D = K_d.shape
+    M = s_d.shape[-2]
+    ops = cp.LibraryOps()
+    saved = torch.empty(ops.saved_bytes(B, H, M, D, K_d.dtype), dtype=torch.uint8, device="cuda")
+    Qv, Zv, L1, L2 = cp.saved_views(saved, B, H, M, D, K_d.dtype)
+    recv = torch.empty((R, cp.exchange_floats(B, H, M, D)), dtype=torch.float32, device="cuda")
+    shards = [(cp.shard_tokens(K_d, R, r), cp.shard_tokens(V_d, R, r)) for r in range(R)]
+    for Q, out, lse in ((s_d, Qv, L1), (Qv, Zv, L2)):
+        for r, (Kr, Vr) in enumerate(shards):
+            ops.encode_lse(Q, Kr, Vr, recv[r])
+        ops.combine(recv, B, H, M, D, K_d.dtype, out, lse)
+    return saved, shards
+
+
+def _emulate_backward(s_d, shards, dYs, saved, R):
+    """The four phases on every emulated rank, with the sum over ranks of the
+    exchange buffers (what the all-reduce returns) between phases."""
+    import torch
+
+    ops = cp.LibraryOps()
+    B, H, _, D = shards[0][0].shape
+    M = s_d.shape[-2]
+    lat = B * H * M * D
+    states = [ops.backward_state(s_d, Kr, M) for Kr, _ in shards]
+    grads = [(torch.empty_like(s_d), torch.empty_like(Kr), torch.empty_like(Vr)) for Kr, Vr in shards]
+    for phase, n in ((0, 2 * lat), (1, lat), (2, H * M * D), (3, 0)):
+        for r in range(R):
+            ops.backward_phase(phase, s_d, shards[r][0], shards[r][1], dYs[r], saved, states[r][0], states[r][1],
+                               grads[r])
+        if n:
+            total = torch.stack([st[0][:n] for st in states]).sum(0)
+            for st in states:
+                st[0][:n].copy_(total)
+    return grads
+
+
+def test_sharded_backward_one_rank_matches_saved():
+    """One rank, no exchange: the four phases give flarepp_mix_backward_saved's bits."""
+    import torch
+
+    require_cuda()
+    w = inputs.custom(1, 2, 700, 256, 64, dtype="bf16", seed_index=90)
+    seeds, K, V = inputs.make_inputs(w)
+    dY = inputs.make_upstream(w)
+    dev = [to_dev(x, "bf16") for x in (seeds, K, V, dY)]
+    _, saved = flare.flarepp_mix_save(*dev[:3])
+    want = flare.flarepp_mix_backward_saved(*dev, saved)
+    got = _emulate_backward(dev[0], [(dev[1], dev[2])], [dev[3]], saved, 1)[0]
+    for a, b in zip(got, want):
+        assert torch.equal(a, b)
+    assert flare.flare_check_status() == (0, 0)
+
+
+@pytest.mark.parametrize("name,R", [("cloud", 3), ("long", 2), ("tiny_f32", 2)])
+def test_sharded_backward_emulated_ranks(name, R):
+    """R ranks: dK and dV of each rank's tokens and the common d_seeds, against
+    the oracle's backward of the stored chain (the sharded forward's Q_dyn, Z)."""
+    import torch
+
+    require_cuda()
+    w = inputs.WORKLOADS[name]
+    seeds, K, V = inputs.make_inputs(w)
+    dY = inputs.make_upstream(w)
+    s_d, K_d, V_d, dY_d = (to_dev(x, w.dtype) for x in (seeds, K, V, dY))
+    saved, shards = _emulate_save(s_d, K_d, V_d, R)
+    dYs = [cp.shard_tokens(dY_d, R, r) for r in range(R)]
+    grads = _emulate_backward(s_d, shards, dYs, saved, R)
+    assert flare.flare_check_status() == (0, 0)
+    for g in grads[1:]:
+        assert torch.equal(g[0], grads[0][0])  # the same summed d_seeds on every rank
+    got = [to_host(grads[0][0]), to_host(torch.cat([g[1] for g in grads], dim=2)),
+           to_host(torch.cat([g[2] for g in grads], dim=2))]
+    Qv, Zv, _, _ = cp.saved_views(saved, w.B, w.H, w.M, w.D, K_d.dtype)
+    want = oracle.flarepp_backward(*(x.astype(np.float64) for x in (seeds, K, V, dY)), Q_dyn=to_host(Qv),
+                                   Z=to_host(Zv))
+    tensor_cores = w.dtype == "bf16" and w.D <= 64
+    for label, g, r in zip(("d_seeds", "dK", "dV"), got, want):
+        assert_backward_bar(f"{name}.cp{R}.{label}", g, r, w.dtype, tensor_cores)
+
+
+def test_sharded_backward_with_an_empty_rank():
+    """3 tokens over 5 ranks: the two ranks without tokens contribute zeros."""
+    import torch
+
+    require_cuda()
+    w = inputs.custom(2, 2, 3, 16, 16, dtype="f32", seed_index=91)
+    seeds, K, V = inputs.make_inputs(w)
+    dY = inputs.make_upstream(w)
+    s_d, K_d, V_d, dY_d = (to_dev(x, "f32") for x in (seeds, K, V, dY))
+    saved, shards = _emulate_save(s_d, K_d, V_d, 5)
+    grads = _emulate_backward(s_d, shards, [cp.shard_tokens(dY_d, 5, r) for r in range(5)], saved, 5)
+    assert flare.flare_check_status() == (0, 0)
+    want = oracle.flarepp_backward(*(x.astype(np.float64) for x in (seeds, K, V, dY)))
+    got = [to_host(grads[0][0]), to_host(torch.cat([g[1] for g in grads], dim=2)),
+           to_host(torch.cat([g[2] for g in grads], dim=2))]
+    for g, r in zip(got, want):
+        assert np.max(np.abs(g - r)) <= 1e-4
+
+
+def test_nccl_world_of_one_training_step():
+    """flarepp_mix_cp(save=True) and flarepp_mix_backward_cp over a real NCCL
+    group of one rank: the same Y as flarepp_mix; gradients within the
+    backward's bars of the single-GPU saved-state backward."""
+    import torch
+    import torch.distributed as dist
+
+    require_cuda()
+    w = inputs.custom(1, 2, 3000, 64, 32, dtype="bf16", seed_index=92)
+    seeds, K, V = inputs.make_inputs(w)
+    dY = inputs.make_upstream(w)
+    s_d, K_d, V_d, dY_d = (to_dev(x, "bf16") for x in (seeds, K, V, dY))
+    dist.init_process_group("nccl", store=dist.HashStore(), rank=0, world_size=1,
+                            timeout=datetime.timedelta(seconds=60), device_id=torch.device("cuda", 0))
+    try:
+        Y, saved = cp.flarepp_mix_cp(s_d, K_d, V_d, save=True)
+        grads = cp.flarepp_mix_backward_cp(s_d, K_d, V_d, dY_d, saved)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert flare.flare_check_status() == (0, 0)
+    assert torch.equal(Y, flare.flarepp_mix(s_d, K_d, V_d))
+    Qv, Zv, _, _ = cp.saved_views(saved, 1, 2, 64, 32, torch.bfloat16)
+    want = oracle.flarepp_backward(*(x.astype(np.float64) for x in (seeds, K, V, dY)), Q_dyn=to_host(Qv),
+                                   Z=to_host(Zv))
+    for label, g, r in zip(("d_seeds", "dK", "dV"), grads, want):
+        assert_backward_bar(f"nccl1.{label}", to_host(g), r, "bf16", True)
