@@ -52,13 +52,16 @@ def exchange_floats(B: int, H: int, M: int, D: int) -> int:
     return B * H * M * (D + 1)
 
 
-def saved_views(saved, B: int, H: int, M: int, D: int, dtype):
+def saved_views(saved, B: int, H: int, M: int, D: int, dtype, lse_dtype=None):
     """Views (Q_dyn, Z, lse1, lse2) into a saved-state byte buffer laid out as
     flarepp_mix_save writes it: Q_dyn and Z [B,H,M,D] in dtype, then lse1 and
-    lse2 [B,H,M] fp32, each region starting on a 256-byte boundary."""
+    lse2 [B,H,M] (fp32 unless lse_dtype says otherwise), each region starting
+    on a 256-byte boundary."""
     import torch
 
+    lse_dtype = lse_dtype or torch.float32
     esz = torch.empty((), dtype=dtype).element_size()
+    lsz = torch.empty((), dtype=lse_dtype).element_size()
     lat = B * H * M
 
     def region(off, n, dt, shape):
@@ -67,9 +70,9 @@ def saved_views(saved, B: int, H: int, M: int, D: int, dtype):
     r = lambda x: (x + 255) // 256 * 256  # noqa: E731
     o1 = r(lat * D * esz)
     o2 = o1 + r(lat * D * esz)
-    o3 = o2 + r(lat * 4)
+    o3 = o2 + r(lat * lsz)
     return (region(0, lat * D, dtype, (B, H, M, D)), region(o1, lat * D, dtype, (B, H, M, D)),
-            region(o2, lat, torch.float32, (B, H, M)), region(o3, lat, torch.float32, (B, H, M)))
+            region(o2, lat, lse_dtype, (B, H, M)), region(o3, lat, lse_dtype, (B, H, M)))
 
 
 def all_reduce_sum(t, group=None):
@@ -180,7 +183,7 @@ def flarepp_mix_cp(seeds, K, V, *, group=None, ops=None, return_intermediates=Fa
     saved = views = None
     if save:
         saved = torch.empty(ops.saved_bytes(B, H, M, D, K.dtype), dtype=torch.uint8, device=K.device)
-        views = saved_views(saved, B, H, M, D, K.dtype)
+        views = saved_views(saved, B, H, M, D, K.dtype, getattr(ops, "lse_dtype", None))
 
     ops.encode_lse(seeds, K, V, send)
     Q_dyn = ops.combine(ops.all_gather(send), B, H, M, D, K.dtype,
