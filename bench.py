@@ -391,7 +391,30 @@ def run_native(args):
     if st != (0, 0):
         raise RuntimeError(f"device status after the context-parallel steps: {st}")
     cp_exchange = 2 * cp.exchange_floats(1, w.H, w.M, w.D) * 4
-    del K_r, V_r, ws_cp
+
+    # ---- a token-sharded training step: forward with saved state, then the
+    # four-phase backward with an all-reduce of its token sums between phases
+    gdy = torch.Generator(device=dev).manual_seed(6)
+    dY_r = torch.randn(K_r.shape, device=dev, generator=gdy).to(torch.bfloat16)
+
+    def cp_train_step():
+        Yt, saved_t = cp.flarepp_mix_cp(s_d, K_r, V_r, ops=cp_ops, save=True)
+        return cp.flarepp_mix_backward_cp(s_d, K_r, V_r, dY_r, saved_t, ops=cp_ops)
+
+    nct = max(1, min(args.steps, 10))
+    for _ in range(2):
+        cp_train_step()
+    barrier()
+    ev0.record(stream)
+    for _ in range(nct):
+        cp_train_step()
+    ev1.record(stream)
+    barrier()
+    cp_train_ms = max_over_ranks(ev0.elapsed_time(ev1)) / nct
+    st = flare.flare_check_status()
+    if st != (0, 0):
+        raise RuntimeError(f"device status after the context-parallel training steps: {st}")
+    del K_r, V_r, ws_cp, dY_r
 
     # ---- backward: gradients of sum(dY * Y) for the seeds, K and V
     gdy = torch.Generator(device=dev).manual_seed(5)
@@ -542,7 +565,9 @@ def run_native(args):
         "context_parallel": {"ms_per_step": cp_ms, "tokens_per_s": w.N / (cp_ms * 1e-3), "ranks": world,
                              "scaling": "strong", "tokens": w.N, "steps": ncp,
                              "exchange_bytes_per_rank_per_step": cp_exchange,
-                             "collective": "all_gather_into_tensor (NCCL), 2 per step" if world > 1 else "none (1 rank)"},
+                             "collective": "all_gather_into_tensor (NCCL), 2 per step" if world > 1 else "none (1 rank)",
+                             "training_step_ms": cp_train_ms,
+                             "training_collectives": "2 all-gathers + 3 all-reduces per step" if world > 1 else "none (1 rank)"},
         "backward": {"ms_per_step": bwd_ms, "tokens_per_s": ranks.job_tokens_per_s(w.N, env, bwd_ms), "steps": nb,
                      "launches": bwd_launches, "kernel_ms": bwd_split,
                      "executed_gemm_tflops": 25 * 2.0 * w.N * w.M * w.D * w.H / (bwd_ms * 1e-3) / 1e12,
