@@ -99,3 +99,29 @@ def test_option_hooks_round_trip(L):
     assert L.flare_set_split_override(old) == 5
     old = L.flare_set_wait_limit_ms(123)
     assert L.flare_set_wait_limit_ms(old) == 123
+
+
+def test_header_is_plain_c_and_links(tmp_path):
+    """include/flarepp.h compiles as pedantic C99; a C program links against
+    libflarepp.so and calls a host-side query (no GPU needed)."""
+    import os
+    import shutil
+
+    gcc = shutil.which("gcc")
+    if gcc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "use_abi.c"
+    src.write_text(
+        '#include <stdio.h>\n#include "flarepp.h"\n'
+        "int main(void) {\n"
+        "  size_t a = flarepp_saved_bytes(1, 16, 256, 64, FLARE_BF16);\n"
+        "  size_t b = flarepp_saved_bytes(1, 1, 17, 64, FLARE_BF16);\n"
+        '  printf("%zu %zu\\n", a, b);\n'
+        "  return 0;\n}\n")
+    lib_dir = os.path.dirname(flare.LIB_PATH)
+    exe = tmp_path / "use_abi"
+    subprocess.run([gcc, "-std=c99", "-Wall", "-Wextra", "-pedantic", "-Werror", "-I",
+                    os.path.dirname(flare.HEADER_PATH), str(src), "-L", lib_dir, "-lflarepp",
+                    f"-Wl,-rpath,{lib_dir}", "-o", str(exe)], check=True, capture_output=True)
+    out = subprocess.run([str(exe)], check=True, capture_output=True, text=True).stdout.split()
+    assert out == [str(flare.flarepp_saved_bytes(1, 16, 256, 64, 1)), "0"]
