@@ -274,10 +274,22 @@ int flarepp_mix_host(const void* seeds, const void* K, const void* V, void* Y, i
  * Synchronises `stream`, then reads and clears the current device's status
  * word.  Returns FLARE_OK or the first error a kernel recorded since the last
  * check (FLARE_ERR_TIMEOUT); *site (if not NULL) receives the kernel role
- * that recorded it (1-3 encode producer/MMA/softmax, 4-6 decode).  Returns
+ * that recorded it (1-3 encode producer/MMA/softmax, 4-6 decode producer/
+ * MMA/softmax, 7-12 the backward's tensor-core kernels, 13 the wait
+ * self-test).  Returns
  * FLARE_ERR_CUDA if the synchronisation itself fails.
  */
 int flare_check_status(void* stream, int* site);
+
+/*
+ * Self-test of the kernels' bounded waits: one warp waits on an mbarrier
+ * that nothing arrives at.  The wait gives up after limit_ms (1..1000) of
+ * %globaltimer, the kernel records FLARE_ERR_TIMEOUT with site 13 in the
+ * status word (as any kernel that gives up waiting does) and returns; the
+ * context stays usable.  flare_check_status then returns FLARE_ERR_TIMEOUT.
+ * The probe holds no TMA copy, MMA or tensor memory.
+ */
+int flare_selftest_wait_timeout(int limit_ms, void* stream);
 
 /* Static, human-readable name of a status code. */
 const char* flare_status_string(int status);

@@ -87,6 +87,7 @@ _SIGNATURES = {
     "flare_communication_workspace_size": (_c_size, _SIZES),
     "flare_communication_matrix": (_c_int, [_vp, _c_int, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_set_split_override": (_c_int, [_c_int]),
+    "flare_selftest_wait_timeout": (_c_int, [_c_int, _vp]),
     "flare_set_wait_limit_ms": (_c_int, [_c_int]),
     "flare_profile_begin": (_c_int, [_c_int]),
     "flare_profile_end": (_c_int, [ctypes.POINTER(ctypes.c_float), ctypes.POINTER(_c_int), _c_int]),

@@ -927,6 +927,26 @@ int run_backward(const void* seeds, const void* K, const void* V, const void* dY
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
 }
 
+// Self-test of the bounded wait every kernel uses: one warp waits on an
+// mbarrier that nothing arrives at.  ptx::mbar_wait gives up after limit_ns
+// (%globaltimer), and the kernel records FLARE_ERR_TIMEOUT with its site in
+// the device status word and returns, as the real kernels do on a timeout.
+// No TMA copy, MMA or TMEM is involved, so nothing else has to drain.
+constexpr int kSiteWaitProbe = 13;
+
+__global__ void __launch_bounds__(32) wait_probe_kernel(int* status, unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    ptx::mbar_init(&bar, 1);
+    abort_flag = 0;
+    ptx::fence_mbar_init();
+  }
+  __syncwarp();
+  const bool ok = ptx::mbar_wait(&bar, 0, &abort_flag, limit_ns);  // phase 0 never completes
+  if (!ok && threadIdx.x == 0) record_error(status, kErrTimeout, kSiteWaitProbe);
+}
+
 // fp32 tensor in device memory with 4-byte alignment (the per-latent
 // statistics of a slice of a gathered [R][B][H][M] array need no more).
 bool device_ptr_f32(const void* p) {
@@ -1268,6 +1288,17 @@ int flarepp_mix_host(const void* seeds, const void* K, const void* V, void* Y, i
     t_last_launches = launches;
   }
   return rc;
+}
+
+int flare_selftest_wait_timeout(int limit_ms, void* stream) {
+  if (limit_ms < 1 || limit_ms > 1000) return FLARE_ERR_INVALID_ARG;
+  int* status = status_ptr();
+  if (!status) return FLARE_ERR_CUDA;
+  wait_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      status, static_cast<unsigned long long>(limit_ms) * 1000000ull);
+  if (cudaGetLastError() != cudaSuccess) return FLARE_ERR_CUDA;
+  t_last_launches = 1;
+  return FLARE_OK;
 }
 
 int flare_check_status(void* stream, int* site) {
