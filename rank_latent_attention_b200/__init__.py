@@ -434,15 +434,16 @@ def flarepp_mix(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, stream=N
     return Y
 
 
-def flarepp_mix_debug(seeds, K, V, *, out_dtype=None, workspace=None, stream=None):
-    """As flarepp_mix, also returning the intermediates: (Y, Q_dyn, Z)."""
+def flarepp_mix_debug(seeds, K, V, *, Y=None, Q_dyn=None, Z=None, out_dtype=None, workspace=None, stream=None):
+    """As flarepp_mix, also returning the intermediates: (Y, Q_dyn, Z)
+    (allocated unless given)."""
     torch = _torch()
     B, H, N, D = K.shape
     M = seeds.shape[1]
     code, odt = _mix_mode(K, out_dtype)
-    Y = torch.empty(K.shape, dtype=odt, device=K.device)
-    Qd = torch.empty((B, H, M, D), dtype=odt, device=K.device)
-    Z = torch.empty_like(Qd)
+    Y = torch.empty(K.shape, dtype=odt, device=K.device) if Y is None else Y
+    Qd = torch.empty((B, H, M, D), dtype=odt, device=K.device) if Q_dyn is None else Q_dyn
+    Z = torch.empty_like(Qd) if Z is None else Z
     ws, wsb = _ws(workspace)
     _check(lib().flarepp_mix_debug(_ptr(seeds, "seeds", K.dtype), _ptr(K, "K", K.dtype), _ptr(V, "V", K.dtype),
                                    _ptr(Y, "Y", odt), _ptr(Qd, "Q_dyn", odt), _ptr(Z, "Z", odt),
