@@ -46,11 +46,18 @@
 // (D = 128); Q after the accumulators as bf16 pairs when it fits (Q.K^T then
 // reads it as the TMEM A operand), else in shared memory.
 //
-// Online softmax with a lazy reference: a row's reference max only moves when
-// a tile's max exceeds it by more than 2^8, so the O rescale in tensor memory
-// is rare.  Any reference gives the same normalised result because P and l
-// use the same one.  Of every 16 column pairs, those in kEncPolyPairs take
-// their exponentials from exp2_poly3 (FMA pipe) instead of MUFU.
+// Online softmax with a lazy reference.  Any reference gives the same
+// normalised result because P and l use the same one, so a row's reference
+// only has to keep 2^(x log2e - reference) inside the fp32 range:
+//   - past the first tile (split accumulators), a group takes the exponentials
+//     of a full tile against the reference it has, without the half-row max,
+//     and keeps them if every row's sum stays within 2^32;
+//   - otherwise (first tile, ragged tile, a sum above 2^32 or inf, or a shared
+//     O) it takes the half-row max, and the reference moves to it when the max
+//     exceeds the reference by more than 2^8; the O rescale in tensor memory
+//     is rare.
+// Of every 16 column pairs, those in kEncPolyPairs take their exponentials
+// from exp2_poly3 (FMA pipe) instead of MUFU.
 //
 // Epilogue: each CTA writes one partial per head (O_part[split] etc.), the
 // accumulators that cover the same latent rows folded with their weights
@@ -171,6 +178,39 @@ __device__ __forceinline__ float encode_exp_store(const float* x, float nref, ui
       p[u] = ptx::pack_bf16(e0, e1);
     }
     ptx::tmem_st8(tP + c0 / 2, p);
+  }
+  float s0, s1, s2, s3;
+  ptx::f2_split(ps[0], s0, s1);
+  ptx::f2_split(ps[1], s2, s3);
+  return (s0 + s1) + (s2 + s3);
+}
+
+// P = 2^(x log2e - nref) for the 32 scores of one full half-row, packed to
+// bf16 pairs in p[16]; returns the fp32 sum.  Used against a reference that
+// may sit below the half-row's max: the polynomial's input is clamped at 64
+// (a result of at most 2^64), so that a score far above the reference shows
+// up in the sum (MUFU gives +inf there) instead of wrapping the exponent
+// field.
+__device__ __forceinline__ float encode_exp_pack(const float* x, float nref, uint32_t* p) {
+  const uint64_t kL2 = ptx::f2(kLog2e, kLog2e);
+  const uint64_t nn = ptx::f2(-nref, -nref);
+  uint64_t ps[2] = {0ull, 0ull};
+#pragma unroll
+  for (int u = 0; u < 16; ++u) {
+    const int c = 2 * u;
+    const uint64_t a = ptx::fma2(ptx::f2(x[c], x[c + 1]), kL2, nn);
+    uint64_t e;
+    float a0, a1;
+    ptx::f2_split(a, a0, a1);
+    if ((kEncPolyPairs >> (u & 15)) & 1u) {
+      e = exp2_poly3_x2(ptx::f2(fminf(a0, 64.f), fminf(a1, 64.f)));
+    } else {
+      e = ptx::f2(ptx::ex2(a0), ptx::ex2(a1));
+    }
+    ps[u & 1] = ptx::add2(ps[u & 1], e);
+    float e0, e1;
+    ptx::f2_split(e, e0, e1);
+    p[u] = ptx::pack_bf16(e0, e1);
   }
   float s0, s1, s2, s3;
   ptx::f2_split(ps[0], s0, s1);
@@ -416,53 +456,70 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
         for (int z = 0; z < 32; ++z)
           if (z >= valid) x[z] = -INFINITY;
       }
-      // half-row max as 8 independent 3-input chains
-      float pm[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) pm[u] = fmaxf(x[2 * u], x[2 * u + 1]);
-#pragma unroll
-      for (int u = 0; u < 8; ++u) pm[u] = ptx::max3(pm[u], x[16 + 2 * u], x[17 + 2 * u]);
-      float mx = ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
-      if constexpr (!C::kSplitO) {
-        // shared O: agree on the row max with the other group of the slot
-        // (buffers alternate by tile parity, so a fast group cannot overwrite
-        // a value not yet read); after the barrier both groups have read
-        // their scores and P may overwrite S
-        float* xm = s_xm + ((j * 2 + s) * 2) * kLatRows;
-        xm[c * kLatRows + r] = mx;
-        asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");
-        mx = fmaxf(mx, xm[(c ^ 1) * kLatRows + r]);
-      }
-      mx *= kLog2e;
-      const bool need = mx > mref + 8.f;
-      const float nref = need ? mx : mref;
-      // 0 on the first tile; 1 while a fully masked half-row has no reference
-      const float alpha = nref == mref ? 1.f : ptx::ex2(mref - nref);
-      mref = nref;
-      // P overwrites the first 16 of this group's own 32 score columns
-      const float lt = valid < 32 ? encode_exp_store<true>(x, nref, tS + 32 * c)
-                                  : encode_exp_store<false>(x, nref, tS + 32 * c);
-      l = fmaf(l, alpha, lt);
-      // Rare: the reference moved, so rescale this group's part of O, once the
-      // previous P.V (issued after P(i - 1)) has completed; the next one waits
-      // for P_full.
-      if (i > 0 && __any_sync(0xffffffffu, need)) {
-        if (!__all_sync(0xffffffffu, ptx::mbar_wait(&pv_done[s], (i - 1) & 1, s_abort, args.wait_ns))) {
-          ok = false;
-          break;
+      // Past the first tile the reference is usually high enough: take the
+      // exponentials against it without the half-row max, and fall back to the
+      // max below only if some score of the tile sits far above it (a sum
+      // above 2^32, or inf).  Split accumulators only: with a shared O the two
+      // groups must take the same path.
+      bool done = false;
+      if (C::kSplitO && i > 0 && valid >= 32) {
+        uint32_t p[16];
+        const float lt = encode_exp_pack(x, mref, p);
+        if (__all_sync(0xffffffffu, lt <= 4294967296.f)) {
+          ptx::tmem_st16(tS + 32 * c, p);
+          l += lt;
+          done = true;
         }
-        ptx::tc_fence_after();
-        constexpr int kChunk = kOCols < 32 ? kOCols : 32;
+      }
+      if (!done) {
+        // half-row max as 8 independent 3-input chains
+        float pm[8];
 #pragma unroll
-        for (int z0 = 0; z0 < kOCols; z0 += kChunk) {
-          float o[kChunk];
-          const uint32_t ta = tOwn + z0;
-          if constexpr (kChunk == 32) ptx::tmem_ld32(ta, o); else if constexpr (kChunk == 16) ptx::tmem_ld16(ta, o); else ptx::tmem_ld8(ta, o);
-          ptx::tmem_wait_ld();
-          uint32_t u[kChunk];
+        for (int u = 0; u < 8; ++u) pm[u] = fmaxf(x[2 * u], x[2 * u + 1]);
 #pragma unroll
-          for (int z = 0; z < kChunk; ++z) u[z] = __float_as_uint(o[z] * alpha);
-          if constexpr (kChunk == 32) ptx::tmem_st32(ta, u); else if constexpr (kChunk == 16) ptx::tmem_st16(ta, u); else ptx::tmem_st8(ta, u);
+        for (int u = 0; u < 8; ++u) pm[u] = ptx::max3(pm[u], x[16 + 2 * u], x[17 + 2 * u]);
+        float mx = ptx::max3(ptx::max3(pm[0], pm[1], pm[2]), ptx::max3(pm[3], pm[4], pm[5]), fmaxf(pm[6], pm[7]));
+        if constexpr (!C::kSplitO) {
+          // shared O: agree on the row max with the other group of the slot
+          // (buffers alternate by tile parity, so a fast group cannot overwrite
+          // a value not yet read); after the barrier both groups have read
+          // their scores and P may overwrite S
+          float* xm = s_xm + ((j * 2 + s) * 2) * kLatRows;
+          xm[c * kLatRows + r] = mx;
+          asm volatile("bar.sync %0, 256;" ::"r"(bar_id) : "memory");
+          mx = fmaxf(mx, xm[(c ^ 1) * kLatRows + r]);
+        }
+        mx *= kLog2e;
+        const bool need = mx > mref + 8.f;
+        const float nref = need ? mx : mref;
+        // 0 on the first tile; 1 while a fully masked half-row has no reference
+        const float alpha = nref == mref ? 1.f : ptx::ex2(mref - nref);
+        mref = nref;
+        // P overwrites the first 16 of this group's own 32 score columns
+        const float lt = valid < 32 ? encode_exp_store<true>(x, nref, tS + 32 * c)
+                                    : encode_exp_store<false>(x, nref, tS + 32 * c);
+        l = fmaf(l, alpha, lt);
+        // Rare: the reference moved, so rescale this group's part of O, once the
+        // previous P.V (issued after P(i - 1)) has completed; the next one waits
+        // for P_full.
+        if (i > 0 && __any_sync(0xffffffffu, need)) {
+          if (!__all_sync(0xffffffffu, ptx::mbar_wait(&pv_done[s], (i - 1) & 1, s_abort, args.wait_ns))) {
+            ok = false;
+            break;
+          }
+          ptx::tc_fence_after();
+          constexpr int kChunk = kOCols < 32 ? kOCols : 32;
+#pragma unroll
+          for (int z0 = 0; z0 < kOCols; z0 += kChunk) {
+            float o[kChunk];
+            const uint32_t ta = tOwn + z0;
+            if constexpr (kChunk == 32) ptx::tmem_ld32(ta, o); else if constexpr (kChunk == 16) ptx::tmem_ld16(ta, o); else ptx::tmem_ld8(ta, o);
+            ptx::tmem_wait_ld();
+            uint32_t u[kChunk];
+#pragma unroll
+            for (int z = 0; z < kChunk; ++z) u[z] = __float_as_uint(o[z] * alpha);
+            if constexpr (kChunk == 32) ptx::tmem_st32(ta, u); else if constexpr (kChunk == 16) ptx::tmem_st16(ta, u); else ptx::tmem_st8(ta, u);
+          }
         }
       }
       ptx::tmem_wait_st();
