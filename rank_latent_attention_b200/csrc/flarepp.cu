@@ -105,15 +105,15 @@ bool device_ptr(const void* p) {
 }
 
 // CTAs per head along the token axis: enough CTAs to fill whole waves of the
-// SMs (one CTA per SM), at most ~32768 tokens per CTA; `tile` is the kernel's
-// token tile (64 for the encode, 128 for the decode).
-int choose_splits(int BH, int64_t N, int tile) {
+// SMs' CTA slots (per_sm resident CTAs per SM), at most ~32768 tokens per CTA;
+// `tile` is the kernel's token tile (64 for the encode, 128 for the decode).
+int choose_splits(int BH, int64_t N, int tile, int per_sm = 1) {
   const int64_t tiles = ceil_div(N, tile);
   int64_t s = g_split_override.load();
   if (s <= 0) {
-    const int sms = sm_count();
-    const int64_t waves = std::max<int64_t>(1, ceil_div(BH * tiles, int64_t(sms) * (32768 / tile)));
-    s = ceil_div(waves * sms, BH);
+    const int64_t slots = int64_t(sm_count()) * per_sm;
+    const int64_t waves = std::max<int64_t>(1, ceil_div(BH * tiles, slots * (32768 / tile)));
+    s = ceil_div(waves * slots, BH);
   }
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(s, tiles)));
 }
@@ -618,7 +618,8 @@ bool backward_tc(int D, int dtype) { return dtype == FLARE_BF16 && D <= 64; }
 
 // Token splits of the latent-side kernels (the partial blocks' S).
 int backward_latent_splits(int BH, int64_t N, int M, int D, int dtype) {
-  if (backward_tc(D, dtype)) return choose_splits(BH * static_cast<int>(ceil_div(M, 128)), N, kBltcTok);
+  // two CTAs per SM (256 TMEM columns each)
+  if (backward_tc(D, dtype)) return choose_splits(BH * static_cast<int>(ceil_div(M, 128)), N, kBltcTok, 2);
   return backward_splits(BH, N, M);
 }
 
@@ -707,7 +708,7 @@ cudaError_t launch_token_stats_tc(const BwdArgs& a, const BackwardWs& w, int BH,
   t.N = a.N;
   t.M = a.M;
   t.tiles = static_cast<int>(ceil_div(N, 128));
-  t.splits = choose_splits(BH, N, 128);
+  t.splits = choose_splits(BH, N, 128, 2);  // two CTAs per SM
   t.lse3 = a.lse3;
   t.delta = a.delta;
   t.status = status_ptr();
