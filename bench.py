@@ -431,10 +431,13 @@ def run_native(args):
     bwd_launches = flare.flare_last_launch_count()
     nb = max(1, min(args.steps, 20))
     barrier()
+    # NVTX range "backward": lets a profiler select these launches alone
+    torch.cuda.nvtx.range_push("backward")
     ev0.record(stream)
     for _ in range(nb):
         bwd_step()
     ev1.record(stream)
+    torch.cuda.nvtx.range_pop()
     barrier()
     bwd_ms = max_over_ranks(ev0.elapsed_time(ev1)) / nb
     flare.flare_profile_begin(64)
