@@ -34,6 +34,12 @@ the data path.  Rank 0 prints one JSON line:
   seeded N(0,1) dY) on the same inputs, with its per-kernel split, and
   the same backward reading the state flarepp_mix_save kept
   (saved_state_ms_per_step).
+* small_configs: the four smaller seeded workloads (the parity cases c1-c4),
+  one flarepp_mix call each, median of 20 CUDA-event-timed calls after 3
+  warm-ups, L2-warm and L2-cold (a 256 MB scrub write before each call,
+  outside the timed events), each call queued behind a short device-side
+  spin so the events time the device's work; with tokens/s, TFLOP/s and the
+  fraction of their single-pass HBM / tensor roofline.
 
 --impl reference times the oracle (the reference arm of this comparison) on
 the host cores, rank 0 only, and prints the same line with "impl": "reference".
@@ -581,9 +587,72 @@ def run_native(args):
         "e2e": {"value": ranks.job_tokens_per_s(w.N, env, e2e_ms), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms, "steps": ne},
     }
+    line["small_configs"] = small_configs(torch, flare, inputs, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
     print(json.dumps(line), flush=True)
+
+
+# the four smaller seeded workloads, by the configuration tag they carry
+SMALL_CONFIGS = (("c1", "tiny_f32"), ("c2", "cloud"), ("c3", "mesh2d"), ("c4", "long"))
+L2_SCRUB_BYTES = 256 << 20  # written before each L2-cold call: twice the 126 MB L2
+
+
+def small_configs(torch, flare, inputs, dev, peaks):
+    """One flarepp_mix call per small workload: median of 20 event-timed calls
+    after 3 warm-ups, L2-warm and L2-cold.  Roofline per call: the larger of
+    12 N M D B H FLOP at the sustained bf16 GEMM peak (bf16 workloads) and
+    the single-pass bytes (K and V read once, Y written once) at the measured
+    copy bandwidth; these heads fit in L2, so one pass is the minimum."""
+    scrub = torch.empty(L2_SCRUB_BYTES, dtype=torch.uint8, device=dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    out = {}
+    for tag, name in SMALL_CONFIGS:
+        w = inputs.WORKLOADS[name]
+        tdt = torch.float32 if w.dtype == "f32" else torch.bfloat16
+        s_d, K_d, V_d = (torch.from_numpy(x).to(dev).to(tdt) for x in inputs.make_inputs(w))
+        Y_d = torch.empty_like(K_d)
+        ws = torch.empty(flare.flarepp_workspace_size(w.B, w.H, w.N, w.M, w.D, 0 if w.dtype == "f32" else 1),
+                         dtype=torch.uint8, device=dev)
+
+        def call():
+            flare.flarepp_mix(s_d, K_d, V_d, Y_d, workspace=ws)
+
+        for _ in range(3):
+            call()
+        times = {"warm": [], "cold": []}
+        for mode in ("warm", "cold"):
+            for _ in range(20):
+                if mode == "cold":
+                    scrub.fill_(1)
+                # a short device-side spin ahead of the call, so that its
+                # launches are queued before the start event: the events then
+                # time the device's work, not the host's launch overhead
+                torch.cuda._sleep(200_000)
+                e0.record()
+                call()
+                e1.record()
+                e1.synchronize()
+                times[mode].append(e0.elapsed_time(e1))
+        st = flare.flare_check_status()
+        if st != (0, 0):
+            raise RuntimeError(f"device status after the {name} calls: {st}")
+        ms_w, ms_c = statistics.median(times["warm"]), statistics.median(times["cold"])
+        esz = 4 if w.dtype == "f32" else 2
+        flops = 12.0 * w.N * w.M * w.D * w.B * w.H
+        nbytes = 3.0 * w.N * w.D * w.B * w.H * esz
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+        t_tensor = flops / (tensor_peak * 1e12) * 1e3 if w.dtype != "f32" else 0.0
+        t_roof = max(t_hbm, t_tensor)
+        out[tag] = {"workload": name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "dtype": w.dtype,
+                    "ms_warm": ms_w, "ms_cold": ms_c, "tokens_per_s_cold": w.B * w.N / (ms_c * 1e-3),
+                    "tflops_cold": flops / (ms_c * 1e-3) / 1e12, "roofline_ms": t_roof,
+                    "bound": "tensor" if t_tensor > t_hbm else "hbm", "frac_cold": t_roof / ms_c,
+                    "calls": 20}
+        del s_d, K_d, V_d, Y_d, ws
+    del scrub
+    return out
 
 
 def main():
