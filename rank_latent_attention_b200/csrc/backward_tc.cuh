@@ -563,6 +563,14 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_S, i & 1, s_abort, args.wait_ns));
       if (!ok) break;
       ptx::tc_fence_after();
+      // Token pairs as packed fp32 (f32x2): the exponent argument, g - c and
+      // the product take one instruction per pair, with the same roundings
+      // as the scalar fmaf / subtract / multiply.  Columns past the last
+      // token (a ragged final tile only) give e = w = 0.
+      const bool ragged = live_cols < kBltcTok;  // uniform
+      const float4* stat4 = reinterpret_cast<const float4*>(stat);
+      const uint64_t kL2e2 = ptx::f2(kL2e, kL2e);
+      const uint64_t nL = ptx::f2(-Lm, -Lm), nc = ptx::f2(-cm, -cm);
 #pragma unroll
       for (int p = 0; p < 4; ++p) {
         float sv[16], gv[16];
@@ -572,25 +580,31 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
         uint32_t pe[8], pw[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
-          float e[2], w[2];
-#pragma unroll
-          for (int q = 0; q < 2; ++q) {
-            const int j = 16 * p + 2 * u + q;
-            float ee, ww;
-            if constexpr (kDec) {
-              const float2 tj = stat[j];
-              ee = ptx::ex2(fmaf(sv[2 * u + q], kL2e, -tj.x));
-              ww = ee * (gv[2 * u + q] - tj.y);
-            } else {
-              ee = ptx::ex2(fmaf(sv[2 * u + q], kL2e, -Lm));
-              ww = ee * (gv[2 * u + q] - cm);
-            }
-            const bool live = j < live_cols;
-            e[q] = live ? ee : 0.f;
-            w[q] = live ? ww : 0.f;
+          const int j = 16 * p + 2 * u;  // tokens j, j + 1
+          uint64_t a, b;
+          if constexpr (kDec) {
+            const float4 tj = stat4[j / 2];  // {lse3, delta} of tokens j and j + 1
+            a = ptx::fma2(ptx::f2(sv[2 * u], sv[2 * u + 1]), kL2e2, ptx::f2(-tj.x, -tj.z));
+            b = ptx::add2(ptx::f2(gv[2 * u], gv[2 * u + 1]), ptx::f2(-tj.y, -tj.w));
+          } else {
+            a = ptx::fma2(ptx::f2(sv[2 * u], sv[2 * u + 1]), kL2e2, nL);
+            b = ptx::add2(ptx::f2(gv[2 * u], gv[2 * u + 1]), nc);
           }
-          pe[u] = ptx::pack_bf16(e[0], e[1]);
-          pw[u] = ptx::pack_bf16(w[0], w[1]);
+          float a0, a1;
+          ptx::f2_split(a, a0, a1);
+          const uint64_t e = ptx::f2(ptx::ex2(a0), ptx::ex2(a1));
+          const uint64_t w = ptx::mul2(e, b);
+          float e0, e1, w0, w1;
+          ptx::f2_split(e, e0, e1);
+          ptx::f2_split(w, w0, w1);
+          if (ragged) {
+            e0 = j < live_cols ? e0 : 0.f;
+            w0 = j < live_cols ? w0 : 0.f;
+            e1 = j + 1 < live_cols ? e1 : 0.f;
+            w1 = j + 1 < live_cols ? w1 : 0.f;
+          }
+          pe[u] = ptx::pack_bf16(e0, e1);
+          pw[u] = ptx::pack_bf16(w0, w1);
         }
         // over columns of S and G this thread has already read
         ptx::tmem_st8(trow + 0 + 8 * p, pe);
