@@ -25,6 +25,11 @@ What pins what:
   the shard results combined equal the pure-Python encode over all tokens;
   each shard's log-sum-exp equals a scalar ``math.log(fsum(exp))`` and
   scipy's ``logsumexp``; one-token and empty shards take their closed forms.
+* logits past float64's exp range (up to ~1.3e3, the regime the softmaxes'
+  max shift exists for): the encode against the pure-Python brute force and
+  against the encode over the dominant tokens alone; the shards' lse against
+  scipy's logsumexp; the combined shards; the chained head finite and inside
+  the values' hull.
 * backward: torch float64 autograd through three SDPA calls; central finite
   differences of the oracle's own forward along random directions; closed
   forms (N = 1: dV = dY, dK = 0, d_seeds = 0; K = 0: dV = mean of dY,
@@ -290,6 +295,52 @@ def pin_shard_combine(o):
     assert np.all(out == 0) and np.all(np.isneginf(L))
 
 
+# ---------------------------------------------------------------- extreme logits
+def _extreme_case(seed, N=48, M=3, D=4):
+    """Logits that climb by ~25 per token past float64's exp range (up to
+    ~1.3e3), a block of four tokens (40-43) 200 above the climb, and the
+    tokens after it 400 below: only a max-shifted softmax stays finite."""
+    g = _rng(seed)
+    e = g.standard_normal(D)
+    e /= np.linalg.norm(e)
+    Q = e[None, :] + 0.02 * g.standard_normal((M, D))
+    a = 25.0 * np.arange(N, dtype=np.float64)
+    a[40:44] += 200.0
+    a[44:] -= 400.0
+    K = a[:, None] * e[None, :] + 0.02 * g.standard_normal((N, D))
+    V = g.standard_normal((N, D))
+    return Q, K, V
+
+
+def pin_extreme_logits(o):
+    from scipy.special import logsumexp
+
+    Q, K, V = _extreme_case(1100)
+    S = Q @ K.T
+    assert S.max() > 1000.0  # exp of it overflows float64
+    Z = o.flare_encode(Q, K, V)
+    assert np.all(np.isfinite(Z))
+    assert np.allclose(Z, _bf_encode(Q.tolist(), K.tolist(), V.tolist()), rtol=1e-12, atol=1e-13)
+    # every token outside 40-43 sits at least ~180 below them (weight below
+    # e^-180 of theirs): the encode over those four tokens alone agrees
+    assert np.allclose(Z, o.flare_encode(Q, K[40:44], V[40:44]), rtol=1e-13, atol=1e-14)
+    assert np.allclose(o.attention_weights(Q, K).sum(axis=1), 1.0, atol=1e-13)
+    cuts = [0, 16, 40, 48]
+    parts = [o.encode_shard(Q, K[a:b], V[a:b]) for a, b in zip(cuts[:-1], cuts[1:])]
+    for (Op, lp), a, b in zip(parts, cuts[:-1], cuts[1:]):
+        assert np.all(np.isfinite(Op)) and np.all(np.isfinite(lp)), ("shard", a, b)
+        assert np.allclose(lp, logsumexp(S[:, a:b], axis=1), rtol=1e-14, atol=1e-11), ("lse", a, b)
+        assert np.allclose(lp, _bf_lse(Q.tolist(), K[a:b].tolist()), rtol=1e-14, atol=1e-11), ("lse", a, b)
+    out, L = o.combine_shards([p[0] for p in parts], [p[1] for p in parts])
+    assert np.allclose(out, Z, rtol=1e-12, atol=1e-13)
+    assert np.allclose(L, logsumexp(S, axis=1), rtol=1e-14, atol=1e-11)
+    # the chained head: routing and decode logits grow larger still
+    Qd, Zh, Y = o.flarepp_head(Q, K, V)
+    lo, hi = V.min(axis=0), V.max(axis=0)
+    for X in (Qd, Zh, Y):
+        assert np.all(np.isfinite(X)) and np.all(X >= lo - 1e-12) and np.all(X <= hi + 1e-12)
+
+
 # ---------------------------------------------------------------- backward
 def _torch_chain_grads(seeds, K, V, dY):
     import torch
@@ -360,5 +411,6 @@ ALL_PINS = [
     pin_invariants,
     pin_mix_layout,
     pin_shard_combine,
+    pin_extreme_logits,
     pin_backward,
 ]

@@ -66,20 +66,33 @@ MUTANTS = {
     "bwd_seeds_not_summed": ("d_seeds[h] += g[0]", "d_seeds[h] = g[0]"),
     # the seed encode's key gradient taken with Q_dyn
     "bwd_seed_dk_with_qdyn": ("dK = dK + dS1.T @ seeds", "dK = dK + dS1.T @ Qd"),
+    # the following three equal the oracle in exact arithmetic and at ordinary
+    # logits; they overflow once logits pass float64's exp range
+    # softmax without its max shift
+    "softmax_no_max_shift": ("E = np.exp(S - S.max(axis=axis, keepdims=True))", "E = np.exp(S)"),
+    # shard encode without its max shift (lse then log of the plain sum)
+    "shard_no_max_shift": ("E = np.exp(S - top)\n    tot = E.sum(axis=1)\n    return (E @ V) / tot[:, None], top[:, 0] + np.log(tot)",
+                           "E = np.exp(S)\n    tot = E.sum(axis=1)\n    return (E @ V) / tot[:, None], np.log(tot)"),
+    # shard combine without its max shift
+    "combine_no_max_shift": [("w[:, live] = np.exp(lse[:, live] - top[live])", "w[:, live] = np.exp(lse[:, live])"),
+                             ("L[live] = top[live] + np.log(tot[live])", "L[live] = np.log(tot[live])")],
 }
 
 
-def _mutant(find, repl):
+def _mutant(edits):
+    """edits: one (find, replace) pair, or a list of them applied in order."""
     src = inspect.getsource(base)
-    assert src.count(find) == 1, f"mutation anchor not unique/absent: {find!r}"
+    for find, repl in ([edits] if isinstance(edits, tuple) else edits):
+        assert src.count(find) == 1, f"mutation anchor not unique/absent: {find!r}"
+        src = src.replace(find, repl)
     mod = types.ModuleType("oracle_mutant")
-    exec(compile(src.replace(find, repl), "<oracle_mutant>", "exec"), mod.__dict__)
+    exec(compile(src, "<oracle_mutant>", "exec"), mod.__dict__)
     return mod
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
 def test_mutant_is_caught(name):
-    mod = _mutant(*MUTANTS[name])
+    mod = _mutant(MUTANTS[name])
     caught = []
     for pin in oracle_pins.ALL_PINS:
         try:
