@@ -7,6 +7,7 @@ cannot tell that mistake from the definition.
 import inspect
 import types
 
+import numpy as np
 import pytest
 
 import oracle.flare_oracle as base
@@ -96,7 +97,8 @@ def test_mutant_is_caught(name):
     caught = []
     for pin in oracle_pins.ALL_PINS:
         try:
-            pin(mod)
+            with np.errstate(over="ignore", invalid="ignore", divide="ignore"):  # mutants may overflow
+                pin(mod)
         except AssertionError:
             caught.append(pin.__name__)
         except Exception as e:  # a crash on a pin input also exposes the mutant
