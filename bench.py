@@ -22,6 +22,8 @@ the data path.  Rank 0 prints one JSON line:
   timed per launch with CUDA events bracketing each launch inside a timed
   region, against the measured peaks in MEASURED_PEAKS.json;
 * cpu_baseline: the fp64 oracle on a bounded sample, on the host cores;
+  cpu_small_configs: the oracle on one head of each smaller workload, with
+  all BLAS threads and with one;
 * flare_fixed_query: FLARE with the seeds as fixed latent queries (one
   encode, one decode) on the same inputs, and the FLARE++ : FLARE step-time
   ratio;
@@ -148,6 +150,41 @@ def cpu_baseline(w):
             "sample": f"fp64 NumPy oracle ({api} BLAS, {threads} threads), one head with its first "
                       f"{CPU_SAMPLE_TOKENS} tokens, all three steps, {secs:.2f} s; tokens/s = sample tokens / "
                       f"(time x {w.H} heads) for the B={w.B}, H={w.H} workload"}
+
+
+def cpu_small_configs():
+    """The fp64 oracle on the four smaller seeded workloads, all BLAS threads
+    and one: one whole head (b, h) = (0, 0), all three steps, median of 3
+    runs; tokens/s = N / (time x H), the workload's heads run one after
+    another (its B N tokens take B H head-times)."""
+    import numpy as np
+
+    import oracle
+    from rank_latent_attention_b200 import inputs
+    from threadpoolctl import threadpool_limits
+
+    threads, api = blas_threads()
+    out = {}
+    for tag, name in SMALL_CONFIGS:
+        w = inputs.WORKLOADS[name]
+        K, V = (x.astype(np.float64) for x in inputs.make_head(w, 0, 0))
+        seeds = inputs.make_seeds(w)[0].astype(np.float64)
+
+        def head_seconds():
+            runs = []
+            for _ in range(3):
+                t0 = time.perf_counter()
+                oracle.flarepp_head(seeds, K, V)
+                runs.append(time.perf_counter() - t0)
+            return statistics.median(runs)
+
+        secs_all = head_seconds()
+        with threadpool_limits(limits=1):
+            secs_one = head_seconds()
+        out[tag] = {"workload": name, "tokens_per_s": w.N / (secs_all * w.H), "threads": threads,
+                    "tokens_per_s_1_thread": w.N / (secs_one * w.H), "head_ms": secs_all * 1e3,
+                    "head_ms_1_thread": secs_one * 1e3, "blas": api}
+    return out
 
 
 def run_reference(args):
@@ -590,6 +627,7 @@ def run_native(args):
     line["small_configs"] = small_configs(torch, flare, inputs, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
+        line["cpu_small_configs"] = cpu_small_configs()
     print(json.dumps(line), flush=True)
 
 
