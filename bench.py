@@ -627,7 +627,10 @@ def run_native(args):
     line["small_configs"] = small_configs(torch, flare, inputs, dev, peaks)
     if world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w)
-        line["cpu_small_configs"] = cpu_small_configs()
+        try:  # auxiliary: a failure here must not cost the line
+            line["cpu_small_configs"] = cpu_small_configs()
+        except Exception as e:
+            line["cpu_small_configs"] = {"error": f"{type(e).__name__}: {e}"}
     print(json.dumps(line), flush=True)
 
 
