@@ -84,7 +84,7 @@ WORKLOADS: dict[str, Workload] = {
     ]
 }
 
-_TENSOR_ID = {"seeds": 0, "K": 1, "V": 2, "outliers": 3, "mesh": 4, "dY": 5}
+_TENSOR_ID = {"seeds": 0, "K": 1, "V": 2, "outliers": 3, "mesh": 4, "dY": 5, "climb": 6}
 
 
 def custom(B, H, N, M, D, dtype="bf16", kind="gauss", seed_index=99, scale=None) -> Workload:
@@ -171,6 +171,30 @@ def make_upstream(w: Workload) -> np.ndarray:
         for h in range(w.H):
             dY[b, h] = _rng(w, "dY", b, h).standard_normal((w.N, w.D), dtype=np.float32)
     return _round(dY, w.dtype)
+
+
+def make_climbing(H: int, N: int, M: int, D: int, jump_tile: int, seed_index: int = 131):
+    """Encode inputs whose logits climb along the tokens (bf16, B = 1).
+
+    Query m is e + Q~_m / 4 and key n is a_n e + K_n, with e a seeded unit
+    vector and Q~, K, V a Gaussian workload's.  a_n = 6 t + 2 z_n for token n
+    of 64-token tile t (z ~ N(0, 1)), plus 120 in tile jump_tile and minus 60
+    in the tiles after it, so the logits of token n sit near a_n for every
+    query.  Returns (Q [H,M,D], K [1,H,N,D], V [1,H,N,D]) as float32 holding
+    bf16-exact values.
+    """
+    w = custom(1, H, N, M, D, dtype="bf16", seed_index=seed_index)
+    seeds, K, V = make_inputs(w)
+    g = _rng(w, "climb")
+    e = g.standard_normal(D)
+    e /= np.linalg.norm(e)
+    tile = np.arange(N) // 64
+    a = 6.0 * tile + 2.0 * g.standard_normal(N)
+    a[tile == jump_tile] += 120.0
+    a[tile > jump_tile] -= 60.0
+    Q = e[None, None, :] + 0.25 * seeds.astype(np.float64)
+    Kc = a[None, None, :, None] * e + K.astype(np.float64)
+    return _round(Q.astype(np.float32), "bf16"), _round(Kc.astype(np.float32), "bf16"), V
 
 
 def make_inputs(w: Workload, threads: int | None = None):

@@ -201,45 +201,19 @@ def test_split_counts_agree(name, splits):
     assert_stated("Y", to_host(Y), Yo, w.dtype)
 
 
-def _climbing_logits(H, N, M, D, jump_tile):
-    """Encode inputs whose logits climb along the tokens.
-
-    Every query is a common unit direction e plus Gaussian noise, and key n is
-    a_n e plus Gaussian noise, so the logits of token n sit near a_n for every
-    latent.  a_n rises by about 6 (natural log units) per 64-token tile, so a
-    running reference set on an early tile falls behind by 2^32 within a few
-    tiles; tile jump_tile jumps about 120 above the ramp, past the fp32 range
-    of 2^(x - reference) for any earlier reference; the tiles after it fall
-    back below the ramp.  Returned rounded to bf16 as float32.
-    """
-    import torch
-
-    w = inputs.custom(1, H, N, M, D, dtype="bf16", seed_index=131)
-    seeds, K, V = inputs.make_inputs(w)
-    rng = np.random.default_rng(131)
-    e = rng.standard_normal(D)
-    e /= np.linalg.norm(e)
-    tile = np.arange(N) // 64
-    a = 6.0 * tile + 2.0 * rng.standard_normal(N)
-    a[tile == jump_tile] += 120.0
-    a[tile > jump_tile] -= 60.0
-    Q = e[None, None, :] + 0.25 * seeds.astype(np.float64)       # [H, M, D]
-    Kc = a[None, None, :, None] * e + K.astype(np.float64)       # [1, H, N, D]
-    rnd = lambda x: torch.from_numpy(np.ascontiguousarray(x, dtype=np.float32)).bfloat16().float().numpy()
-    return rnd(Q), rnd(Kc), V
-
-
 @pytest.mark.parametrize("M,D", [(256, 64), (64, 64), (144, 32), (256, 16), (128, 128)])
 @pytest.mark.parametrize("splits", [1, 0])
 def test_encode_reference_far_behind(M, D, splits):
     """The encode keeps each row's running reference until a tile's sum of
     2^(x log2e - reference) leaves [0, 2^32]; then it takes the tile's max.
-    Logits that climb tile after tile, and one tile that jumps past the fp32
-    range, exercise that fallback (one CTA per head, so every tile after the
-    first goes through it; and the default split count)."""
+    Logits that climb about 6 per 64-token tile (inputs.make_climbing: a
+    reference falls 2^32 behind within a few tiles) and one tile that jumps
+    120 higher, past the fp32 range of 2^(x - reference), exercise that
+    fallback: with one CTA per head every tile after the first goes through
+    it; and with the default split count.  D = 128 always takes the max."""
     require_cuda()
     H, N = 2, 64 * 70 + 37
-    Q, K, V = _climbing_logits(H, N, M, D, jump_tile=50)
+    Q, K, V = inputs.make_climbing(H, N, M, D, jump_tile=50)
     old = flare.flare_set_split_override(splits)
     try:
         Z = flare.flare_encode(to_dev(Q, "bf16"), to_dev(K, "bf16"), to_dev(V, "bf16"))
