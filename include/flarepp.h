@@ -299,8 +299,12 @@ int flare_last_launch_count(void);
 
 /*
  * Tuning / test hooks (process-wide, not thread-safe against concurrent calls):
- *   flare_set_split_override(s): use s CTAs per head along the tokens (clamped
- *     to the number of 128-token tiles); 0 restores the built-in choice.
+ *   flare_set_split_override(s): use s CTAs per head along the tokens in
+ *     every token-split kernel, each clamped to that kernel's number of token
+ *     tiles (64 tokens for the encode and the backward's latent-side kernel,
+ *     128 for the decode, the statistics and the token-gradient kernels); 0
+ *     restores the built-in choice (whole waves of the SMs' resident CTA
+ *     slots, at most ~32k tokens per CTA).
  *   flare_set_wait_limit_ms(ms): how long a tensor-core kernel waits on one
  *     barrier before recording FLARE_ERR_TIMEOUT and returning (default 2000).
  * Both return the previous value.
