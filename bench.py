@@ -20,7 +20,12 @@ the data path.  Rank 0 prints one JSON line:
   the timed region (the library overlaps them with the compute, head by head);
 * roofline: the dominant kernel (the tcgen05 encode, launched twice a step),
   timed per launch with CUDA events bracketing each launch inside a timed
-  region, against the measured peaks in MEASURED_PEAKS.json;
+  region, against the measured peaks in MEASURED_PEAKS.json: the burst GEMM
+  figure when the SM clock sampled under load stayed within 5% of its
+  maximum, the sustained (power-capped) one otherwise;
+* step_roofline: the whole step (the three chained steps of the mixer, its
+  unit of work) against the slower of its tensor and HBM bounds, with the
+  same choice of peak and the fraction against each measured figure;
 * cpu_baseline: the fp64 oracle on a bounded sample, on the host cores;
   cpu_small_configs: the oracle on one head of each smaller workload, with
   all BLAS threads and with one;
@@ -110,6 +115,38 @@ def measured_peaks():
             p = json.load(f)
         return p, "measured"
     return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}, "fallback"
+
+
+def tensor_peak_for_clocks(peaks, clk):
+    """(bf16 GEMM peak in TFLOP/s, which one) for the clocks sampled under load."""
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    mhz, top = clk.get("sm_mhz"), clk.get("sm_max_mhz")
+    if mhz and top and mhz >= 0.95 * top:
+        return burst, f"burst (median SM clock {mhz:.0f} of {top:.0f} MHz)"
+    if mhz and top:
+        return sustained, f"sustained (median SM clock {mhz:.0f} of {top:.0f} MHz, power-capped)"
+    return burst, "burst (no clock record)"
+
+
+def step_roofline(flops, nbytes, ms, peaks, peak_kind, tensor_peak, tensor_peak_kind):
+    """The whole flarepp_mix step against the slower of its tensor and HBM bounds.
+
+    frac uses the GEMM peak that matches the sampled clocks; frac_burst and
+    frac_sustained give it against each measured figure."""
+    t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9)
+
+    def t_roof(tf):
+        return max(flops / (tf * 1e12), t_hbm)
+
+    t = t_roof(tensor_peak)
+    burst = peaks["bf16_tflops"]
+    sustained = peaks.get("bf16_tflops_sustained", burst)
+    return {"t_roofline_ms": t * 1e3, "bound": "tensor" if flops / (tensor_peak * 1e12) >= t_hbm else "hbm",
+            "frac": t * 1e3 / ms, "frac_burst": t_roof(burst) * 1e3 / ms,
+            "frac_sustained": t_roof(sustained) * 1e3 / ms, "tensor_peak_tflops": tensor_peak,
+            "tensor_peak": tensor_peak_kind, "hbm_peak_gbs": peaks["hbm_gbs"], "peaks": peak_kind,
+            "achieved_tflops": flops / (ms * 1e-3) / 1e12}
 
 
 def blas_threads():
@@ -546,9 +583,12 @@ def run_native(args):
     value = ranks.job_tokens_per_s(w.N, env, ms)  # B = 1 per rank
     flops_step = 12.0 * w.N * w.M * w.D * w.H * world
     bytes_step = 12.0 * w.N * w.D * w.H * world  # K,V + K,V + K + Y, bf16
-    # every number here is timed inside a long run of steps: the sustained
-    # (power-capped) GEMM peak is the matching denominator
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    # The GEMM peak that matches the clocks this run saw: the burst figure
+    # when the sampled SM clock under load stayed within 5% of its maximum
+    # (a short timed region at full clock), the sustained (power-capped) one
+    # when the clocks sat lower.  Both fractions are reported.
+    clk = clocks.summary()
+    tensor_peak, tensor_peak_kind = tensor_peak_for_clocks(peaks, clk)
     t_tensor = flops_step / world / (tensor_peak * 1e12)
     t_hbm = bytes_step / world / (peaks["hbm_gbs"] * 1e9)
     # dominant kernel: the encode (two launches per step); algorithmic work per launch
@@ -568,12 +608,11 @@ def run_native(args):
     roof["algorithmic_bytes"] = enc_bytes
     roof["kernel"] = "encode_tc"
     roof["ms_per_launch"] = enc_ms
-    roof["peak_source"] = f"{peak_kind} (sustained bf16 GEMM / STREAM copy)"
+    roof["peak_source"] = f"{peak_kind}: {tensor_peak_kind} bf16 GEMM / STREAM copy"
     # The exponential unit binds in practice: one 2^x per score, N*M per head
     # per encode launch, at 16 results per clock per SM (MUFU ex2) on 148 SMs.
     # Peak at the maximum SM clock; frac_at_clock uses the median SM clock
     # sampled under load (the kernels run power-capped).
-    clk = clocks.summary()
     exps = float(w.N) * w.M * w.H
     alu_peak = 16.0 * 148 * (clk["sm_max_mhz"] or 1965.0) * 1e6  # 1965 MHz: the B200's clocks.max.sm
     alu_at_clock = 16.0 * 148 * clk["sm_mhz"] * 1e6 if clk.get("sm_mhz") else None
@@ -598,8 +637,8 @@ def run_native(args):
                    "D": w.D, "parallelism": f"batch-sharded x{world}, no collectives",
                    "l2": "inputs (4.3 GB K/V per step) larger than L2; no flush"},
         "tflops": flops_step / (ms * 1e-3) / 1e12,
-        "step_roofline": {"t_roofline_ms": max(t_tensor, t_hbm) * 1e3, "bound": "tensor" if t_tensor >= t_hbm else "hbm",
-                          "frac": max(t_tensor, t_hbm) * 1e3 / ms, "peaks": peak_kind},
+        "step_roofline": step_roofline(flops_step / world, bytes_step / world, ms, peaks, peak_kind, tensor_peak,
+                                       tensor_peak_kind),
         "roofline": roof,
         "alu_roofline": alu_roof,
         "kernel_ms_per_step": step_kernel_ms,
@@ -642,12 +681,13 @@ L2_SCRUB_BYTES = 256 << 20  # written before each L2-cold call: twice the 126 MB
 def small_configs(torch, flare, inputs, dev, peaks):
     """One flarepp_mix call per small workload: median of 20 event-timed calls
     after 3 warm-ups, L2-warm and L2-cold.  Roofline per call: the larger of
-    12 N M D B H FLOP at the sustained bf16 GEMM peak (bf16 workloads) and
-    the single-pass bytes (K and V read once, Y written once) at the measured
-    copy bandwidth; these heads fit in L2, so one pass is the minimum."""
+    12 N M D B H FLOP at the burst bf16 GEMM peak (bf16 workloads; each call
+    is a short region timed alone) and the single-pass bytes (K and V read
+    once, Y written once) at the measured copy bandwidth; these heads fit in
+    L2, so one pass is the minimum."""
     scrub = torch.empty(L2_SCRUB_BYTES, dtype=torch.uint8, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    tensor_peak = peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"])
+    tensor_peak = peaks["bf16_tflops"]
     out = {}
     for tag, name in SMALL_CONFIGS:
         w = inputs.WORKLOADS[name]

@@ -30,6 +30,19 @@ __device__ int g_status[2];  // {first error code, site} per device
 std::atomic<int> g_split_override{0};
 std::atomic<int> g_wait_ms{2000};
 thread_local int t_last_launches = 0;
+// The split override as this thread's current entry-point call first read
+// it (-1 outside a call): every split count inside one call, the workspace
+// check's and the kernels' alike, comes from the same value even if another
+// thread changes the override meanwhile.
+thread_local int t_split_pin = -1;
+
+struct SplitPin {
+  int prev;
+  SplitPin() : prev(t_split_pin) {
+    if (prev < 0) t_split_pin = g_split_override.load();
+  }
+  ~SplitPin() { t_split_pin = prev; }
+};
 
 constexpr int kMaxDevices = 64;
 
@@ -69,7 +82,10 @@ int* status_ptr() {
   std::lock_guard<std::mutex> lock(mu);
   if (!ptrs[dev]) {
     void* p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return nullptr;
+    if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) {
+      cudaGetLastError();  // the failed lookup must not read as a later launch's error
+      return nullptr;
+    }
     ptrs[dev] = static_cast<int*>(p);
   }
   return ptrs[dev];
@@ -109,7 +125,7 @@ bool device_ptr(const void* p) {
 // `tile` is the kernel's token tile (64 for the encode, 128 for the decode).
 int choose_splits(int BH, int64_t N, int tile, int per_sm = 1) {
   const int64_t tiles = ceil_div(N, tile);
-  int64_t s = g_split_override.load();
+  int64_t s = t_split_pin >= 0 ? t_split_pin : g_split_override.load();
   if (s <= 0) {
     const int64_t slots = int64_t(sm_count()) * per_sm;
     const int64_t waves = std::max<int64_t>(1, ceil_div(BH * tiles, slots * (32768 / tile)));
@@ -970,17 +986,20 @@ __global__ void empty_shard_kernel(float* O, float* lse, size_t rows, int D) {
 extern "C" {
 
 size_t flare_encode_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  SplitPin pin;
   if (check_sizes(B, H, N, M, D, dtype)) return 0;
   return encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
 }
 
 size_t flarepp_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  SplitPin pin;
   if (check_sizes(B, H, N, M, D, dtype)) return 0;
   return mix_ws_bytes(B, H, N, M, D, dtype);
 }
 
 int flare_encode(const void* Q, int q_batched, const void* K, const void* V, void* Z, int B, int H, int64_t N,
                  int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
@@ -1002,6 +1021,7 @@ int flare_encode(const void* Q, int q_batched, const void* K, const void* V, voi
 }
 
 size_t flare_encode_lse_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  SplitPin pin;
   if (N <= 0) return 0;  // an empty shard needs none
   if (check_sizes(B, H, N, M, D, dtype)) return 0;
   return encode_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
@@ -1010,6 +1030,7 @@ size_t flare_encode_lse_workspace_size(int B, int H, int64_t N, int M, int D, in
 int flare_encode_lse(const void* Q, int q_batched, const void* K, const void* V, float* O, float* lse, int B,
                      int H, int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes,
                      void* stream) {
+  SplitPin pin;
   if (N < 0) return FLARE_ERR_INVALID_ARG;
   int rc = check_sizes(B, H, N == 0 ? 1 : N, M, D, dtype);
   if (rc) return rc;
@@ -1067,6 +1088,7 @@ int flare_lse_combine(const float* O_parts, const float* lse_parts, int R, int64
 }
 
 size_t flarepp_mix_backward_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  SplitPin pin;
   if (check_sizes(B, H, N, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
   return backward_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
 }
@@ -1074,6 +1096,7 @@ size_t flarepp_mix_backward_workspace_size(int B, int H, int64_t N, int M, int D
 int flarepp_mix_backward(const void* seeds, const void* K, const void* V, const void* dY, void* d_seeds, void* dK,
                          void* dV, int B, int H, int64_t N, int M, int D, int dtype, void* workspace,
                          size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
@@ -1102,6 +1125,7 @@ size_t flarepp_saved_bytes(int B, int H, int M, int D, int dtype) {
 
 int flarepp_mix_save(const void* seeds, const void* K, const void* V, void* Y, void* saved, int B, int H, int64_t N,
                      int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
@@ -1113,6 +1137,7 @@ int flarepp_mix_save(const void* seeds, const void* K, const void* V, void* Y, v
 int flarepp_mix_backward_saved(const void* seeds, const void* K, const void* V, const void* dY, const void* saved,
                                void* d_seeds, void* dK, void* dV, int B, int H, int64_t N, int M, int D, int dtype,
                                void* workspace, size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
@@ -1141,6 +1166,7 @@ size_t flarepp_backward_shard_exchange_floats(int B, int H, int M, int D) {
 }
 
 size_t flarepp_backward_shard_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  SplitPin pin;
   if (N < 0 || check_sizes(B, H, N == 0 ? 1 : N, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
   return backward_ws_layout(nullptr, B * H, N, M, D, dtype).bytes;
 }
@@ -1149,6 +1175,7 @@ int flarepp_mix_backward_shard(int phase, const void* seeds, const void* K, cons
                                const void* saved, float* exchange, void* d_seeds, void* dK, void* dV, int B, int H,
                                int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes,
                                void* stream) {
+  SplitPin pin;
   if (phase < 0 || phase > 3 || N < 0) return FLARE_ERR_INVALID_ARG;
   int rc = check_sizes(B, H, N == 0 ? 1 : N, M, D, dtype);
   if (rc) return rc;
@@ -1170,6 +1197,7 @@ int flarepp_mix_backward_shard(int phase, const void* seeds, const void* K, cons
 
 int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N,
                  int M, int D, int dtype, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
@@ -1183,22 +1211,26 @@ int flare_decode(const void* K, const void* Q, int q_batched, const void* Z, voi
 
 int flarepp_mix(const void* seeds, const void* K, const void* V, void* Y, int B, int H, int64_t N, int M, int D,
                 int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   return mix_impl(seeds, K, V, Y, nullptr, nullptr, B, H, N, M, D, dtype, workspace, workspace_bytes, stream);
 }
 
 int flarepp_mix_debug(const void* seeds, const void* K, const void* V, void* Y, void* Q_dyn, void* Z, int B, int H,
                       int64_t N, int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   if (!Q_dyn || !Z) return FLARE_ERR_INVALID_ARG;
   return mix_impl(seeds, K, V, Y, Q_dyn, Z, B, H, N, M, D, dtype, workspace, workspace_bytes, stream);
 }
 
 size_t flare_communication_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  SplitPin pin;
   if (check_sizes(B, H, N, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
   return comm_ws_layout(B, H, N, M, D, dtype).bytes;
 }
 
 int flare_communication_matrix(const void* Q, int q_batched, const void* K, void* C, int B, int H, int64_t N, int M,
                                int D, int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
@@ -1221,12 +1253,14 @@ int flare_communication_matrix(const void* Q, int q_batched, const void* K, void
 }
 
 size_t flarepp_mix_host_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
+  SplitPin pin;
   if (check_sizes(B, H, N, M, D, dtype)) return 0;
   return host_ws_layout(H, N, M, D, dtype).bytes;
 }
 
 int flarepp_mix_host(const void* seeds, const void* K, const void* V, void* Y, int B, int H, int64_t N, int M, int D,
                      int dtype, void* workspace, size_t workspace_bytes, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (!host_ptr(seeds) || !host_ptr(K) || !host_ptr(V) || !host_ptr(Y)) return FLARE_ERR_INVALID_ARG;
@@ -1402,6 +1436,7 @@ char* noalloc_scratch() {
 
 extern "C" int flare_encode_noalloc(const void* Q, int q_batched, const void* K, const void* V, void* Z, int B,
                                     int H, int64_t N, int M, int D, int dtype, void* stream) {
+  SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
   if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
