@@ -29,10 +29,16 @@
  *   the tensor cores; intermediates Q_dyn and Z are stored as bf16, rounded to
  *   nearest, as three chained bf16 SDPA calls would return them) or FLARE_F32
  *   (fp32 everywhere, CUDA-core path); every tensor of a call has that dtype.
- *   FLARE_BF16_F32OUT (flarepp_mix / flarepp_mix_debug only) takes bf16 seeds,
- *   K and V and computes, stores Q_dyn and Z, and writes Y in fp32 on the
- *   CUDA cores: for inputs whose outputs are so heavy-tailed that bf16
- *   storage of Y alone exceeds an accuracy budget.
+ *   FLARE_BF16_F32OUT (flarepp_mix / flarepp_mix_debug / flarepp_mix_host
+ *   only) takes bf16 seeds, K and V and returns Q_dyn, Z and Y in fp32: for
+ *   inputs whose outputs are so heavy-tailed (or whose logits are so large)
+ *   that bf16 storage of the chain exceeds an accuracy budget.  For
+ *   M % 16 == 0 and D <= 64 it runs on the tensor cores in split precision:
+ *   the rounded MMA operands are carried as pairs hi = round(x),
+ *   lo = round(x - hi) of 16-bit numbers and each product takes one MMA per
+ *   part (the encodes' softmax weights and Q_dyn as bf16 pairs, Z as an fp16
+ *   pair scaled per head by a power of two; the decode's weights, in [0, 1],
+ *   as fp16).  Other sizes run on the fp32 CUDA-core kernels.
  * - Supported sizes: B >= 1, H >= 1, B*H <= 65535, 1 <= N < 2^31 - 256,
  *   D in {16, 32, 64, 128}, 1 <= M <= 256; for FLARE_BF16 additionally
  *   M % 16 == 0.  N needs no alignment: the last tile of each head is masked.
@@ -63,7 +69,7 @@ extern "C" {
 typedef enum {
   FLARE_F32 = 0,         /* fp32 storage and arithmetic (CUDA cores)                            */
   FLARE_BF16 = 1,        /* bf16 storage; tcgen05 bf16 MMAs, fp32 accumulation and softmax      */
-  FLARE_BF16_F32OUT = 2  /* flarepp_mix only: bf16 seeds/K/V; fp32 arithmetic, fp32 Q_dyn, Z, Y */
+  FLARE_BF16_F32OUT = 2  /* mixer only: bf16 seeds/K/V; split-precision MMAs, fp32 Q_dyn, Z, Y   */
 } flare_dtype_t;
 
 typedef enum {

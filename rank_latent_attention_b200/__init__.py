@@ -40,7 +40,6 @@ __all__ = [
     "flarepp_workspace_size",
     "flarepp_mix_host",
     "flare_communication_matrix",
-    "flare_communication_eigenvalues",
     "flare_check_status",
     "flare_last_launch_count",
     "flare_set_split_override",
@@ -379,8 +378,10 @@ def flare_communication_matrix(Q, K, C=None, *, workspace=None, stream=None):
     """C = softmax_N(Q K^T) softmax_M(K Q^T) per head: [B,H,M,M], row-stochastic.
 
     Its eigenvalues are the nonzero eigenvalues of the rank-M token-to-token
-    communication matrix W = W_dec W_enc.  Q is [H,M,D] (shared) or
-    [B,H,M,D] (e.g. FLARE++'s routing queries Q_dyn)."""
+    communication matrix W = W_dec W_enc; the library forms C (the O(M^2 N)
+    part) and leaves the O(M^3) eigen-solve of the small M x M matrices to the
+    caller.  Q is [H,M,D] (shared) or [B,H,M,D] (e.g. FLARE++'s routing
+    queries Q_dyn)."""
     torch = _torch()
     B, H, N, D = K.shape
     q_batched = 1 if Q.dim() == 4 else 0
@@ -392,18 +393,6 @@ def flare_communication_matrix(Q, K, C=None, *, workspace=None, stream=None):
                                             _ptr(C, "C", K.dtype), B, H, N, M, D, _dtype_code(K), ws, wsb,
                                             _stream(stream)), "flare_communication_matrix")
     return C
-
-
-def flare_communication_eigenvalues(Q, K, *, stream=None):
-    """Eigenvalues of each head's communication matrix, [B,H,M] complex128,
-    sorted by decreasing modulus.  The O(M^2 N) product C runs in the
-    library's kernels; the O(M^3) eigen-solve of the M x M matrices is a
-    LAPACK call on the host (torch.linalg.eigvals in float64)."""
-    torch = _torch()
-    C = flare_communication_matrix(Q, K, stream=stream)
-    ev = torch.linalg.eigvals(C.to("cpu", torch.float64))
-    order = torch.argsort(ev.abs(), dim=-1, descending=True)
-    return torch.gather(ev, -1, order)
 
 
 def _mix_mode(K, out_dtype):
@@ -419,7 +408,7 @@ def _mix_mode(K, out_dtype):
 def flarepp_mix(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, stream=None):
     """FLARE++ mixer forward: seeds [H,M,D], K/V [B,H,N,D] -> Y [B,H,N,D].
 
-    out_dtype=torch.float32 with bf16 inputs selects the fp32-arithmetic,
+    out_dtype=torch.float32 with bf16 inputs selects the split-precision,
     fp32-output mode (FLARE_BF16_F32OUT)."""
     torch = _torch()
     B, H, N, D = K.shape

@@ -37,7 +37,24 @@
 // P of group 1 at [3 MP / 4, MP) (its chunks processed last to first, so each
 // P chunk lands on scores already read); O at kColO: [MP / 4, MP / 4 + D) for
 // MP = 256 (free once both groups have stored P), [128, 128 + D) for MP = 128.
+//
+// Split precision (PREC = 1).  Each rounded MMA operand is carried as a pair
+// hi + lo of 16-bit numbers (hi = round(x), lo = round(x - hi)), and each
+// product takes one MMA per part:
+//   S = K Q_hi^T + K Q_lo^T          Q_dyn as a bf16 pair (K is exact bf16);
+//   O = P Z_hi + P Z_lo              P and Z in fp16, on kind::f16 with fp16
+//                                    operands.
+// P lies in [0, 1] (the row max is subtracted exactly), so fp16 holds it to
+// 2^-11 relative, 8x finer than bf16, in the same 16 bits of TMEM: the slot
+// layout above is unchanged.  Z is read as fp32 from global memory; each CTA
+// scales its head's Z by 2^-e, with e chosen from the head's max|Z| so that
+// the scaled values lie below 2^15 (inside fp16's range, whatever the inputs'
+// range), writes the fp16 pair into shared memory in the swizzled layout the
+// tensor map would have produced, and multiplies Y by 2^e in the epilogue.
+// Y is written in fp32 (16-byte stores of four floats).
 #pragma once
+
+#include <cuda_fp16.h>
 
 #include "common.cuh"
 
@@ -50,7 +67,8 @@ struct DecodeArgs {
   int H;
   int splits;
   int tiles;
-  __nv_bfloat16* Y;  // [BH][N][D]
+  void* Y;  // [BH][N][D]: bf16, or fp32 with split precision
+  const float* Zf;  // split precision: Z as fp32 [BH][M][D] (the bf16 Z map is unused)
   int* status;
   unsigned long long wait_ns;
 };
@@ -60,10 +78,11 @@ struct DecodeArgs {
 // difference, 2/16 is slower, 5/16 much slower).
 constexpr uint32_t kDecPolyPairs = 0x0000u;
 
-template <int D, int MP, int NS>
+template <int D, int MP, int NS, int PREC = 0>
 struct DecodeCfg {
   using G = TileGeom<D>;
   static_assert(MP == 128 || MP == 256, "padded latent count");
+  static constexpr int kLatParts = PREC ? 2 : 1;  // Q_dyn and Z as hi (+ lo)
   static constexpr int kHalf = MP / 2;      // latents per group
   static constexpr int kChunks = kHalf / 32;  // 32-latent chunks per group
   static constexpr int kProducerWarp = 16;
@@ -73,14 +92,17 @@ struct DecodeCfg {
   static constexpr int kTileBytes = G::bytes(kTileN);
   static constexpr int kOffQ = 0;
   static constexpr int kOffZ = kLatBytes;
-  static constexpr int kOffStages = 2 * kLatBytes;
+  static constexpr int kOffQlo = 2 * kLatBytes;  // split precision only
+  static constexpr int kOffZlo = 3 * kLatBytes;
+  static constexpr int kOffStages = 2 * kLatParts * kLatBytes;
   static constexpr int kOffBars = kOffStages + NS * kTileBytes;
   // full[NS], empty[NS], qz_full, S_full[2], P_full[2], O_full[2], O_free[2], turn[2], drain
   static constexpr int kNumBars = 2 * NS + 12;
   static constexpr int kOffXM = kOffBars + 8 * kNumBars;  // float [2 slot][2 half][128]: half-row max
   static constexpr int kOffXL = kOffXM + 2 * 2 * 128 * 4;  // float [2 slot][2 half][128]: half-row sum
   static constexpr int kOffMisc = kOffXL + 2 * 2 * 128 * 4;
-  static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
+  static constexpr int kOffRed = kOffMisc + 16;  // float [16]: per-warp max|Z| (split precision)
+  static constexpr int kSmemBytes = kOffRed + 64 + 1024;
   static constexpr uint32_t kTmemCols = 512;
   static constexpr uint32_t kSlotCols = 256;
   static constexpr uint32_t kColP1 = 3 * MP / 4;
@@ -89,7 +111,10 @@ struct DecodeCfg {
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
   static constexpr uint32_t kIdescQK = ptx::idesc_bf16(kTileN, MP, 0, 0);
   static constexpr uint32_t kIdescQKHalf = ptx::idesc_bf16(kTileN, kLatRows, 0, 0);  // one latent half
-  static constexpr uint32_t kIdescPV = ptx::idesc_bf16(kTileN, D, 0, 1);
+  static constexpr uint32_t kIdescPV = PREC ? ptx::idesc_f16(kTileN, D, 0, 1) : ptx::idesc_bf16(kTileN, D, 0, 1);
+  // qz_full: the producer's expect_tx arrival, plus (split precision) one per
+  // softmax warp once its part of the fp16 Z is in shared memory
+  static constexpr int kQzArrivals = PREC ? 1 + 16 : 1;
   // TMEM column (within the slot) of P for latents [16 kk, +16): the PV K step kk
   __host__ __device__ static constexpr uint32_t col_pk(int kk) {
     return kk < MP / 32 ? 8 * kk : kColP1 + 8 * (kk - MP / 32);
@@ -99,7 +124,7 @@ struct DecodeCfg {
 // P for one 32-latent chunk of a row: 2^(x log2e - mref) for the valid
 // columns (16-column groups at or past M give P = 0), packed to bf16 pairs
 // into 16 TMEM columns at tP; returns the fp32 sum.
-template <int MP>
+template <int MP, bool F16P = false>
 __device__ __forceinline__ float decode_exp_chunk(const float* x, float mref, int col0, int M, uint32_t tP) {
   const uint64_t kL2 = ptx::f2(kLog2e, kLog2e);
   const uint64_t nn = ptx::f2(-mref, -mref);
@@ -123,7 +148,7 @@ __device__ __forceinline__ float decode_exp_chunk(const float* x, float mref, in
         ps[u & 1] = ptx::add2(ps[u & 1], e);
         float e0, e1;
         ptx::f2_split(e, e0, e1);
-        p[u] = ptx::pack_bf16(e0, e1);
+        p[u] = F16P ? ptx::pack_f16(e0, e1) : ptx::pack_bf16(e0, e1);
       }
     } else {
 #pragma unroll
@@ -137,10 +162,77 @@ __device__ __forceinline__ float decode_exp_chunk(const float* x, float mref, in
   return (s0 + s1) + (s2 + s3);
 }
 
+// Split precision: the head's fp32 Z [M][D] (rows past M as zeros), scaled by
+// 2^-e with e = the exponent that puts the head's max|Z| in [2^14, 2^15),
+// into shared memory as an fp16 pair (hi at kOffZ, lo at kOffZlo) in the
+// layout a TMA load with the tile's swizzle produces (16-byte chunks of a row
+// permuted by address bits 7 and up); run by the 512 softmax threads (tid),
+// returns 2^e.  Every thread fences its stores for the tensor core's reads.
+template <int D, int MP, int NS, int PREC>
+__device__ __forceinline__ float stage_z_f16(const DecodeArgs& args, uint8_t* smem, int tid) {
+  using C = DecodeCfg<D, MP, NS, PREC>;
+  using G = typename C::G;
+  static_assert(D <= 64, "one column block");
+  constexpr int kRowChunks = D / 8;  // 16-byte chunks of 8 fp16 per row
+  constexpr int kChunks = MP * kRowChunks;
+  constexpr uint32_t kSwzMask = G::kSwizzle == 2u ? 7u : (G::kSwizzle == 4u ? 3u : 1u);  // 128 / 64 / 32 B
+  float* red = reinterpret_cast<float*>(smem + C::kOffRed);
+  const float* Zh = args.Zf + static_cast<size_t>(blockIdx.y) * args.M * D;
+  float mx = 0.f;
+  for (int q = tid; q < kChunks; q += 512) {
+    const int row = q / kRowChunks;
+    if (row < args.M) {
+      const float4* src = reinterpret_cast<const float4*>(Zh + static_cast<size_t>(row) * D + (q % kRowChunks) * 8);
+      const float4 a = src[0], b = src[1];
+      mx = fmaxf(mx, ptx::max3(ptx::max3(fabsf(a.x), fabsf(a.y), fabsf(a.z)), ptx::max3(fabsf(a.w), fabsf(b.x), fabsf(b.y)),
+                               fmaxf(fabsf(b.z), fabsf(b.w))));
+    }
+  }
+#pragma unroll
+  for (int o = 16; o; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  if ((tid & 31) == 0) red[tid >> 5] = mx;
+  asm volatile("bar.sync 5, 512;" ::: "memory");
+#pragma unroll
+  for (int w = 0; w < 16; ++w) mx = fmaxf(mx, red[w]);
+  int e = 0;
+  if (mx > 0.f && mx <= 3.4e38f) {
+    int ex;
+    frexpf(mx, &ex);  // mx = f 2^ex, f in [1/2, 1)
+    e = ex - 15;
+  }
+  const float down = ldexpf(1.f, -e);
+  for (int q = tid; q < kChunks; q += 512) {
+    const int row = q / kRowChunks, ch = q % kRowChunks;
+    float v[8];
+    if (row < args.M) {
+      const float4* src = reinterpret_cast<const float4*>(Zh + static_cast<size_t>(row) * D + ch * 8);
+      const float4 a = src[0], b = src[1];
+      v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+    } else {
+#pragma unroll
+      for (int z = 0; z < 8; ++z) v[z] = 0.f;
+    }
+    uint32_t hi[4], lo[4];
+#pragma unroll
+    for (int z = 0; z < 4; ++z) {
+      const float a = v[2 * z] * down, b = v[2 * z + 1] * down;
+      hi[z] = ptx::pack_f16(a, b);
+      const float2 h = __half22float2(*reinterpret_cast<const __half2*>(&hi[z]));
+      lo[z] = ptx::pack_f16(a - h.x, b - h.y);
+    }
+    const uint32_t lin = static_cast<uint32_t>(row * G::kRowBytes + ch * 16);
+    const uint32_t off = lin ^ (((lin >> 7) & kSwzMask) << 4);
+    *reinterpret_cast<uint4*>(smem + C::kOffZ + off) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+    *reinterpret_cast<uint4*>(smem + C::kOffZlo + off) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+  }
+  ptx::fence_proxy_async_smem();
+  return ldexpf(1.f, e);
+}
+
 // The softmax / epilogue loop of one group (slot s, latent half CH).
-template <int D, int MP, int NS>
+template <int D, int MP, int NS, int PREC>
 struct DecodeGroup {
-  using C = DecodeCfg<D, MP, NS>;
+  using C = DecodeCfg<D, MP, NS, PREC>;
   const DecodeArgs& args;
   uint32_t tmem;
   int warp, lane, s, tile0, T;
@@ -148,6 +240,7 @@ struct DecodeGroup {
   float* xm;  // [2 half][128] of this slot
   float* xl;
   volatile int* s_abort;
+  float zscale;  // 2^e, the factor the fp16 Z was scaled down by (1 without split precision)
 
   template <int CH>
   __device__ __forceinline__ void run() {
@@ -202,7 +295,7 @@ struct DecodeGroup {
         float x[32];
         ptx::tmem_ld32(tS + kLat0 + 32 * k, x);
         ptx::tmem_wait_ld();
-        l += decode_exp_chunk<MP>(x, mref, kLat0 + 32 * k, M, tS + (CH == 0 ? 16 * k : C::kColP1 + 16 * k));
+        l += decode_exp_chunk<MP, PREC != 0>(x, mref, kLat0 + 32 * k, M, tS + (CH == 0 ? 16 * k : C::kColP1 + 16 * k));
       }
       xl[CH * 128 + r] = l;
       __syncwarp();
@@ -218,7 +311,7 @@ struct DecodeGroup {
         break;
       }
       asm volatile("bar.sync %0, 256;" ::"r"(3 + s) : "memory");  // both halves' sums are in xl
-      const float inv = 1.f / (xl[r] + xl[128 + r]);
+      const float inv = zscale / (xl[r] + xl[128 + r]);
       ptx::tc_fence_after();
       constexpr int kHD = D / 2;
       const uint32_t tO = tS + C::kColO + CH * kHD;
@@ -240,15 +333,23 @@ struct DecodeGroup {
 
       const long long tok = static_cast<long long>(tile0 + t) * kTileN + r;
       if (tok < args.N) {
-        uint4* dst = reinterpret_cast<uint4*>(args.Y + (static_cast<size_t>(blockIdx.y) * args.N + tok) * D + CH * kHD);
+        const size_t row = (static_cast<size_t>(blockIdx.y) * args.N + tok) * D + CH * kHD;
+        if constexpr (PREC) {
+          float4* dst = reinterpret_cast<float4*>(static_cast<float*>(args.Y) + row);
 #pragma unroll
-        for (int z = 0; z < kHD / 8; ++z) {
-          uint4 v;
-          v.x = ptx::pack_bf16(o[8 * z + 0] * inv, o[8 * z + 1] * inv);
-          v.y = ptx::pack_bf16(o[8 * z + 2] * inv, o[8 * z + 3] * inv);
-          v.z = ptx::pack_bf16(o[8 * z + 4] * inv, o[8 * z + 5] * inv);
-          v.w = ptx::pack_bf16(o[8 * z + 6] * inv, o[8 * z + 7] * inv);
-          dst[z] = v;
+          for (int z = 0; z < kHD / 4; ++z)
+            dst[z] = make_float4(o[4 * z] * inv, o[4 * z + 1] * inv, o[4 * z + 2] * inv, o[4 * z + 3] * inv);
+        } else {
+          uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(args.Y) + row);
+#pragma unroll
+          for (int z = 0; z < kHD / 8; ++z) {
+            uint4 v;
+            v.x = ptx::pack_bf16(o[8 * z + 0] * inv, o[8 * z + 1] * inv);
+            v.y = ptx::pack_bf16(o[8 * z + 2] * inv, o[8 * z + 3] * inv);
+            v.z = ptx::pack_bf16(o[8 * z + 4] * inv, o[8 * z + 5] * inv);
+            v.w = ptx::pack_bf16(o[8 * z + 6] * inv, o[8 * z + 7] * inv);
+            dst[z] = v;
+          }
         }
       }
     }
@@ -259,11 +360,12 @@ struct DecodeGroup {
   }
 };
 
-template <int D, int MP, int NS>
-__global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
+template <int D, int MP, int NS, int PREC>
+__global__ void __launch_bounds__(DecodeCfg<D, MP, NS, PREC>::kThreads, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmQ,
-                     const __grid_constant__ CUtensorMap tmZ, const DecodeArgs args) {
-  using C = DecodeCfg<D, MP, NS>;
+                     const __grid_constant__ CUtensorMap tmZ, const __grid_constant__ CUtensorMap tmQlo,
+                     const __grid_constant__ CUtensorMap tmZlo, const DecodeArgs args) {
+  using C = DecodeCfg<D, MP, NS, PREC>;
   using G = typename C::G;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -295,7 +397,7 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], 1);
     }
-    ptx::mbar_init(qz_full, 1);
+    ptx::mbar_init(qz_full, C::kQzArrivals);
     for (int s = 0; s < 2; ++s) {
       ptx::mbar_init(&S_full[s], 1);
       ptx::mbar_init(&P_full[s], 8);  // one arrival per warp of the slot's two groups
@@ -322,14 +424,17 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
     if (lane == 0) {
       ptx::prefetch_tmap(&tmK);
       ptx::prefetch_tmap(&tmQ);
-      ptx::prefetch_tmap(&tmZ);
+      // split precision: Q_hi and Q_lo by TMA, the fp16 Z pair from the softmax warps
+      const CUtensorMap* second = PREC ? &tmQlo : &tmZ;
+      ptx::prefetch_tmap(second);
       const int qidx = args.q_batched ? bh : bh % args.H;
       ptx::mbar_arrive_expect_tx(qz_full, 2 * C::kLatBytes);
       for (int h = 0; h < MP / kLatRows; ++h)
         for (int b = 0; b < G::kBlocks; ++b) {
           const int off = b * MP * 128 + h * kLatRows * G::kRowBytes;
           ptx::tma_load_3d(smem + C::kOffQ + off, &tmQ, qz_full, b * 64, h * kLatRows, qidx);
-          ptx::tma_load_3d(smem + C::kOffZ + off, &tmZ, qz_full, b * 64, h * kLatRows, bh);
+          ptx::tma_load_3d(smem + (PREC ? C::kOffQlo : C::kOffZ) + off, second, qz_full, b * 64, h * kLatRows,
+                           PREC ? qidx : bh);
         }
       const uint64_t pol = ptx::policy_evict_first();
       int issued = 0;
@@ -358,6 +463,8 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
     const uint64_t dK0 = G::kmajor(sbase + C::kOffStages, kTileN, 0);
     const uint64_t dQ0 = G::kmajor(sbase + C::kOffQ, MP, 0);
     const uint64_t dZ0 = G::mnmajor(sbase + C::kOffZ, MP, 0);
+    // the low parts (split precision) sit 2 kLatBytes further: one descriptor offset
+    constexpr uint32_t kLoStep = static_cast<uint32_t>(2 * C::kLatBytes) >> 4;
     const uint32_t tS = tmem + slot * C::kSlotCols;
     auto wait_stage = [&](int t) -> bool {
       return ptx::mbar_wait(&full[t % NS], (t / NS) & 1, s_abort, args.wait_ns);
@@ -370,8 +477,11 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
       const uint32_t tD = tS + (h > 0 ? h * kLatRows : 0);
       const uint32_t idesc = h < 0 ? C::kIdescQK : C::kIdescQKHalf;
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k)
-        ptx::mma_ss(tD, dK + G::kmajor_step(kTileN, k), dQ + G::kmajor_step(MP, k), idesc, k > 0 ? 1u : 0u);
+      for (int part = 0; part < C::kLatParts; ++part)
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k)
+          ptx::mma_ss(tD, dK + G::kmajor_step(kTileN, k), dQ + part * kLoStep + G::kmajor_step(MP, k), idesc,
+                      (k > 0 || part > 0) ? 1u : 0u);
     };
     auto commit_s = [&](int t) {
       ptx::mma_commit(&S_full[slot]);
@@ -405,8 +515,11 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
-        for (int k = 0; k < MP / 16; ++k)
-          ptx::mma_ts(tS + C::kColO, tS + C::col_pk(k), dZ0 + G::mnmajor_step(k), C::kIdescPV, k > 0 ? 1u : 0u);
+        for (int part = 0; part < C::kLatParts; ++part)
+#pragma unroll
+          for (int k = 0; k < MP / 16; ++k)
+            ptx::mma_ts(tS + C::kColO, tS + C::col_pk(k), dZ0 + part * kLoStep + G::mnmajor_step(k), C::kIdescPV,
+                        (k > 0 || part > 0) ? 1u : 0u);
         ptx::mma_commit(&O_full[slot]);
         if (next) {
           if constexpr (MP == 256) {
@@ -440,8 +553,14 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS>::kThreads, 1)
   } else {
     // ------------------------------------------------------------ softmax / epilogue groups
     const int s = warp >> 3;  // slot
-    DecodeGroup<D, MP, NS> grp{args, tmem, warp, lane, s, tile0, T, S_full, P_full, O_full, O_free, turn,
-                               s_xm + (s * 2) * 128, s_xl + (s * 2) * 128, s_abort};
+    float zscale = 1.f;
+    if constexpr (PREC != 0) {
+      zscale = stage_z_f16<D, MP, NS, PREC>(args, smem, threadIdx.x);
+      __syncwarp();
+      if (lane == 0) ptx::mbar_arrive(qz_full);
+    }
+    DecodeGroup<D, MP, NS, PREC> grp{args, tmem, warp, lane, s, tile0, T, S_full, P_full, O_full, O_free, turn,
+                               s_xm + (s * 2) * 128, s_xl + (s * 2) * 128, s_abort, zscale};
     if ((warp >> 2) & 1) grp.template run<1>(); else grp.template run<0>();
   }
 

@@ -62,6 +62,19 @@
 // Epilogue: each CTA writes one partial per head (O_part[split] etc.), the
 // accumulators that cover the same latent rows folded with their weights
 // 2^(mref_a - max_a mref_a).
+//
+// Split precision (PREC > 0, D <= 64).  bf16 operands carry 8 significant
+// bits; for outputs whose largest values sit tens of times above their RMS
+// that rounding alone exceeds a 2e-2 x RMS budget.  Each rounded operand x is
+// then carried as the pair hi = bf16(x), lo = bf16(x - hi), which holds x to
+// about 2^-17, and a product takes one MMA per pair member:
+//   PREC >= 1: P = P_hi + P_lo, and O += P_hi V + P_lo V (V is an exact
+//              bf16 input); P_hi over the first 16 of the group's 32 score
+//              columns, P_lo over the other 16;
+//   PREC == 2: the queries too (the routing encode's Q_dyn, given as a hi
+//              and a lo array): S = Q_hi K^T + Q_lo K^T.
+// Every exponential of a split-precision tile is taken on MUFU (the FMA-pipe
+// polynomial's 7.5e-5 relative error would be the largest term left).
 #pragma once
 
 #include "common.cuh"
@@ -72,6 +85,7 @@ constexpr int kEncTile = 64;  // tokens per encode tile
 
 struct EncodeArgs {
   const void* Q;  // bf16 [BH or H][M][D]: read into TMEM directly when D <= 64
+  const void* Q_lo;  // split precision (PREC == 2): the low parts of Q, same layout
   int N;          // tokens per head
   int M;          // latents
   int q_batched;  // Q indexed by bh (1) or by h = bh % H (0)
@@ -98,9 +112,12 @@ __host__ __device__ constexpr int encode_partials_per_split(int /*D*/, int /*nha
 // power-capped) than the MUFU time they free.
 constexpr uint32_t kEncPolyPairs = 0x0001u;
 
-template <int D, int NHALF, int NS>
+template <int D, int NHALF, int NS, int PREC = 0>
 struct EncodeCfg {
   using G = TileGeom<D>;
+  static_assert(PREC == 0 || D <= 64, "split precision needs the split accumulators (D <= 64)");
+  static constexpr bool kPSplit = PREC >= 1;  // P as hi + lo
+  static constexpr int kQParts = PREC == 2 ? 2 : 1;  // Q as hi (+ lo)
   // D <= 64: each column-half group accumulates its own O with its own
   // reference (no exchange of row maxima); D = 128: the two groups of a slot
   // share one O and agree on the reference through shared memory.
@@ -112,12 +129,12 @@ struct EncodeCfg {
   static constexpr uint32_t kColO = 4 * kEncTile;
   static constexpr uint32_t kColQ = kColO + 2 * kAccPerSlot * D;
   // Q in TMEM (TS Q.K^T) when it fits beside S and O, else in shared memory (SS)
-  static constexpr bool kQTmem = kColQ + D <= 512;
+  static constexpr bool kQTmem = kColQ + kQParts * D <= 512;
   static constexpr int kQHalfBytes = kQTmem ? 0 : G::bytes(kLatRows);
   static constexpr int kTileBytes = G::bytes(kEncTile);
   static constexpr int kStageBytes = 2 * kTileBytes;
-  static constexpr int kOffQ = 0;
-  static constexpr int kOffStages = NHALF * kQHalfBytes;
+  static constexpr int kOffQ = 0;  // [part][half] blocks of kQHalfBytes
+  static constexpr int kOffStages = kQParts * NHALF * kQHalfBytes;
   static constexpr int kOffBars = kOffStages + NS * kStageBytes;
   // full[NS], empty[NS], q_ready, S_full[4], P_full[4], pv_done[2], O_final[2], drain
   static constexpr int kNumBars = 2 * NS + 14;
@@ -138,14 +155,29 @@ struct EncodeCfg {
   __host__ __device__ static constexpr uint32_t col_o(int s, int c) {
     return kColO + (kSplitO ? 2 * s + c : s) * D;
   }
-  __host__ __device__ static constexpr uint32_t col_q(int s) { return kColQ + (NHALF == 2 ? s : 0) * (D / 2); }
+  // Q of slot s in TMEM: part 0 (hi) then part 1 (lo), each NHALF x D / 2 columns
+  __host__ __device__ static constexpr uint32_t col_q(int s, int part = 0) {
+    return kColQ + part * NHALF * (D / 2) + (NHALF == 2 ? s : 0) * (D / 2);
+  }
 };
+
+// The low part of a bf16 pair: bf16(e - hi) for each half, hi = the pair
+// pack_bf16 rounded e to (e - hi is exact in fp32).
+__device__ __forceinline__ uint32_t bf16_pair_residual(uint64_t e, uint32_t hi) {
+  const uint64_t h = ptx::f2(__uint_as_float(hi << 16), __uint_as_float(hi & 0xffff0000u));
+  const uint64_t r = ptx::fma2(h, ptx::f2(-1.f, -1.f), e);
+  float r0, r1;
+  ptx::f2_split(r, r0, r1);
+  return ptx::pack_bf16(r0, r1);
+}
 
 // P = 2^(x log2e - nref) for the 32 scores of one half-row, packed to bf16
 // pairs and stored into 16 TMEM columns at tP; returns the fp32 sum.
 // RAGGED (a tile past the end of the tokens, masked columns at -inf): every
 // exponential on MUFU, and masked columns give exactly 0.
-template <bool RAGGED>
+// PSPLIT: P on MUFU only, its low parts (P - bf16(P)) into the 16 columns
+// after tP.
+template <bool RAGGED, bool PSPLIT = false>
 __device__ __forceinline__ float encode_exp_store(const float* x, float nref, uint32_t tP) {
   // pairs of columns as packed fp32 (f32x2): x log2e - nref, the polynomial
   // exponentials and the running sums take one instruction per pair
@@ -154,13 +186,13 @@ __device__ __forceinline__ float encode_exp_store(const float* x, float nref, ui
   uint64_t ps[2] = {0ull, 0ull};  // two independent packed partial sums (+0.0f pairs)
 #pragma unroll
   for (int c0 = 0; c0 < 32; c0 += 16) {
-    uint32_t p[8];
+    uint32_t p[8], pl[8];
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int c = c0 + 2 * u;
       const uint64_t a = ptx::fma2(ptx::f2(x[c], x[c + 1]), kL2, nn);
       uint64_t e;
-      if (!RAGGED && ((kEncPolyPairs >> ((c / 2) & 15)) & 1u)) {
+      if (!RAGGED && !PSPLIT && ((kEncPolyPairs >> ((c / 2) & 15)) & 1u)) {
         e = exp2_poly3_x2(a);
       } else {
         float a0, a1;
@@ -176,8 +208,10 @@ __device__ __forceinline__ float encode_exp_store(const float* x, float nref, ui
       float e0, e1;
       ptx::f2_split(e, e0, e1);
       p[u] = ptx::pack_bf16(e0, e1);
+      if constexpr (PSPLIT) pl[u] = bf16_pair_residual(e, p[u]);
     }
     ptx::tmem_st8(tP + c0 / 2, p);
+    if constexpr (PSPLIT) ptx::tmem_st8(tP + 16 + c0 / 2, pl);
   }
   float s0, s1, s2, s3;
   ptx::f2_split(ps[0], s0, s1);
@@ -190,8 +224,9 @@ __device__ __forceinline__ float encode_exp_store(const float* x, float nref, ui
 // may sit below the half-row's max: the polynomial's input is clamped at 64
 // (a result of at most 2^64), so that a score far above the reference shows
 // up in the sum (MUFU gives +inf there) instead of wrapping the exponent
-// field.
-__device__ __forceinline__ float encode_exp_pack(const float* x, float nref, uint32_t* p) {
+// field.  PSPLIT: on MUFU only, with the low parts in pl[16].
+template <bool PSPLIT = false>
+__device__ __forceinline__ float encode_exp_pack(const float* x, float nref, uint32_t* p, uint32_t* pl) {
   const uint64_t kL2 = ptx::f2(kLog2e, kLog2e);
   const uint64_t nn = ptx::f2(-nref, -nref);
   uint64_t ps[2] = {0ull, 0ull};
@@ -202,7 +237,7 @@ __device__ __forceinline__ float encode_exp_pack(const float* x, float nref, uin
     uint64_t e;
     float a0, a1;
     ptx::f2_split(a, a0, a1);
-    if ((kEncPolyPairs >> (u & 15)) & 1u) {
+    if (!PSPLIT && ((kEncPolyPairs >> (u & 15)) & 1u)) {
       e = exp2_poly3_x2(ptx::f2(fminf(a0, 64.f), fminf(a1, 64.f)));
     } else {
       e = ptx::f2(ptx::ex2(a0), ptx::ex2(a1));
@@ -211,6 +246,7 @@ __device__ __forceinline__ float encode_exp_pack(const float* x, float nref, uin
     float e0, e1;
     ptx::f2_split(e, e0, e1);
     p[u] = ptx::pack_bf16(e0, e1);
+    if constexpr (PSPLIT) pl[u] = bf16_pair_residual(e, p[u]);
   }
   float s0, s1, s2, s3;
   ptx::f2_split(ps[0], s0, s1);
@@ -218,11 +254,12 @@ __device__ __forceinline__ float encode_exp_pack(const float* x, float nref, uin
   return (s0 + s1) + (s2 + s3);
 }
 
-template <int D, int NHALF, int NS>
-__global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
+template <int D, int NHALF, int NS, int PREC>
+__global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS, PREC>::kThreads, 1)
     encode_tc_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
-                     const __grid_constant__ CUtensorMap tmV, const EncodeArgs args) {
-  using C = EncodeCfg<D, NHALF, NS>;
+                     const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmQlo,
+                     const EncodeArgs args) {
+  using C = EncodeCfg<D, NHALF, NS, PREC>;
   using G = typename C::G;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -288,11 +325,13 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
       ptx::prefetch_tmap(&tmV);
       if constexpr (!C::kQTmem) {
         ptx::prefetch_tmap(&tmQ);
-        ptx::mbar_arrive_expect_tx(q_ready, NHALF * C::kQHalfBytes);
-        for (int h = 0; h < NHALF; ++h)
-          for (int b = 0; b < G::kBlocks; ++b)
-            ptx::tma_load_3d(smem + C::kOffQ + h * C::kQHalfBytes + b * kLatRows * 128, &tmQ, q_ready, b * 64,
-                             h * kLatRows, qidx);
+        if constexpr (C::kQParts == 2) ptx::prefetch_tmap(&tmQlo);
+        ptx::mbar_arrive_expect_tx(q_ready, C::kQParts * NHALF * C::kQHalfBytes);
+        for (int part = 0; part < C::kQParts; ++part)
+          for (int h = 0; h < NHALF; ++h)
+            for (int b = 0; b < G::kBlocks; ++b)
+              ptx::tma_load_3d(smem + C::kOffQ + (part * NHALF + h) * C::kQHalfBytes + b * kLatRows * 128,
+                               part ? &tmQlo : &tmQ, q_ready, b * 64, h * kLatRows, qidx);
       }
       const uint64_t pol = ptx::policy_evict_first();
       int issued = 0;
@@ -328,6 +367,10 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
     const uint64_t dV0 = G::mnmajor(sbase + C::kOffStages + C::kTileBytes, kEncTile, 0);
     const uint64_t dQ = G::kmajor(sbase + C::kOffQ + (NHALF == 2 ? s : 0) * C::kQHalfBytes, kLatRows, 0);
     const uint32_t tQ = tmem + C::col_q(s);
+    // the low parts of Q (split precision): NHALF half blocks further in smem,
+    // or their own TMEM columns
+    constexpr uint32_t kQloSmemStep = static_cast<uint32_t>(NHALF * C::kQHalfBytes) >> 4;
+    const uint32_t tQlo = tmem + C::col_q(s, C::kQParts - 1);
     auto wait_stage = [&](int t) -> bool {
       return ptx::mbar_wait(&full[t % NS], (t / NS) & 1, s_abort, args.wait_ns);
     };
@@ -336,12 +379,16 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
       const uint32_t tS = tmem + C::col_s(s, i & 1);
       const uint64_t dK = dK0 + static_cast<uint32_t>((t % NS) * (C::kStageBytes >> 4));
 #pragma unroll
-      for (int k = 0; k < D / 16; ++k) {
-        if constexpr (C::kQTmem)
-          ptx::mma_ts(tS, tQ + k * 8, dK + G::kmajor_step(kEncTile, k), C::kIdescQK, k > 0 ? 1u : 0u);
-        else
-          ptx::mma_ss(tS, dQ + G::kmajor_step(kLatRows, k), dK + G::kmajor_step(kEncTile, k), C::kIdescQK,
-                      k > 0 ? 1u : 0u);
+      for (int part = 0; part < C::kQParts; ++part) {
+#pragma unroll
+        for (int k = 0; k < D / 16; ++k) {
+          const uint32_t acc = (k > 0 || part > 0) ? 1u : 0u;
+          if constexpr (C::kQTmem)
+            ptx::mma_ts(tS, (part ? tQlo : tQ) + k * 8, dK + G::kmajor_step(kEncTile, k), C::kIdescQK, acc);
+          else
+            ptx::mma_ss(tS, dQ + part * kQloSmemStep + G::kmajor_step(kLatRows, k), dK + G::kmajor_step(kEncTile, k),
+                        C::kIdescQK, acc);
+        }
       }
       ptx::mma_commit(&S_full[2 * s + (i & 1)]);
     };
@@ -369,12 +416,16 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
         const uint32_t tP = tmem + C::col_s(s, i & 1);
         const uint64_t dV = dV0 + static_cast<uint32_t>((t % NS) * (C::kStageBytes >> 4));
         // K steps 0-1 carry the tokens of column half 0, steps 2-3 those of half 1
+        // (split precision: each step once with P_hi, once with P_lo 16 columns on)
 #pragma unroll
         for (int kk = 0; kk < kEncTile / 16; ++kk) {
           const int cu = kk / 2;
-          const bool acc = i > 0 || (C::kSplitO ? (kk & 1) : kk) > 0;
-          ptx::mma_ts(tmem + C::col_o(s, cu), tP + cu * 32 + (kk & 1) * 8, dV + G::mnmajor_step(kk), C::kIdescPV,
-                      acc ? 1u : 0u);
+#pragma unroll
+          for (int part = 0; part < (C::kPSplit ? 2 : 1); ++part) {
+            const bool acc = i > 0 || (C::kSplitO ? (kk & 1) : kk) > 0 || part > 0;
+            ptx::mma_ts(tmem + C::col_o(s, cu), tP + cu * 32 + part * 16 + (kk & 1) * 8, dV + G::mnmajor_step(kk),
+                        C::kIdescPV, acc ? 1u : 0u);
+          }
         }
         ptx::mma_commit(&empty[t % NS]);
         ptx::mma_commit(&pv_done[s]);
@@ -426,6 +477,24 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
         }
         const uint32_t ta = tmem + lane_off + C::col_q(s) + col0;
         if constexpr (kPart == 16) ptx::tmem_st16(ta, qv); else ptx::tmem_st8(ta, qv);
+        if constexpr (C::kQParts == 2) {
+          // the low parts of the same row into their own columns
+          if (m < args.M) {
+            const uint4* src = reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(args.Q_lo) +
+                                                              (static_cast<size_t>(qidx) * args.M + m) * D) +
+                               col0 / 4;
+#pragma unroll
+            for (int z = 0; z < kPart / 4; ++z) {
+              const uint4 v = src[z];
+              qv[4 * z] = v.x;
+              qv[4 * z + 1] = v.y;
+              qv[4 * z + 2] = v.z;
+              qv[4 * z + 3] = v.w;
+            }
+          }
+          const uint32_t tl = tmem + lane_off + C::col_q(s, 1) + col0;
+          if constexpr (kPart == 16) ptx::tmem_st16(tl, qv); else ptx::tmem_st8(tl, qv);
+        }
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
@@ -463,10 +532,11 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
       // groups must take the same path.
       bool done = false;
       if (C::kSplitO && i > 0 && valid >= 32) {
-        uint32_t p[16];
-        const float lt = encode_exp_pack(x, mref, p);
+        uint32_t p[16], pl[16];
+        const float lt = encode_exp_pack<C::kPSplit>(x, mref, p, pl);
         if (__all_sync(0xffffffffu, lt <= 4294967296.f)) {
           ptx::tmem_st16(tS + 32 * c, p);
+          if constexpr (C::kPSplit) ptx::tmem_st16(tS + 32 * c + 16, pl);
           l += lt;
           done = true;
         }
@@ -496,8 +566,8 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS>::kThreads, 1)
         const float alpha = nref == mref ? 1.f : ptx::ex2(mref - nref);
         mref = nref;
         // P overwrites the first 16 of this group's own 32 score columns
-        const float lt = valid < 32 ? encode_exp_store<true>(x, nref, tS + 32 * c)
-                                    : encode_exp_store<false>(x, nref, tS + 32 * c);
+        const float lt = valid < 32 ? encode_exp_store<true, C::kPSplit>(x, nref, tS + 32 * c)
+                                    : encode_exp_store<false, C::kPSplit>(x, nref, tS + 32 * c);
         l = fmaf(l, alpha, lt);
         // Rare: the reference moved, so rescale this group's part of O, once the
         // previous P.V (issued after P(i - 1)) has completed; the next one waits

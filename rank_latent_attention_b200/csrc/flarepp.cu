@@ -203,47 +203,73 @@ bool make_map(CUtensorMap* map, const void* ptr, int D, int64_t rows, int64_t pl
 }
 
 // ------------------------------------------------------------------ launchers
-template <int D, int NHALF, int NS>
-cudaError_t launch_encode_tc_t(const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                               const EncodeArgs& a, int BH, cudaStream_t st) {
-  using C = EncodeCfg<D, NHALF, NS>;
-  auto kern = encode_tc_kernel<D, NHALF, NS>;
+// Tensor maps of one encode: Q (hi), K, V, and the low parts of Q (split
+// precision; a copy of Q's map otherwise, never read).
+struct EncodeMaps {
+  CUtensorMap q, k, v, qlo;
+};
+
+template <int D, int NHALF, int NS, int PREC>
+cudaError_t launch_encode_tc_t(const EncodeMaps& m, const EncodeArgs& a, int BH, cudaStream_t st) {
+  using C = EncodeCfg<D, NHALF, NS, PREC>;
+  auto kern = encode_tc_kernel<D, NHALF, NS, PREC>;
   static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(q, k, v, a);
+  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(m.q, m.k, m.v, m.qlo, a);
   return cudaGetLastError();
 }
 
-template <int NHALF>
-cudaError_t launch_encode_tc_n(int D, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
-                               const EncodeArgs& a, int BH, cudaStream_t st) {
+template <int NHALF, int PREC>
+cudaError_t launch_encode_tc_n(int D, const EncodeMaps& m, const EncodeArgs& a, int BH, cudaStream_t st) {
   switch (D) {
-    case 16: return launch_encode_tc_t<16, NHALF, 16>(q, k, v, a, BH, st);
-    case 32: return launch_encode_tc_t<32, NHALF, 8>(q, k, v, a, BH, st);
-    case 64: return launch_encode_tc_t<64, NHALF, 8>(q, k, v, a, BH, st);
-    default: return launch_encode_tc_t<128, NHALF, NHALF == 2 ? 4 : 5>(q, k, v, a, BH, st);
+    case 16: return launch_encode_tc_t<16, NHALF, 16, PREC>(m, a, BH, st);
+    case 32: return launch_encode_tc_t<32, NHALF, 8, PREC>(m, a, BH, st);
+    case 64: return launch_encode_tc_t<64, NHALF, 8, PREC>(m, a, BH, st);
+    default:
+      if constexpr (PREC == 0) return launch_encode_tc_t<128, NHALF, NHALF == 2 ? 4 : 5, 0>(m, a, BH, st);
+      return cudaErrorInvalidValue;  // split precision: D <= 64 only (checked by the caller)
   }
 }
 
-template <int D, int MP, int NS>
-cudaError_t launch_decode_tc_t(const CUtensorMap& k, const CUtensorMap& q, const CUtensorMap& z,
-                               const DecodeArgs& a, int BH, cudaStream_t st) {
-  using C = DecodeCfg<D, MP, NS>;
-  auto kern = decode_tc_kernel<D, MP, NS>;
+cudaError_t launch_encode_tc(int D, int M, int prec, const EncodeMaps& m, const EncodeArgs& a, int BH,
+                             cudaStream_t st) {
+  if (M > kLatRows) {
+    if (prec == 2) return launch_encode_tc_n<2, 2>(D, m, a, BH, st);
+    if (prec == 1) return launch_encode_tc_n<2, 1>(D, m, a, BH, st);
+    return launch_encode_tc_n<2, 0>(D, m, a, BH, st);
+  }
+  if (prec == 2) return launch_encode_tc_n<1, 2>(D, m, a, BH, st);
+  if (prec == 1) return launch_encode_tc_n<1, 1>(D, m, a, BH, st);
+  return launch_encode_tc_n<1, 0>(D, m, a, BH, st);
+}
+
+// Tensor maps of one decode: K, Q (hi), Z, and the low parts of Q (split
+// precision, which reads Z as fp32 instead of through a map; unused maps are
+// copies of Q's, never read).
+struct DecodeMaps {
+  CUtensorMap k, q, z, qlo, zlo;
+};
+
+template <int D, int MP, int NS, int PREC>
+cudaError_t launch_decode_tc_t(const DecodeMaps& m, const DecodeArgs& a, int BH, cudaStream_t st) {
+  using C = DecodeCfg<D, MP, NS, PREC>;
+  auto kern = decode_tc_kernel<D, MP, NS, PREC>;
   static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(k, q, z, a);
+  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(m.k, m.q, m.z, m.qlo, m.zlo, a);
   return cudaGetLastError();
 }
 
-template <int MP>
-cudaError_t launch_decode_tc_m(int D, const CUtensorMap& k, const CUtensorMap& q, const CUtensorMap& z,
-                               const DecodeArgs& a, int BH, cudaStream_t st) {
+template <int MP, int PREC>
+cudaError_t launch_decode_tc_m(int D, const DecodeMaps& m, const DecodeArgs& a, int BH, cudaStream_t st) {
   switch (D) {
-    case 16: return launch_decode_tc_t<16, MP, 8>(k, q, z, a, BH, st);
-    case 32: return launch_decode_tc_t<32, MP, 8>(k, q, z, a, BH, st);
-    case 64: return launch_decode_tc_t<64, MP, 8>(k, q, z, a, BH, st);
-    default: return launch_decode_tc_t<128, MP, 2>(k, q, z, a, BH, st);
+    case 16: return launch_decode_tc_t<16, MP, 8, PREC>(m, a, BH, st);
+    case 32: return launch_decode_tc_t<32, MP, 8, PREC>(m, a, BH, st);
+    // split precision holds four resident latent blocks: a shallower K ring
+    case 64: return launch_decode_tc_t<64, MP, (PREC && MP == 256) ? 5 : 8, PREC>(m, a, BH, st);
+    default:
+      if constexpr (PREC == 0) return launch_decode_tc_t<128, MP, 2, 0>(m, a, BH, st);
+      return cudaErrorInvalidValue;  // split precision: D <= 64 only (checked by the caller)
   }
 }
 
@@ -284,23 +310,31 @@ cudaError_t launch_decode_f32_d(int D, const DecodeF32Args& a, int BH, cudaStrea
 // `out`; lse_out (optional) receives the natural-log log-sum-exp per latent.
 template <typename T>
 cudaError_t launch_merge(const EncodeWs& w, void* out, float* lse_out, int BH, int P, int M, int D,
-                         cudaStream_t st) {
+                         cudaStream_t st, SplitOut split = SplitOut{nullptr, nullptr}) {
   const MergeGeom g{P, M, D, static_cast<long long>(P) * M * D, static_cast<long long>(M) * D,
                     static_cast<long long>(P) * M, M};
   lse_merge_kernel<T, false><<<dim3(static_cast<unsigned>(ceil_div(int64_t(M) * D, 256)), BH), 256, 0, st>>>(
-      w.O, w.m, w.l, static_cast<T*>(out), lse_out, g);
+      w.O, w.m, w.l, static_cast<T*>(out), lse_out, g, split);
   return cudaGetLastError();
 }
+
+// The split-precision tensor-core form of FLARE_BF16_F32OUT covers M % 16 == 0
+// and D <= 64; other sizes of that mode run on the CUDA-core kernels.
+bool f32out_on_tensor_cores(int M, int D) { return M % 16 == 0 && D <= 64; }
 
 // ------------------------------------------------------------------ steps
 // One encode (partials + merge) into `out`; Q indexed per q_batched.
 // dtype FLARE_BF16: everything bf16, tensor cores.  FLARE_F32: everything
-// fp32.  FLARE_BF16_F32OUT: K, V bf16, out fp32, Q bf16 if q_bf16 else fp32.
+// fp32.  FLARE_BF16_F32OUT: K, V bf16, out fp32, Q bf16 if q_bf16 else fp32
+// (CUDA cores), or with prec > 0 the split-precision tensor-core encode:
+// prec 1 takes bf16 Q, prec 2 takes Q as bf16 parts Q (hi) and Q_lo; `split`
+// (optional) also receives the fp32 result as a hi/lo bf16 pair.
 // lse_out: when set, `out` is fp32 whatever the dtype and the merge also
 // writes the natural-log log-sum-exp of each latent's logits ([B][H][M]).
 int run_encode(const void* Q, int q_batched, const void* K, const void* V, void* out, int B, int H, int64_t N,
                int M, int D, int dtype, char* ws, cudaStream_t st, int* launches, bool q_bf16 = false,
-               float* lse_out = nullptr, bool f32_out = false) {
+               float* lse_out = nullptr, bool f32_out = false, int prec = 0, const void* Q_lo = nullptr,
+               SplitOut split = SplitOut{nullptr, nullptr}) {
   const int BH = B * H;
   const int splits = choose_splits(BH, N, kEncTile);
   const int P = partials(M, D, splits, dtype);
@@ -308,13 +342,19 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
   int* status = status_ptr();
   if (!status) return FLARE_ERR_CUDA;
   cudaError_t e;
-  if (dtype == FLARE_BF16) {
-    CUtensorMap tq, tk, tv;
-    if (!make_map(&tq, Q, D, M, q_batched ? BH : H, kLatRows) || !make_map(&tk, K, D, N, BH, kEncTile) ||
-        !make_map(&tv, V, D, N, BH, kEncTile))
+  if (dtype == FLARE_BF16 || prec > 0) {
+    EncodeMaps maps;
+    if (!make_map(&maps.q, Q, D, M, q_batched ? BH : H, kLatRows) || !make_map(&maps.k, K, D, N, BH, kEncTile) ||
+        !make_map(&maps.v, V, D, N, BH, kEncTile))
       return FLARE_ERR_CUDA;
+    if (prec == 2) {
+      if (!make_map(&maps.qlo, Q_lo, D, M, q_batched ? BH : H, kLatRows)) return FLARE_ERR_CUDA;
+    } else {
+      maps.qlo = maps.q;
+    }
     EncodeArgs a;
     a.Q = Q;
+    a.Q_lo = prec == 2 ? Q_lo : Q;
     a.N = static_cast<int>(N);
     a.M = M;
     a.q_batched = q_batched;
@@ -329,13 +369,12 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
     {
       ProfScope prof(FLARE_KERNEL_ENCODE_TC, st);
-      e = M > kLatRows ? launch_encode_tc_n<2>(D, tq, tk, tv, a, BH, st)
-                       : launch_encode_tc_n<1>(D, tq, tk, tv, a, BH, st);
+      e = launch_encode_tc(D, M, prec, maps, a, BH, st);
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
     ProfScope prof(FLARE_KERNEL_MERGE, st);
-    e = f32_out ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st)
-                : launch_merge<__nv_bfloat16>(w, out, lse_out, BH, P, M, D, st);
+    e = (f32_out || prec > 0) ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st, split)
+                              : launch_merge<__nv_bfloat16>(w, out, lse_out, BH, P, M, D, st);
   } else {
     EncodeF32Args a;
     a.N = static_cast<int>(N);
@@ -368,17 +407,32 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
 }
 
+// One decode into Y.  With `lo` (FLARE_BF16_F32OUT on the tensor cores), Q
+// is the hi part of the bf16 pair whose low part is lo->Q_lo, Z is read as
+// fp32 from lo->Zf (the `Z` argument is unused), and Y is fp32.
+struct DecodeLo {
+  const void* Q_lo;
+  const float* Zf;
+};
+
 int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N, int M,
-               int D, int dtype, cudaStream_t st, int* launches) {
+               int D, int dtype, cudaStream_t st, int* launches, const DecodeLo* lo = nullptr) {
   const int BH = B * H;
   cudaError_t e;
-  if (dtype == FLARE_BF16) {
+  if (dtype == FLARE_BF16 || lo) {
     int* status = status_ptr();
     if (!status) return FLARE_ERR_CUDA;
-    CUtensorMap tk, tq, tz;
-    if (!make_map(&tk, K, D, N, BH, kTileN) || !make_map(&tq, Q, D, M, q_batched ? BH : H, kLatRows) ||
-        !make_map(&tz, Z, D, M, BH, kLatRows))
+    DecodeMaps maps;
+    if (!make_map(&maps.k, K, D, N, BH, kTileN) || !make_map(&maps.q, Q, D, M, q_batched ? BH : H, kLatRows))
       return FLARE_ERR_CUDA;
+    if (lo) {
+      if (!make_map(&maps.qlo, lo->Q_lo, D, M, q_batched ? BH : H, kLatRows)) return FLARE_ERR_CUDA;
+      maps.z = maps.q;
+    } else {
+      if (!make_map(&maps.z, Z, D, M, BH, kLatRows)) return FLARE_ERR_CUDA;
+      maps.qlo = maps.q;
+    }
+    maps.zlo = maps.q;
     DecodeArgs a;
     a.N = static_cast<int>(N);
     a.M = M;
@@ -386,12 +440,15 @@ int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void*
     a.H = H;
     a.splits = choose_splits(BH, N, kTileN);
     a.tiles = static_cast<int>(ceil_div(N, kTileN));
-    a.Y = static_cast<__nv_bfloat16*>(Y);
+    a.Y = Y;
+    a.Zf = lo ? lo->Zf : nullptr;
     a.status = status;
     a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
     ProfScope prof(FLARE_KERNEL_DECODE_TC, st);
-    e = M > kLatRows ? launch_decode_tc_m<256>(D, tk, tq, tz, a, BH, st)
-                     : launch_decode_tc_m<128>(D, tk, tq, tz, a, BH, st);
+    if (lo)
+      e = M > kLatRows ? launch_decode_tc_m<256, 1>(D, maps, a, BH, st) : launch_decode_tc_m<128, 1>(D, maps, a, BH, st);
+    else
+      e = M > kLatRows ? launch_decode_tc_m<256, 0>(D, maps, a, BH, st) : launch_decode_tc_m<128, 0>(D, maps, a, BH, st);
   } else {
     DecodeF32Args a;
     a.N = static_cast<int>(N);
@@ -409,11 +466,19 @@ int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void*
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
 }
 
+// Workspace of the mixer: the encode's partials, Q_dyn and Z (dtype storage),
+// and for FLARE_BF16_F32OUT on the tensor cores the hi and lo bf16 parts of
+// Q_dyn.
+size_t mix_split_part_bytes(int BH, int M, int D, int dtype) {
+  if (dtype != FLARE_BF16_F32OUT || !f32out_on_tensor_cores(M, D)) return 0;
+  return align256(static_cast<size_t>(BH) * M * D * 2);
+}
+
 size_t mix_ws_bytes(int B, int H, int64_t N, int M, int D, int dtype) {
   const int BH = B * H;
   const size_t enc = encode_ws_layout(nullptr, BH, N, M, D, dtype).bytes;
   const size_t lat = align256(static_cast<size_t>(BH) * M * D * elem_size(dtype));
-  return enc + 2 * lat;
+  return enc + 2 * lat + 2 * mix_split_part_bytes(BH, M, D, dtype);
 }
 
 // Scratch resolution: caller's buffer, or a stream-ordered allocation.
@@ -458,9 +523,25 @@ int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_
   void* Qd = Qd_out ? Qd_out : s.ptr + enc;
   void* Z = Z_out ? Z_out : s.ptr + enc + lat;
   int launches = 0;
-  rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, /*q_bf16=*/true, lse1_out);
-  if (!rc) rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out);
-  if (!rc) rc = run_decode(K, Qd, 1, Z, Y, B, H, N, M, D, dtype, st, &launches);
+  if (const size_t pb = mix_split_part_bytes(BH, M, D, dtype)) {
+    // FLARE_BF16_F32OUT on the tensor cores: the seed encode's merge also
+    // writes Q_dyn as hi/lo bf16 parts, the query operands of the routing
+    // encode and the key operands of the decode; the decode reads the fp32 Z
+    // and makes its own fp16 parts
+    char* parts = s.ptr + enc + 2 * lat;
+    auto* Qhi = reinterpret_cast<__nv_bfloat16*>(parts);
+    auto* Qlo = reinterpret_cast<__nv_bfloat16*>(parts + pb);
+    rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, true, lse1_out, false, 1,
+                    nullptr, SplitOut{Qhi, Qlo});
+    if (!rc)
+      rc = run_encode(Qhi, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out, false, 2, Qlo);
+    const DecodeLo lo{Qlo, static_cast<const float*>(Z)};
+    if (!rc) rc = run_decode(K, Qhi, 1, nullptr, Y, B, H, N, M, D, dtype, st, &launches, &lo);
+  } else {
+    rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, /*q_bf16=*/true, lse1_out);
+    if (!rc) rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out);
+    if (!rc) rc = run_decode(K, Qd, 1, Z, Y, B, H, N, M, D, dtype, st, &launches);
+  }
   const int rc2 = release_scratch(s, st);
   if (!rc) {
     rc = rc2;

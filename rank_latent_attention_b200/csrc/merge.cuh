@@ -50,11 +50,19 @@ struct MergeGeom {
 // lse_out (may be null) receives the natural-log log-sum-exp of the union,
 // ln(2^m* sum_p w_p l_p); a row with no tokens at all gets out = 0 and
 // lse_out = -inf.
+// split (may be null; fp32 out only): {hi, lo} receive the result as a bf16
+// pair, hi = bf16(out), lo = bf16(out - hi), the operand form of the next
+// step's split-precision MMAs.
+struct SplitOut {
+  __nv_bfloat16* hi;
+  __nv_bfloat16* lo;
+};
 template <typename OutT, bool FROM_LSE>
 __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict__ O_part,
                                                         const float* __restrict__ m_part,
                                                         const float* __restrict__ l_part, OutT* __restrict__ out,
-                                                        float* __restrict__ lse_out, MergeGeom g) {
+                                                        float* __restrict__ lse_out, MergeGeom g,
+                                                        SplitOut split = SplitOut{nullptr, nullptr}) {
   constexpr float kLn2 = 0.6931471805599453f;
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= g.M * g.D) return;
@@ -85,7 +93,13 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
     }
   }
   const size_t orow = static_cast<size_t>(bh) * g.M + m;
-  out[orow * g.D + d] = to_out<OutT>(den > 0.f ? num / den : 0.f);
+  const float v = den > 0.f ? num / den : 0.f;
+  out[orow * g.D + d] = to_out<OutT>(v);
+  if (split.hi) {
+    const __nv_bfloat16 h = __float2bfloat16_rn(v);
+    split.hi[orow * g.D + d] = h;
+    split.lo[orow * g.D + d] = __float2bfloat16_rn(v - __bfloat162float(h));
+  }
   if (lse_out && d == 0) lse_out[orow] = den > 0.f ? (mx + log2f(den)) * kLn2 : -INFINITY;
 }
 
