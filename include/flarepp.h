@@ -313,10 +313,19 @@ int flare_last_launch_count(void);
  *     slots, at most ~32k tokens per CTA).
  *   flare_set_wait_limit_ms(ms): how long a tensor-core kernel waits on one
  *     barrier before recording FLARE_ERR_TIMEOUT and returning (default 2000).
- * Both return the previous value.
+ *   flare_set_launch_overlap(mode): whether the mixer's merges, routing
+ *     encode and decode are launched with programmatic stream serialisation,
+ *     so that each may start its set-up (barriers, tensor memory, the first
+ *     K/V loads) while the kernel before it finishes; every such kernel
+ *     waits for its predecessor before it reads that kernel's output, and the
+ *     seed encode never overlaps whatever precedes the call.  1 always, 0
+ *     never, -1 (the default) when each encode CTA has at most 64 token
+ *     tiles, where the fixed cost of a launch is a large share of the call.
+ * All return the previous value.
  */
 int flare_set_split_override(int splits);
 int flare_set_wait_limit_ms(int ms);
+int flare_set_launch_overlap(int mode);
 
 /*
  * Communication matrix of the latent routing, per head (b, h):

@@ -43,6 +43,7 @@ __all__ = [
     "flare_check_status",
     "flare_last_launch_count",
     "flare_set_split_override",
+    "flare_set_launch_overlap",
     "flare_set_wait_limit_ms",
     "flare_profile_begin",
     "flare_profile_end",
@@ -86,6 +87,7 @@ _SIGNATURES = {
     "flare_communication_workspace_size": (_c_size, _SIZES),
     "flare_communication_matrix": (_c_int, [_vp, _c_int, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_set_split_override": (_c_int, [_c_int]),
+    "flare_set_launch_overlap": (_c_int, [_c_int]),
     "flare_selftest_wait_timeout": (_c_int, [_c_int, _vp]),
     "flare_set_wait_limit_ms": (_c_int, [_c_int]),
     "flare_profile_begin": (_c_int, [_c_int]),
@@ -454,6 +456,11 @@ def flare_last_launch_count() -> int:
 
 def flare_set_split_override(splits: int) -> int:
     return lib().flare_set_split_override(splits)
+
+
+def flare_set_launch_overlap(mode: int) -> int:
+    """1: the mixer's later kernels overlap their predecessors' tails; 0: never; -1: by size (default)."""
+    return lib().flare_set_launch_overlap(mode)
 
 
 def flare_set_wait_limit_ms(ms: int) -> int:

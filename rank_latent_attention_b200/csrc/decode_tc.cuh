@@ -418,11 +418,28 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS, PREC>::kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = ptx::smem_u32(smem);
+  // Launched with programmatic serialisation (the decode of a mixer call),
+  // this kernel may start while the kernel before it finishes: every thread
+  // but the producer's waits for it here; the producer first prefetches K
+  // stages (an input of the call) and waits before it loads Q and Z.
+  if (warp != C::kProducerWarp || lane != 0) ptx::grid_dep_wait();
 
   if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       ptx::prefetch_tmap(&tmK);
+      const uint64_t pol = ptx::policy_evict_first();
+      int issued = 0;
+      auto load_stage = [&](int t) {
+        const int st = t % NS;
+        uint8_t* sk = smem + C::kOffStages + st * C::kTileBytes;
+        ptx::mbar_arrive_expect_tx(&full[st], C::kTileBytes);
+        for (int b = 0; b < G::kBlocks; ++b)
+          ptx::tma_load_3d_hint(sk + b * kTileN * 128, &tmK, &full[st], b * 64, (tile0 + t) * kTileN, bh, pol);
+        issued = t + 1;
+      };
+      for (int t = 0; t < NS && t < T; ++t) load_stage(t);
+      ptx::grid_dep_wait();
       ptx::prefetch_tmap(&tmQ);
       // split precision: Q_hi and Q_lo by TMA, the fp16 Z pair from the softmax warps
       const CUtensorMap* second = PREC ? &tmQlo : &tmZ;
@@ -436,21 +453,16 @@ __global__ void __launch_bounds__(DecodeCfg<D, MP, NS, PREC>::kThreads, 1)
           ptx::tma_load_3d(smem + (PREC ? C::kOffQlo : C::kOffZ) + off, second, qz_full, b * 64, h * kLatRows,
                            PREC ? qidx : bh);
         }
-      const uint64_t pol = ptx::policy_evict_first();
-      int issued = 0;
-      for (int t = 0; t < T; ++t) {
-        const int st = t % NS;
-        if (t >= NS && !ptx::mbar_wait(&empty[st], ((t / NS) - 1) & 1, s_abort, args.wait_ns)) {
+      for (int t = issued; t < T; ++t) {
+        if (t >= NS && !ptx::mbar_wait(&empty[t % NS], ((t / NS) - 1) & 1, s_abort, args.wait_ns)) {
           record_error(args.status, kErrTimeout, kSiteDecProducer);
           *s_abort = 1;
           break;
         }
-        uint8_t* sk = smem + C::kOffStages + st * C::kTileBytes;
-        ptx::mbar_arrive_expect_tx(&full[st], C::kTileBytes);
-        for (int b = 0; b < G::kBlocks; ++b)
-          ptx::tma_load_3d_hint(sk + b * kTileN * 128, &tmK, &full[st], b * 64, (tile0 + t) * kTileN, bh, pol);
-        issued = t + 1;
+        load_stage(t);
       }
+      // this CTA's loads are all issued: the next kernel of the stream may start
+      ptx::grid_dep_launch();
       ptx::mbar_wait_drain(qz_full, 0);
       for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)
         ptx::mbar_wait_drain(&full[t % NS], (t / NS) & 1);

@@ -317,12 +317,34 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS, PREC>::kThreads, 1)
   ptx::tc_fence_after();
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = ptx::smem_u32(smem);
+  // Launched with programmatic serialisation (the routing encode of a mixer
+  // call), this kernel may start while the kernel before it finishes: every
+  // thread but the producer's waits for it here; the producer first
+  // prefetches K/V stages (inputs of the call, which no earlier kernel of it
+  // writes) and waits before it loads Q.
+  if (warp != C::kProducerWarp || lane != 0) ptx::grid_dep_wait();
 
   if (warp == C::kProducerWarp) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       ptx::prefetch_tmap(&tmK);
       ptx::prefetch_tmap(&tmV);
+      const uint64_t pol = ptx::policy_evict_first();
+      int issued = 0;
+      auto load_stage = [&](int t) {
+        const int st = t % NS;
+        uint8_t* sk = smem + C::kOffStages + st * C::kStageBytes;
+        uint8_t* sv = sk + C::kTileBytes;
+        const int tok = (tile0 + t) * kEncTile;
+        ptx::mbar_arrive_expect_tx(&full[st], C::kStageBytes);
+        for (int b = 0; b < G::kBlocks; ++b)
+          ptx::tma_load_3d_hint(sk + b * kEncTile * 128, &tmK, &full[st], b * 64, tok, bh, pol);
+        for (int b = 0; b < G::kBlocks; ++b)
+          ptx::tma_load_3d_hint(sv + b * kEncTile * 128, &tmV, &full[st], b * 64, tok, bh, pol);
+        issued = t + 1;
+      };
+      for (int t = 0; t < NS && t < T; ++t) load_stage(t);
+      ptx::grid_dep_wait();
       if constexpr (!C::kQTmem) {
         ptx::prefetch_tmap(&tmQ);
         if constexpr (C::kQParts == 2) ptx::prefetch_tmap(&tmQlo);
@@ -333,25 +355,16 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS, PREC>::kThreads, 1)
               ptx::tma_load_3d(smem + C::kOffQ + (part * NHALF + h) * C::kQHalfBytes + b * kLatRows * 128,
                                part ? &tmQlo : &tmQ, q_ready, b * 64, h * kLatRows, qidx);
       }
-      const uint64_t pol = ptx::policy_evict_first();
-      int issued = 0;
-      for (int t = 0; t < T; ++t) {
-        const int st = t % NS;
-        if (t >= NS && !ptx::mbar_wait(&empty[st], ((t / NS) - 1) & 1, s_abort, args.wait_ns)) {
+      for (int t = issued; t < T; ++t) {
+        if (t >= NS && !ptx::mbar_wait(&empty[t % NS], ((t / NS) - 1) & 1, s_abort, args.wait_ns)) {
           record_error(args.status, kErrTimeout, kSiteEncProducer);
           *s_abort = 1;
           break;
         }
-        uint8_t* sk = smem + C::kOffStages + st * C::kStageBytes;
-        uint8_t* sv = sk + C::kTileBytes;
-        const int tok = (tile0 + t) * kEncTile;
-        ptx::mbar_arrive_expect_tx(&full[st], C::kStageBytes);
-        for (int b = 0; b < G::kBlocks; ++b)
-          ptx::tma_load_3d_hint(sk + b * kEncTile * 128, &tmK, &full[st], b * 64, tok, bh, pol);
-        for (int b = 0; b < G::kBlocks; ++b)
-          ptx::tma_load_3d_hint(sv + b * kEncTile * 128, &tmV, &full[st], b * 64, tok, bh, pol);
-        issued = t + 1;
+        load_stage(t);
       }
+      // this CTA's loads are all issued: the next kernel of the stream may start
+      ptx::grid_dep_launch();
       // Every load issued must land before the CTA may exit (matters on the abort path only).
       if constexpr (!C::kQTmem) ptx::mbar_wait_drain(q_ready, 0);
       for (int t = (issued > NS ? issued - NS : 0); t < issued; ++t)

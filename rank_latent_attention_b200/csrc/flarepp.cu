@@ -10,6 +10,7 @@
 #include <algorithm>
 #include <atomic>
 #include <mutex>
+#include <utility>
 #include <vector>
 
 #include <type_traits>
@@ -28,6 +29,9 @@ namespace {
 __device__ int g_status[2];  // {first error code, site} per device
 
 std::atomic<int> g_split_override{0};
+// Programmatic dependent launch of a mixer call's later kernels: -1 by size
+// (overlap_launches), 0 never, 1 always (flare_set_launch_overlap)
+std::atomic<int> g_launch_overlap{-1};
 std::atomic<int> g_wait_ms{2000};
 thread_local int t_last_launches = 0;
 // The split override as this thread's current entry-point call first read
@@ -203,6 +207,42 @@ bool make_map(CUtensorMap* map, const void* ptr, int D, int64_t rows, int64_t pl
 }
 
 // ------------------------------------------------------------------ launchers
+// Launch with programmatic stream serialisation when pdl is set: the kernel
+// may start while the previous kernel of the stream finishes.  Only kernels
+// that wait (grid_dep_wait) before reading anything an earlier kernel of the
+// call writes are launched that way: the merges, and the routing encode and
+// the decode of a mixer call, whose K and V are the call's inputs.
+template <typename... Exp, typename... Act>
+cudaError_t launch_k(bool pdl, void (*kern)(Exp...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                     Act&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = pdl ? 1 : 0;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Act>(args)...);
+}
+
+// Encode tiles per CTA up to which a mixer call overlaps launches by default.
+constexpr int64_t kOverlapMaxTilesPerCta = 64;
+
+// Whether a mixer call overlaps its kernels' prologues with the kernels
+// before them.  By default only when each encode CTA has few tiles: there the
+// fixed cost of a kernel (launch, barrier and TMEM set-up, the first loads)
+// is a large share of the call; on long token runs the overlap was measured
+// slower (the early CTAs' Q load waits behind their K/V prefetch).
+bool overlap_launches(int BH, int64_t N) {
+  const int mode = g_launch_overlap.load();
+  if (mode >= 0) return mode > 0;
+  const int64_t tiles = ceil_div(N, kEncTile);
+  return ceil_div(tiles, choose_splits(BH, N, kEncTile)) <= kOverlapMaxTilesPerCta;
+}
+
 // Tensor maps of one encode: Q (hi), K, V, and the low parts of Q (split
 // precision; a copy of Q's map otherwise, never read).
 struct EncodeMaps {
@@ -210,37 +250,36 @@ struct EncodeMaps {
 };
 
 template <int D, int NHALF, int NS, int PREC>
-cudaError_t launch_encode_tc_t(const EncodeMaps& m, const EncodeArgs& a, int BH, cudaStream_t st) {
+cudaError_t launch_encode_tc_t(const EncodeMaps& m, const EncodeArgs& a, int BH, cudaStream_t st, bool pdl) {
   using C = EncodeCfg<D, NHALF, NS, PREC>;
   auto kern = encode_tc_kernel<D, NHALF, NS, PREC>;
   static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(m.q, m.k, m.v, m.qlo, a);
-  return cudaGetLastError();
+  return launch_k(pdl, kern, dim3(a.splits, BH), dim3(C::kThreads), C::kSmemBytes, st, m.q, m.k, m.v, m.qlo, a);
 }
 
 template <int NHALF, int PREC>
-cudaError_t launch_encode_tc_n(int D, const EncodeMaps& m, const EncodeArgs& a, int BH, cudaStream_t st) {
+cudaError_t launch_encode_tc_n(int D, const EncodeMaps& m, const EncodeArgs& a, int BH, cudaStream_t st, bool pdl) {
   switch (D) {
-    case 16: return launch_encode_tc_t<16, NHALF, 16, PREC>(m, a, BH, st);
-    case 32: return launch_encode_tc_t<32, NHALF, 8, PREC>(m, a, BH, st);
-    case 64: return launch_encode_tc_t<64, NHALF, 8, PREC>(m, a, BH, st);
+    case 16: return launch_encode_tc_t<16, NHALF, 16, PREC>(m, a, BH, st, pdl);
+    case 32: return launch_encode_tc_t<32, NHALF, 8, PREC>(m, a, BH, st, pdl);
+    case 64: return launch_encode_tc_t<64, NHALF, 8, PREC>(m, a, BH, st, pdl);
     default:
-      if constexpr (PREC == 0) return launch_encode_tc_t<128, NHALF, NHALF == 2 ? 4 : 5, 0>(m, a, BH, st);
+      if constexpr (PREC == 0) return launch_encode_tc_t<128, NHALF, NHALF == 2 ? 4 : 5, 0>(m, a, BH, st, pdl);
       return cudaErrorInvalidValue;  // split precision: D <= 64 only (checked by the caller)
   }
 }
 
 cudaError_t launch_encode_tc(int D, int M, int prec, const EncodeMaps& m, const EncodeArgs& a, int BH,
-                             cudaStream_t st) {
+                             cudaStream_t st, bool pdl) {
   if (M > kLatRows) {
-    if (prec == 2) return launch_encode_tc_n<2, 2>(D, m, a, BH, st);
-    if (prec == 1) return launch_encode_tc_n<2, 1>(D, m, a, BH, st);
-    return launch_encode_tc_n<2, 0>(D, m, a, BH, st);
+    if (prec == 2) return launch_encode_tc_n<2, 2>(D, m, a, BH, st, pdl);
+    if (prec == 1) return launch_encode_tc_n<2, 1>(D, m, a, BH, st, pdl);
+    return launch_encode_tc_n<2, 0>(D, m, a, BH, st, pdl);
   }
-  if (prec == 2) return launch_encode_tc_n<1, 2>(D, m, a, BH, st);
-  if (prec == 1) return launch_encode_tc_n<1, 1>(D, m, a, BH, st);
-  return launch_encode_tc_n<1, 0>(D, m, a, BH, st);
+  if (prec == 2) return launch_encode_tc_n<1, 2>(D, m, a, BH, st, pdl);
+  if (prec == 1) return launch_encode_tc_n<1, 1>(D, m, a, BH, st, pdl);
+  return launch_encode_tc_n<1, 0>(D, m, a, BH, st, pdl);
 }
 
 // Tensor maps of one decode: K, Q (hi), Z, and the low parts of Q (split
@@ -251,24 +290,24 @@ struct DecodeMaps {
 };
 
 template <int D, int MP, int NS, int PREC>
-cudaError_t launch_decode_tc_t(const DecodeMaps& m, const DecodeArgs& a, int BH, cudaStream_t st) {
+cudaError_t launch_decode_tc_t(const DecodeMaps& m, const DecodeArgs& a, int BH, cudaStream_t st, bool pdl) {
   using C = DecodeCfg<D, MP, NS, PREC>;
   auto kern = decode_tc_kernel<D, MP, NS, PREC>;
   static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
   if (attr != cudaSuccess) return attr;
-  kern<<<dim3(a.splits, BH), C::kThreads, C::kSmemBytes, st>>>(m.k, m.q, m.z, m.qlo, m.zlo, a);
-  return cudaGetLastError();
+  return launch_k(pdl, kern, dim3(a.splits, BH), dim3(C::kThreads), C::kSmemBytes, st, m.k, m.q, m.z, m.qlo, m.zlo,
+                  a);
 }
 
 template <int MP, int PREC>
-cudaError_t launch_decode_tc_m(int D, const DecodeMaps& m, const DecodeArgs& a, int BH, cudaStream_t st) {
+cudaError_t launch_decode_tc_m(int D, const DecodeMaps& m, const DecodeArgs& a, int BH, cudaStream_t st, bool pdl) {
   switch (D) {
-    case 16: return launch_decode_tc_t<16, MP, 8, PREC>(m, a, BH, st);
-    case 32: return launch_decode_tc_t<32, MP, 8, PREC>(m, a, BH, st);
+    case 16: return launch_decode_tc_t<16, MP, 8, PREC>(m, a, BH, st, pdl);
+    case 32: return launch_decode_tc_t<32, MP, 8, PREC>(m, a, BH, st, pdl);
     // split precision holds four resident latent blocks: a shallower K ring
-    case 64: return launch_decode_tc_t<64, MP, (PREC && MP == 256) ? 5 : 8, PREC>(m, a, BH, st);
+    case 64: return launch_decode_tc_t<64, MP, (PREC && MP == 256) ? 5 : 8, PREC>(m, a, BH, st, pdl);
     default:
-      if constexpr (PREC == 0) return launch_decode_tc_t<128, MP, 2, 0>(m, a, BH, st);
+      if constexpr (PREC == 0) return launch_decode_tc_t<128, MP, 2, 0>(m, a, BH, st, pdl);
       return cudaErrorInvalidValue;  // split precision: D <= 64 only (checked by the caller)
   }
 }
@@ -310,12 +349,12 @@ cudaError_t launch_decode_f32_d(int D, const DecodeF32Args& a, int BH, cudaStrea
 // `out`; lse_out (optional) receives the natural-log log-sum-exp per latent.
 template <typename T>
 cudaError_t launch_merge(const EncodeWs& w, void* out, float* lse_out, int BH, int P, int M, int D,
-                         cudaStream_t st, SplitOut split = SplitOut{nullptr, nullptr}) {
+                         cudaStream_t st, bool pdl, SplitOut split = SplitOut{nullptr, nullptr}) {
   const MergeGeom g{P, M, D, static_cast<long long>(P) * M * D, static_cast<long long>(M) * D,
                     static_cast<long long>(P) * M, M};
-  lse_merge_kernel<T, false><<<dim3(static_cast<unsigned>(ceil_div(int64_t(M) * D, 256)), BH), 256, 0, st>>>(
-      w.O, w.m, w.l, static_cast<T*>(out), lse_out, g, split);
-  return cudaGetLastError();
+  return launch_k(pdl, lse_merge_kernel<T, false>, dim3(static_cast<unsigned>(ceil_div(int64_t(M) * D, 256)), BH),
+                  dim3(256), 0, st, static_cast<const float*>(w.O), static_cast<const float*>(w.m),
+                  static_cast<const float*>(w.l), static_cast<T*>(out), lse_out, g, split);
 }
 
 // The split-precision tensor-core form of FLARE_BF16_F32OUT covers M % 16 == 0
@@ -334,7 +373,7 @@ bool f32out_on_tensor_cores(int M, int D) { return M % 16 == 0 && D <= 64; }
 int run_encode(const void* Q, int q_batched, const void* K, const void* V, void* out, int B, int H, int64_t N,
                int M, int D, int dtype, char* ws, cudaStream_t st, int* launches, bool q_bf16 = false,
                float* lse_out = nullptr, bool f32_out = false, int prec = 0, const void* Q_lo = nullptr,
-               SplitOut split = SplitOut{nullptr, nullptr}) {
+               SplitOut split = SplitOut{nullptr, nullptr}, bool pdl = false, bool pdl_merge = false) {
   const int BH = B * H;
   const int splits = choose_splits(BH, N, kEncTile);
   const int P = partials(M, D, splits, dtype);
@@ -369,12 +408,12 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
     {
       ProfScope prof(FLARE_KERNEL_ENCODE_TC, st);
-      e = launch_encode_tc(D, M, prec, maps, a, BH, st);
+      e = launch_encode_tc(D, M, prec, maps, a, BH, st, pdl);
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
     ProfScope prof(FLARE_KERNEL_MERGE, st);
-    e = (f32_out || prec > 0) ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st, split)
-                              : launch_merge<__nv_bfloat16>(w, out, lse_out, BH, P, M, D, st);
+    e = (f32_out || prec > 0) ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st, pdl_merge, split)
+                              : launch_merge<__nv_bfloat16>(w, out, lse_out, BH, P, M, D, st, pdl_merge);
   } else {
     EncodeF32Args a;
     a.N = static_cast<int>(N);
@@ -401,7 +440,7 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
     ProfScope prof(FLARE_KERNEL_MERGE, st);
-    e = launch_merge<float>(w, out, lse_out, BH, P, M, D, st);
+    e = launch_merge<float>(w, out, lse_out, BH, P, M, D, st, false);
   }
   *launches += 2;
   return e == cudaSuccess ? FLARE_OK : FLARE_ERR_CUDA;
@@ -416,7 +455,7 @@ struct DecodeLo {
 };
 
 int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void* Y, int B, int H, int64_t N, int M,
-               int D, int dtype, cudaStream_t st, int* launches, const DecodeLo* lo = nullptr) {
+               int D, int dtype, cudaStream_t st, int* launches, const DecodeLo* lo = nullptr, bool pdl = false) {
   const int BH = B * H;
   cudaError_t e;
   if (dtype == FLARE_BF16 || lo) {
@@ -446,9 +485,11 @@ int run_decode(const void* K, const void* Q, int q_batched, const void* Z, void*
     a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
     ProfScope prof(FLARE_KERNEL_DECODE_TC, st);
     if (lo)
-      e = M > kLatRows ? launch_decode_tc_m<256, 1>(D, maps, a, BH, st) : launch_decode_tc_m<128, 1>(D, maps, a, BH, st);
+      e = M > kLatRows ? launch_decode_tc_m<256, 1>(D, maps, a, BH, st, pdl)
+                       : launch_decode_tc_m<128, 1>(D, maps, a, BH, st, pdl);
     else
-      e = M > kLatRows ? launch_decode_tc_m<256, 0>(D, maps, a, BH, st) : launch_decode_tc_m<128, 0>(D, maps, a, BH, st);
+      e = M > kLatRows ? launch_decode_tc_m<256, 0>(D, maps, a, BH, st, pdl)
+                       : launch_decode_tc_m<128, 0>(D, maps, a, BH, st, pdl);
   } else {
     DecodeF32Args a;
     a.N = static_cast<int>(N);
@@ -523,6 +564,10 @@ int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_
   void* Qd = Qd_out ? Qd_out : s.ptr + enc;
   void* Z = Z_out ? Z_out : s.ptr + enc + lat;
   int launches = 0;
+  // the merges, the routing encode and the decode may start while the kernel
+  // before each finishes (K and V are the call's inputs, not that kernel's
+  // output)
+  const bool pdl = overlap_launches(BH, N);
   if (const size_t pb = mix_split_part_bytes(BH, M, D, dtype)) {
     // FLARE_BF16_F32OUT on the tensor cores: the seed encode's merge also
     // writes Q_dyn as hi/lo bf16 parts, the query operands of the routing
@@ -532,15 +577,20 @@ int mix_impl(const void* seeds, const void* K, const void* V, void* Y, void* Qd_
     auto* Qhi = reinterpret_cast<__nv_bfloat16*>(parts);
     auto* Qlo = reinterpret_cast<__nv_bfloat16*>(parts + pb);
     rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, true, lse1_out, false, 1,
-                    nullptr, SplitOut{Qhi, Qlo});
+                    nullptr, SplitOut{Qhi, Qlo}, false, pdl);
     if (!rc)
-      rc = run_encode(Qhi, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out, false, 2, Qlo);
+      rc = run_encode(Qhi, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out, false, 2, Qlo,
+                      SplitOut{nullptr, nullptr}, pdl, pdl);
     const DecodeLo lo{Qlo, static_cast<const float*>(Z)};
-    if (!rc) rc = run_decode(K, Qhi, 1, nullptr, Y, B, H, N, M, D, dtype, st, &launches, &lo);
+    if (!rc) rc = run_decode(K, Qhi, 1, nullptr, Y, B, H, N, M, D, dtype, st, &launches, &lo, pdl);
   } else {
-    rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, /*q_bf16=*/true, lse1_out);
-    if (!rc) rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out);
-    if (!rc) rc = run_decode(K, Qd, 1, Z, Y, B, H, N, M, D, dtype, st, &launches);
+    // the seed encode waits for whatever came before the call (it may write K/V)
+    rc = run_encode(seeds, 0, K, V, Qd, B, H, N, M, D, dtype, s.ptr, st, &launches, /*q_bf16=*/true, lse1_out,
+                    false, 0, nullptr, SplitOut{nullptr, nullptr}, false, pdl);
+    if (!rc)
+      rc = run_encode(Qd, 1, K, V, Z, B, H, N, M, D, dtype, s.ptr, st, &launches, false, lse2_out, false, 0, nullptr,
+                      SplitOut{nullptr, nullptr}, pdl, pdl);
+    if (!rc) rc = run_decode(K, Qd, 1, Z, Y, B, H, N, M, D, dtype, st, &launches, nullptr, pdl);
   }
   const int rc2 = release_scratch(s, st);
   if (!rc) {
@@ -1445,6 +1495,8 @@ int flare_last_launch_count(void) { return t_last_launches; }
 int flare_set_split_override(int splits) { return g_split_override.exchange(splits < 0 ? 0 : splits); }
 
 int flare_set_wait_limit_ms(int ms) { return g_wait_ms.exchange(ms < 1 ? 1 : ms); }
+
+int flare_set_launch_overlap(int mode) { return g_launch_overlap.exchange(mode < -1 ? -1 : (mode > 1 ? 1 : mode)); }
 
 int flare_profile_begin(int max_launches) {
   std::lock_guard<std::mutex> lock(g_prof.mu);

@@ -64,6 +64,11 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
                                                         float* __restrict__ lse_out, MergeGeom g,
                                                         SplitOut split = SplitOut{nullptr, nullptr}) {
   constexpr float kLn2 = 0.6931471805599453f;
+  // launched with programmatic serialisation after the encode that writes
+  // the partials: let the next kernel start its prologue, wait for the
+  // partials
+  ptx::grid_dep_launch();
+  ptx::grid_dep_wait();
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= g.M * g.D) return;
   const int bh = blockIdx.y;
