@@ -304,6 +304,15 @@ const char* flare_status_string(int status);
 int flare_last_launch_count(void);
 
 /*
+ * Name of the CUDA error the library's own CUDA runtime last recorded on this
+ * host thread ("no error" if none), without clearing it: after a call returned
+ * FLARE_ERR_CUDA this names the failed launch or CUDA call.  The library links
+ * its CUDA runtime statically, so the caller's cudaGetLastError does not see
+ * that state.  Static string.
+ */
+const char* flare_cuda_error_string(void);
+
+/*
  * Tuning / test hooks (process-wide, not thread-safe against concurrent calls):
  *   flare_set_split_override(s): use s CTAs per head along the tokens in
  *     every token-split kernel, each clamped to that kernel's number of token
@@ -340,15 +349,23 @@ int flare_set_launch_overlap(int mode);
  * (q_batched = 1).
  *
  * Q: [H][M][D] (q_batched = 0) or [B][H][M][D]; K: [B][H][N][D]; C:
- * [B][H][M][M], in the storage type of dtype (FLARE_F32: fp32 throughout on
- * CUDA cores; FLARE_BF16: bf16 inputs and C, tensor-core steps).  All
- * pointers are device memory owned by the caller, 16-byte aligned.
- * Computed with the library's own decode and encode: ceil(M / D) rounds of a
- * decode with Z = D columns of the M x M identity (giving those columns of
- * W_dec) and an encode with that block as V.  workspace: at least
- * flare_communication_workspace_size() bytes (it holds one N x D block of
- * W_dec per head), or NULL to allocate on the stream.  Errors as for
- * flare_encode; FLARE_BF16_F32OUT is FLARE_ERR_UNSUPPORTED.
+ * [B][H][M][M].  dtype: FLARE_F32 (fp32 throughout on CUDA cores, C fp32);
+ * FLARE_BF16 (bf16 Q and K, C bf16); FLARE_BF16_F32OUT (bf16 Q and K, C
+ * fp32).  All pointers are device memory owned by the caller, 16-byte
+ * aligned.  The library forms C only: the O(M^3) eigen-solve of the M x M
+ * matrices is left to the caller.
+ * bf16 inputs with M % 16 == 0 and D <= 64 take one pass over the tokens on
+ * the tensor cores: both weights are functions of the same logits,
+ * W_enc[m][n] = exp(s_nm - L2_m) and W_dec[n][m] = exp(s_nm - L3_n), so with
+ * the per-latent log-sum-exp L2 (an encode's merge) C is a plain sum over
+ * tokens of W_enc[:, n] W_dec[n, :], accumulated in fp32 from fp16 weights
+ * (both lie in [0, 1]; 4 launches: encode, merge, the C kernel, the sum of its token-split
+ * partials).  Other sizes (and FLARE_F32) use the library's decode and
+ * encode: ceil(M / D) rounds of a decode with Z = D columns of the M x M
+ * identity (giving those columns of W_dec) and an encode with that block as
+ * V; FLARE_BF16_F32OUT is then FLARE_ERR_UNSUPPORTED.  workspace: at least
+ * flare_communication_workspace_size() bytes, or NULL to allocate on the
+ * stream.  Errors as for flare_encode.
  */
 size_t flare_communication_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
 int flare_communication_matrix(const void* Q, int q_batched, const void* K, void* C, int B, int H, int64_t N, int M,
@@ -364,7 +381,9 @@ typedef enum {
   FLARE_KERNEL_BWD_TOKEN_STATS = 6,  /* backward: per-token lse3, delta       */
   FLARE_KERNEL_BWD_LATENT = 7,       /* backward: latent-side partials        */
   FLARE_KERNEL_BWD_REDUCE = 8,       /* backward: sums of those partials      */
-  FLARE_KERNEL_BWD_TOKEN_GRAD = 9    /* backward: dK, dV                      */
+  FLARE_KERNEL_BWD_TOKEN_GRAD = 9,   /* backward: dK, dV                      */
+  FLARE_KERNEL_COMM_TC = 10,         /* communication matrix, one pass        */
+  FLARE_KERNEL_COMM_REDUCE = 11      /* sum of its token-split partials       */
 } flare_kernel_kind_t;
 
 /*

@@ -42,6 +42,7 @@ __all__ = [
     "flare_communication_matrix",
     "flare_check_status",
     "flare_last_launch_count",
+    "flare_cuda_error_string",
     "flare_set_split_override",
     "flare_set_launch_overlap",
     "flare_set_wait_limit_ms",
@@ -56,6 +57,7 @@ LIB_PATH = os.path.join(_HERE, "libflarepp.so")
 HEADER_PATH = os.path.join(os.path.dirname(_HERE), "include", "flarepp.h")
 
 F32, BF16, BF16_F32OUT = 0, 1, 2
+CUDA_ERROR = 3  # FLARE_ERR_CUDA
 _c_int, _c_i64, _c_size, _vp = ctypes.c_int, ctypes.c_int64, ctypes.c_size_t, ctypes.c_void_p
 _SIZES = [_c_int, _c_int, _c_i64, _c_int, _c_int, _c_int]  # B, H, N, M, D, dtype
 
@@ -82,6 +84,7 @@ _SIGNATURES = {
     "flare_check_status": (_c_int, [_vp, ctypes.POINTER(_c_int)]),
     "flare_status_string": (ctypes.c_char_p, [_c_int]),
     "flare_last_launch_count": (_c_int, []),
+    "flare_cuda_error_string": (ctypes.c_char_p, []),
     "flarepp_mix_host_workspace_size": (_c_size, _SIZES),
     "flarepp_mix_host": (_c_int, [_vp, _vp, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_communication_workspace_size": (_c_size, _SIZES),
@@ -95,7 +98,8 @@ _SIGNATURES = {
 }
 
 KERNEL_NAMES = {1: "encode_tc", 2: "lse_merge", 3: "decode_tc", 4: "encode_f32", 5: "decode_f32",
-                6: "bwd_token_stats", 7: "bwd_latent", 8: "bwd_reduce", 9: "bwd_token_grad"}
+                6: "bwd_token_stats", 7: "bwd_latent", 8: "bwd_reduce", 9: "bwd_token_grad", 10: "comm_tc",
+                11: "comm_reduce"}
 
 _lib = None
 
@@ -103,7 +107,10 @@ _lib = None
 class FlareError(RuntimeError):
     def __init__(self, status: int, where: str):
         self.status = status
-        super().__init__(f"{where}: {lib().flare_status_string(status).decode()} (status {status})")
+        msg = f"{where}: {lib().flare_status_string(status).decode()} (status {status})"
+        if status == CUDA_ERROR:
+            msg += f": {lib().flare_cuda_error_string().decode()}"
+        super().__init__(msg)
 
 
 def lib() -> ctypes.CDLL:
@@ -376,23 +383,25 @@ def flarepp_mix_host(seeds, K, V, Y=None, *, out_dtype=None, workspace=None, str
     return Y
 
 
-def flare_communication_matrix(Q, K, C=None, *, workspace=None, stream=None):
+def flare_communication_matrix(Q, K, C=None, *, out_dtype=None, workspace=None, stream=None):
     """C = softmax_N(Q K^T) softmax_M(K Q^T) per head: [B,H,M,M], row-stochastic.
 
     Its eigenvalues are the nonzero eigenvalues of the rank-M token-to-token
     communication matrix W = W_dec W_enc; the library forms C (the O(M^2 N)
     part) and leaves the O(M^3) eigen-solve of the small M x M matrices to the
     caller.  Q is [H,M,D] (shared) or [B,H,M,D] (e.g. FLARE++'s routing
-    queries Q_dyn)."""
+    queries Q_dyn).  out_dtype=torch.float32 with bf16 inputs returns C in
+    fp32 (FLARE_BF16_F32OUT)."""
     torch = _torch()
     B, H, N, D = K.shape
     q_batched = 1 if Q.dim() == 4 else 0
     M = Q.shape[-2]
+    code, odt = _mix_mode(K, out_dtype)
     if C is None:
-        C = torch.empty((B, H, M, M), dtype=K.dtype, device=K.device)
+        C = torch.empty((B, H, M, M), dtype=odt, device=K.device)
     ws, wsb = _ws(workspace)
     _check(lib().flare_communication_matrix(_ptr(Q, "Q", K.dtype), q_batched, _ptr(K, "K", K.dtype),
-                                            _ptr(C, "C", K.dtype), B, H, N, M, D, _dtype_code(K), ws, wsb,
+                                            _ptr(C, "C", odt), B, H, N, M, D, code, ws, wsb,
                                             _stream(stream)), "flare_communication_matrix")
     return C
 

@@ -18,6 +18,7 @@
 #include "../../include/flarepp.h"
 #include "backward_simt.cuh"
 #include "backward_tc.cuh"
+#include "comm_tc.cuh"
 #include "decode_tc.cuh"
 #include "encode_tc.cuh"
 #include "merge.cuh"
@@ -676,6 +677,104 @@ int run_comm(const void* Q, int q_batched, const void* K, void* C, int B, int H,
     ++*launches;
   }
   return FLARE_OK;
+}
+
+// One pass on the tensor cores (comm_tc.cuh), bf16 inputs: an encode of Q
+// over the tokens (K as its values, only its merge's log-sum-exp per latent
+// is kept), the C kernel per (token split, latent half, head), and the sum of
+// its split partials into C (bf16 or fp32).  Workspace, in order: the
+// encode's partials, its [BH][M][D] fp32 output (unused), lse2 [BH][M], the
+// C partials [BH][S][M][M] fp32.
+struct CommTcWs {
+  size_t enc, z, lse, part, bytes;
+  int splits;
+};
+
+int comm_splits(int BH, int64_t N, int M) {
+  // whole waves of the SMs, over the (head, latent half) CTA columns
+  return choose_splits(BH * (M > kLatRows ? 2 : 1), N, kTileN);
+}
+
+CommTcWs comm_tc_ws_layout(int B, int H, int64_t N, int M, int D) {
+  const int BH = B * H;
+  CommTcWs w;
+  w.splits = comm_splits(BH, N, M);
+  w.enc = encode_ws_layout(nullptr, BH, N, M, D, FLARE_BF16).bytes;
+  w.z = align256(static_cast<size_t>(BH) * M * D * sizeof(float));
+  w.lse = align256(static_cast<size_t>(BH) * M * sizeof(float));
+  w.part = align256(static_cast<size_t>(BH) * w.splits * M * M * sizeof(float));
+  w.bytes = w.enc + w.z + w.lse + w.part;
+  return w;
+}
+
+template <int D, int MP, int NS>
+cudaError_t launch_comm_tc_t(const CUtensorMap& tk, const CUtensorMap& tq, const CommArgs& a, int BH,
+                             cudaStream_t st) {
+  using C = CommCfg<D, MP, NS>;
+  auto kern = comm_tc_kernel<D, MP, NS>;
+  static cudaError_t attr = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::kSmemBytes);
+  if (attr != cudaSuccess) return attr;
+  kern<<<dim3(a.splits, C::kHalves, BH), C::kThreads, C::kSmemBytes, st>>>(tk, tq, a);
+  return cudaGetLastError();
+}
+
+template <int MP>
+cudaError_t launch_comm_tc_m(int D, const CUtensorMap& tk, const CUtensorMap& tq, const CommArgs& a, int BH,
+                             cudaStream_t st) {
+  switch (D) {
+    case 16: return launch_comm_tc_t<16, MP, 4>(tk, tq, a, BH, st);
+    case 32: return launch_comm_tc_t<32, MP, 4>(tk, tq, a, BH, st);
+    default: return launch_comm_tc_t<64, MP, 3>(tk, tq, a, BH, st);
+  }
+}
+
+int run_comm_tc(const void* Q, int q_batched, const void* K, void* C, int B, int H, int64_t N, int M, int D,
+                bool f32_out, char* ws, cudaStream_t st, int* launches) {
+  const int BH = B * H;
+  const CommTcWs w = comm_tc_ws_layout(B, H, N, M, D);
+  float* Ztmp = reinterpret_cast<float*>(ws + w.enc);
+  float* lse2 = reinterpret_cast<float*>(ws + w.enc + w.z);
+  float* part = reinterpret_cast<float*>(ws + w.enc + w.z + w.lse);
+  int rc = run_encode(Q, q_batched, K, K, Ztmp, B, H, N, M, D, FLARE_BF16, ws, st, launches, false, lse2, true);
+  if (rc) return rc;
+  int* status = status_ptr();
+  if (!status) return FLARE_ERR_CUDA;
+  CUtensorMap tk, tq;
+  if (!make_map(&tk, K, D, N, BH, kTileN) || !make_map(&tq, Q, D, M, q_batched ? BH : H, kLatRows))
+    return FLARE_ERR_CUDA;
+  CommArgs a;
+  a.N = static_cast<int>(N);
+  a.M = M;
+  a.H = H;
+  a.q_batched = q_batched;
+  a.splits = w.splits;
+  a.tiles = static_cast<int>(ceil_div(N, kTileN));
+  a.lse2 = lse2;
+  a.C_part = part;
+  a.status = status;
+  a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+  cudaError_t e;
+  {
+    ProfScope prof(FLARE_KERNEL_COMM_TC, st);
+    e = M > kLatRows ? launch_comm_tc_m<256>(D, tk, tq, a, BH, st) : launch_comm_tc_m<128>(D, tk, tq, a, BH, st);
+  }
+  if (e != cudaSuccess) return FLARE_ERR_CUDA;
+  const dim3 grid(static_cast<unsigned>(ceil_div(int64_t(M) * M, 256)), BH);
+  {
+    ProfScope prof(FLARE_KERNEL_COMM_REDUCE, st);
+    if (f32_out)
+      comm_reduce_kernel<float><<<grid, 256, 0, st>>>(part, static_cast<float*>(C), M, w.splits);
+    else
+      comm_reduce_kernel<__nv_bfloat16><<<grid, 256, 0, st>>>(part, static_cast<__nv_bfloat16*>(C), M, w.splits);
+  }
+  if (cudaGetLastError() != cudaSuccess) return FLARE_ERR_CUDA;
+  *launches += 2;
+  return FLARE_OK;
+}
+
+// The one-pass tensor-core form covers bf16 inputs with M % 16 == 0 and D <= 64.
+bool comm_on_tensor_cores(int M, int D, int dtype) {
+  return (dtype == FLARE_BF16 || dtype == FLARE_BF16_F32OUT) && M % 16 == 0 && D <= 64;
 }
 
 // ------------------------------------------------------------------ host-resident inputs
@@ -1355,7 +1454,9 @@ int flarepp_mix_debug(const void* seeds, const void* K, const void* V, void* Y, 
 
 size_t flare_communication_workspace_size(int B, int H, int64_t N, int M, int D, int dtype) {
   SplitPin pin;
-  if (check_sizes(B, H, N, M, D, dtype) || dtype == FLARE_BF16_F32OUT) return 0;
+  if (check_sizes(B, H, N, M, D, dtype)) return 0;
+  if (comm_on_tensor_cores(M, D, dtype)) return comm_tc_ws_layout(B, H, N, M, D).bytes;
+  if (dtype == FLARE_BF16_F32OUT) return 0;
   return comm_ws_layout(B, H, N, M, D, dtype).bytes;
 }
 
@@ -1364,17 +1465,22 @@ int flare_communication_matrix(const void* Q, int q_batched, const void* K, void
   SplitPin pin;
   int rc = check_sizes(B, H, N, M, D, dtype);
   if (rc) return rc;
-  if (dtype == FLARE_BF16_F32OUT) return FLARE_ERR_UNSUPPORTED;
+  const bool tc = comm_on_tensor_cores(M, D, dtype);
+  if (dtype == FLARE_BF16_F32OUT && !tc) return FLARE_ERR_UNSUPPORTED;
   if (q_batched != 0 && q_batched != 1) return FLARE_ERR_INVALID_ARG;
   if (!device_ptr(Q) || !device_ptr(K) || !device_ptr(C)) return FLARE_ERR_INVALID_ARG;
   if (workspace && !device_ptr(workspace)) return FLARE_ERR_INVALID_ARG;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   Scratch s;
-  rc = get_scratch(workspace, workspace_bytes, comm_ws_layout(B, H, N, M, D, dtype).bytes, st, &s);
+  rc = get_scratch(workspace, workspace_bytes,
+                   tc ? comm_tc_ws_layout(B, H, N, M, D).bytes : comm_ws_layout(B, H, N, M, D, dtype).bytes, st, &s);
   if (rc) return rc;
   int launches = 0;
-  rc = dtype == FLARE_BF16 ? run_comm<__nv_bfloat16>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches)
-                           : run_comm<float>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches);
+  if (tc)
+    rc = run_comm_tc(Q, q_batched, K, C, B, H, N, M, D, dtype == FLARE_BF16_F32OUT, s.ptr, st, &launches);
+  else
+    rc = dtype == FLARE_BF16 ? run_comm<__nv_bfloat16>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches)
+                             : run_comm<float>(Q, q_batched, K, C, B, H, N, M, D, dtype, s.ptr, st, &launches);
   const int rc2 = release_scratch(s, st);
   if (!rc) {
     rc = rc2;
@@ -1491,6 +1597,8 @@ const char* flare_status_string(int status) {
 }
 
 int flare_last_launch_count(void) { return t_last_launches; }
+
+const char* flare_cuda_error_string(void) { return cudaGetErrorString(cudaPeekAtLastError()); }
 
 int flare_set_split_override(int splits) { return g_split_override.exchange(splits < 0 ? 0 : splits); }
 
