@@ -76,24 +76,45 @@ __global__ void __launch_bounds__(256) lse_merge_kernel(const float* __restrict_
   const int d = idx - m * g.D;
   const long long sbase = bh * g.s_head + m;
   const long long obase = bh * g.o_head + static_cast<long long>(m) * g.D + d;
-  float mx = -INFINITY;
-  for (int p = 0; p < g.P; ++p) {
-    const long long row = sbase + p * g.s_part;
-    if constexpr (FROM_LSE) {
-      mx = fmaxf(mx, m_part[row] * kLog2e);
-    } else {
-      if (l_part[row] > 0.f) mx = fmaxf(mx, m_part[row]);
+  // One pass with a running maximum: a partial whose reference lies above
+  // the running one rescales the sums so far (exact; usually only the first
+  // few partials do).  The loads of a batch of partials are independent, so
+  // they are issued together instead of one dependent round trip each.
+  float mx = -INFINITY, num = 0.f, den = 0.f;
+  constexpr int kBatch = 8;
+  for (int p0 = 0; p0 < g.P; p0 += kBatch) {
+    float mp[kBatch], lp[kBatch], op[kBatch];
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      const int p = p0 + u;
+      mp[u] = -INFINITY;
+      lp[u] = 0.f;
+      op[u] = 0.f;
+      if (p < g.P) {
+        const long long row = sbase + p * g.s_part;
+        if constexpr (FROM_LSE) {
+          const float lse = m_part[row];
+          mp[u] = lse * kLog2e;
+          lp[u] = lse > -INFINITY ? 1.f : 0.f;
+        } else {
+          mp[u] = m_part[row];
+          lp[u] = l_part[row];
+        }
+        op[u] = O_part[obase + p * g.o_part];
+      }
     }
-  }
-  float num = 0.f, den = 0.f;
-  if (mx > -INFINITY) {
-    for (int p = 0; p < g.P; ++p) {
-      const long long row = sbase + p * g.s_part;
-      const float l = FROM_LSE ? (m_part[row] > -INFINITY ? 1.f : 0.f) : l_part[row];
-      if (l > 0.f) {
-        const float w = exp2f((FROM_LSE ? m_part[row] * kLog2e : m_part[row]) - mx);
-        den = fmaf(w, l, den);
-        num = fmaf(w, O_part[obase + p * g.o_part], num);
+#pragma unroll
+    for (int u = 0; u < kBatch; ++u) {
+      if (lp[u] > 0.f) {  // partials without tokens carry no weight
+        if (mp[u] > mx) {
+          const float scale = mx > -INFINITY ? exp2f(mx - mp[u]) : 0.f;
+          num *= scale;
+          den *= scale;
+          mx = mp[u];
+        }
+        const float w = exp2f(mp[u] - mx);
+        den = fmaf(w, lp[u], den);
+        num = fmaf(w, op[u], num);
       }
     }
   }
