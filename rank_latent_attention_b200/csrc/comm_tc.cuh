@@ -84,8 +84,8 @@ struct CommCfg {
   static constexpr int kOffBars = kOffP + (MP / 64) * kBlockBytes;
   // full[NS], empty[NS], q_full, S_full, S_free, AB_full, P_free, E_free[2], drain
   static constexpr int kNumBars = 2 * NS + 8;
-  static constexpr int kOffL2 = kOffBars + 8 * kNumBars;  // float [MP]: lse2 in log2 units
-  static constexpr int kOffX = kOffL2 + MP * 4;  // float [2 use][kColGroups][128]: partial row max, sum
+  static constexpr int kOffBias = kOffBars + 8 * kNumBars;  // float [MP]: 12 - lse2 log2e (-inf past M)
+  static constexpr int kOffX = kOffBias + MP * 4;  // float [2 use][kColGroups][128]: partial row max, sum
   static constexpr int kOffMisc = kOffX + 2 * kColGroups * 128 * 4;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr uint32_t kTmemCols = 512;
@@ -121,7 +121,7 @@ __global__ void __launch_bounds__(CommCfg<D, MP, NS>::kThreads, 1)
   uint64_t* P_free = q_full + 4;  // the MMA of the last tile has read P
   uint64_t* E_free = q_full + 5;  // [buffer]: the MMA of the last tile that used it has read it
   uint64_t* drain = q_full + 7;
-  float* s_l2 = reinterpret_cast<float*>(smem + C::kOffL2);
+  float* s_bias = reinterpret_cast<float*>(smem + C::kOffBias);
   float* s_x = reinterpret_cast<float*>(smem + C::kOffX);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -151,9 +151,10 @@ __global__ void __launch_bounds__(CommCfg<D, MP, NS>::kThreads, 1)
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
-  // lse2 of the head's latents in log2 units (0 past M: those rows are masked)
+  // the exponent bias of each latent's encode weight, 2^12 / exp(lse2_m) in
+  // log2 units (-inf past M, whose weights are then 0)
   for (int m = threadIdx.x; m < MP; m += C::kThreads)
-    s_l2[m] = m < args.M ? args.lse2[static_cast<size_t>(bh) * args.M + m] * kLog2e : 0.f;
+    s_bias[m] = m < args.M ? C::kEScaleLog2 - args.lse2[static_cast<size_t>(bh) * args.M + m] * kLog2e : -INFINITY;
   if (warp == C::kProducerWarp) {
     ptx::tmem_alloc(s_tmem, C::kTmemCols);
     ptx::tmem_relinquish();
@@ -248,17 +249,21 @@ __global__ void __launch_bounds__(CommCfg<D, MP, NS>::kThreads, 1)
     ptx::mbar_wait_drain(drain, 0);
   } else {
     // ------------------------------------------------------------ token rows
+    // Each warp takes runs of 32 latents, one run in each 128-latent half
+    // (latents [32 cq, +32) and, with MP = 256, [128 + 32 cq, +32)), so every
+    // warp forms the same share of E (its run in half hm) and of P.
     const int q = warp & 3;       // TMEM lane quarter
-    const int cq = warp >> 2;     // column quarter
+    const int cq = warp >> 2;     // which run of each half
     const int r = q * 32 + lane;  // token row of the tile
-    const uint32_t tS = tmem + (static_cast<uint32_t>(q * 32) << 16) + cq * C::kCols;
+    const uint32_t tRow = tmem + (static_cast<uint32_t>(q * 32) << 16);
     const int bar_id = 1 + q;     // the four warps of this lane quarter
     constexpr int kG = C::kColGroups;
+    constexpr int kRuns = C::kCols / 32;  // runs of 32 latents per thread
     float* xm = s_x;              // [cq][128]
     float* xs = s_x + kG * 128;
-    const int c0 = cq * C::kCols;  // first latent of this thread's columns
-    // E columns: this thread's columns all lie in one 128-latent half
-    const bool e_here = c0 / kLatRows == hm;
+    auto run_col = [&](int run) { return run * kLatRows + 32 * cq; };  // first latent of a run
+    const int e_run = hm;  // the run that lies in half hm (MP = 128: hm = 0, one run)
+    const uint64_t kL2 = ptx::f2(kLog2e, kLog2e);
     bool ok = true;
     for (int t = 0; t < T; ++t) {
       if (!__all_sync(0xffffffffu, ptx::mbar_wait(S_full, t & 1, s_abort, args.wait_ns))) {
@@ -268,56 +273,93 @@ __global__ void __launch_bounds__(CommCfg<D, MP, NS>::kThreads, 1)
       ptx::tc_fence_after();
       float x[C::kCols];
 #pragma unroll
-      for (int k = 0; k < C::kCols / 32; ++k) ptx::tmem_ld32(tS + 32 * k, x + 32 * k);
+      for (int run = 0; run < kRuns; ++run) ptx::tmem_ld32(tRow + run_col(run), x + 32 * run);
       ptx::tmem_wait_ld();
       ptx::tc_fence_before();
       __syncwarp();
       if (lane == 0) ptx::mbar_arrive(S_free);
+      // a row past N (a ragged last tile) contributes nothing: its logits
+      // are set to 0 (finite) and its weights zeroed below
       const bool valid = (tile0 + t) * kTileN + r < args.N;
-      // latents past M take no part (M is a multiple of 16)
+      const bool all_valid = __all_sync(0xffffffffu, valid);
+      // latents past M take no part (M is a multiple of 16; only a run that
+      // crosses M needs the mask)
 #pragma unroll
-      for (int j = 0; j < C::kCols; ++j)
-        if (c0 + j >= args.M) x[j] = -INFINITY;
-      float mx = -INFINITY;
+      for (int run = 0; run < kRuns; ++run) {
+        if (run_col(run) + 32 > args.M) {
 #pragma unroll
-      for (int j = 0; j < C::kCols; ++j) mx = fmaxf(mx, x[j]);
-      xm[cq * 128 + r] = mx;
+          for (int j = 0; j < 32; ++j)
+            if (run_col(run) + j >= args.M) x[32 * run + j] = -INFINITY;
+        }
+      }
+      float pm[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+#pragma unroll
+      for (int j = 0; j < C::kCols; j += 8) {
+        pm[0] = ptx::max3(pm[0], x[j], x[j + 1]);
+        pm[1] = ptx::max3(pm[1], x[j + 2], x[j + 3]);
+        pm[2] = ptx::max3(pm[2], x[j + 4], x[j + 5]);
+        pm[3] = ptx::max3(pm[3], x[j + 6], x[j + 7]);
+      }
+      xm[cq * 128 + r] = fmaxf(fmaxf(pm[0], pm[1]), fmaxf(pm[2], pm[3]));
       asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
       const float rowmax = fmaxf(fmaxf(xm[r], xm[128 + r]), fmaxf(xm[256 + r], xm[384 + r])) * kLog2e;
-      // E = 2^(s log2e - lse2_m) from the raw logits, for the latents of half
-      // hm, into E buffer t % 2 once the MMA of tile t - 2 has read it
-      if (e_here) {
-        if (t >= 2 &&
-            !__all_sync(0xffffffffu, ptx::mbar_wait(&E_free[t & 1], ((t - 2) >> 1) & 1, s_abort, args.wait_ns))) {
-          ok = false;
-          break;
-        }
+      // E = 2^(s log2e + 12 - lse2_m) from the raw logits, for this thread's
+      // run in half hm, into E buffer t % 2 once the MMA of tile t - 2 has
+      // read it (s_bias[m] = 12 - lse2_m log2e, -inf past M)
+      if (t >= 2 &&
+          !__all_sync(0xffffffffu, ptx::mbar_wait(&E_free[t & 1], ((t - 2) >> 1) & 1, s_abort, args.wait_ns))) {
+        ok = false;
+        break;
+      }
+      {
         uint8_t* eb = smem + C::kOffE + (t & 1) * C::kEBytes;
+        // the run index is a compile-time constant in each branch, so x
+        // stays in registers
+        auto form_e = [&](auto run_c) {
+          constexpr int run = decltype(run_c)::value;
+          const float2* bias = reinterpret_cast<const float2*>(s_bias + run_col(run));
 #pragma unroll
-        for (int c = 0; c < C::kCols / 8; ++c) {
-          uint32_t e[4];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t e[4];
 #pragma unroll
-          for (int u = 0; u < 4; ++u) {
-            const int j = 8 * c + 2 * u;
-            const float e0 = valid ? ptx::ex2(fmaf(x[j], kLog2e, C::kEScaleLog2 - s_l2[c0 + j])) : 0.f;
-            const float e1 = valid ? ptx::ex2(fmaf(x[j + 1], kLog2e, C::kEScaleLog2 - s_l2[c0 + j + 1])) : 0.f;
-            e[u] = ptx::pack_f16(e0, e1);
+            for (int u = 0; u < 4; ++u) {
+              const int j = 8 * c + 2 * u;
+              const float2 b = bias[j / 2];
+              const uint64_t a = ptx::fma2(ptx::f2(x[32 * run + j], x[32 * run + j + 1]), kL2, ptx::f2(b.x, b.y));
+              float a0, a1;
+              ptx::f2_split(a, a0, a1);
+              float e0 = ptx::ex2(a0), e1 = ptx::ex2(a1);
+              if (!all_valid && !valid) e0 = e1 = 0.f;
+              e[u] = ptx::pack_f16(e0, e1);
+            }
+            const int col = 32 * cq + 8 * c;  // latent within half hm
+            *reinterpret_cast<uint4*>(eb + (col / 64) * C::kBlockBytes + comm_chunk_offset(r, (col % 64) / 8)) =
+                make_uint4(e[0], e[1], e[2], e[3]);
           }
-          const int col = (c0 + 8 * c) - hm * kLatRows;  // latent within half hm
-          *reinterpret_cast<uint4*>(eb + (col / 64) * C::kBlockBytes + comm_chunk_offset(r, (col % 64) / 8)) =
-              make_uint4(e[0], e[1], e[2], e[3]);
-        }
+        };
+        if (kRuns == 1 || e_run == 0)
+          form_e(std::integral_constant<int, 0>{});
+        else
+          form_e(std::integral_constant<int, kRuns - 1>{});
       }
       // decode weights of this row: 2^(s log2e - rowmax), normalised below
-      float sum = 0.f;
+      const uint64_t nr = ptx::f2(-rowmax, -rowmax);
+      uint64_t ps[2] = {0ull, 0ull};
 #pragma unroll
-      for (int j = 0; j < C::kCols; ++j) {
-        x[j] = ptx::ex2(fmaf(x[j], kLog2e, -rowmax));
-        sum += x[j];
+      for (int j = 0; j < C::kCols; j += 2) {
+        float a0, a1;
+        ptx::f2_split(ptx::fma2(ptx::f2(x[j], x[j + 1]), kL2, nr), a0, a1);
+        x[j] = ptx::ex2(a0);
+        x[j + 1] = ptx::ex2(a1);
+        ps[(j >> 1) & 1] = ptx::add2(ps[(j >> 1) & 1], ptx::f2(x[j], x[j + 1]));
       }
-      xs[cq * 128 + r] = sum;
+      float s0, s1, s2, s3;
+      ptx::f2_split(ps[0], s0, s1);
+      ptx::f2_split(ps[1], s2, s3);
+      xs[cq * 128 + r] = (s0 + s1) + (s2 + s3);
       asm volatile("bar.sync %0, 128;" ::"r"(bar_id) : "memory");
       const float inv = valid ? 1.f / ((xs[r] + xs[128 + r]) + (xs[256 + r] + xs[384 + r])) : 0.f;
+      const uint64_t inv2 = ptx::f2(inv, inv);
       // the previous tile's MMA has read the P buffer
       if (t > 0 && !__all_sync(0xffffffffu, ptx::mbar_wait(P_free, (t - 1) & 1, s_abort, args.wait_ns))) {
         ok = false;
@@ -326,14 +368,16 @@ __global__ void __launch_bounds__(CommCfg<D, MP, NS>::kThreads, 1)
       // P: chunks of 8 latents into the column blocks of 64
 #pragma unroll
       for (int c = 0; c < C::kCols / 8; ++c) {
-        const int col = c0 + 8 * c;  // first latent of the chunk
-        uint4 v;
-        v.x = ptx::pack_f16(x[8 * c + 0] * inv, x[8 * c + 1] * inv);
-        v.y = ptx::pack_f16(x[8 * c + 2] * inv, x[8 * c + 3] * inv);
-        v.z = ptx::pack_f16(x[8 * c + 4] * inv, x[8 * c + 5] * inv);
-        v.w = ptx::pack_f16(x[8 * c + 6] * inv, x[8 * c + 7] * inv);
+        const int col = run_col(c / 4) + 8 * (c % 4);  // first latent of the chunk
+        uint32_t v[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float p0, p1;
+          ptx::f2_split(ptx::mul2(ptx::f2(x[8 * c + 2 * u], x[8 * c + 2 * u + 1]), inv2), p0, p1);
+          v[u] = ptx::pack_f16(p0, p1);
+        }
         *reinterpret_cast<uint4*>(smem + C::kOffP + (col / 64) * C::kBlockBytes + comm_chunk_offset(r, (col % 64) / 8)) =
-            v;
+            make_uint4(v[0], v[1], v[2], v[3]);
       }
       ptx::fence_proxy_async_smem();
       __syncwarp();
@@ -349,6 +393,7 @@ __global__ void __launch_bounds__(CommCfg<D, MP, NS>::kThreads, 1)
     if (ok && T > 0 && __all_sync(0xffffffffu, ptx::mbar_wait(P_free, (T - 1) & 1, s_abort, args.wait_ns))) {
       ptx::tc_fence_after();
       const int m = hm * kLatRows + r;
+      const int c0 = cq * C::kCols;  // this warp's contiguous share of C's columns
       float* dst = args.C_part + ((static_cast<size_t>(bh) * args.splits + split) * args.M + m) * args.M;
 #pragma unroll
       for (int k = 0; k < C::kCols / 32; ++k) {
