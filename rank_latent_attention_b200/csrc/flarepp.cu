@@ -8,6 +8,7 @@
 #include <stdio.h>
 
 #include <algorithm>
+#include <limits>
 #include <atomic>
 #include <mutex>
 #include <utility>
@@ -125,16 +126,33 @@ bool device_ptr(const void* p) {
   return attr.type == cudaMemoryTypeDevice || attr.type == cudaMemoryTypeManaged;
 }
 
-// CTAs per head along the token axis: enough CTAs to fill whole waves of the
-// SMs' CTA slots (per_sm resident CTAs per SM), at most ~32768 tokens per CTA;
+// CTAs per head along the token axis.  A kernel's time is about
+//   (waves of the SMs' CTA slots) x (tiles per CTA + a fixed cost per CTA),
+// waves = ceil(BH s / slots) with per_sm resident CTAs per SM; the fixed
+// cost (launch share, barrier and TMEM set-up, the first loads, the
+// epilogue: about 384 tokens' worth of work) makes fewer, longer CTAs win
+// ties.  The count minimising that estimate is taken among s from the
+// smallest that keeps a CTA at most ~32768 tokens, over eight more waves'
+// worth of CTAs per head.  Rounding the split count up to fill the waves
+// instead sent few-head workloads just past a wave boundary (32 heads: 5
+// splits, 160 CTAs = 1.08 waves, twice the time of 4 splits).
 // `tile` is the kernel's token tile (64 for the encode, 128 for the decode).
 int choose_splits(int BH, int64_t N, int tile, int per_sm = 1) {
   const int64_t tiles = ceil_div(N, tile);
   int64_t s = t_split_pin >= 0 ? t_split_pin : g_split_override.load();
   if (s <= 0) {
     const int64_t slots = int64_t(sm_count()) * per_sm;
-    const int64_t waves = std::max<int64_t>(1, ceil_div(BH * tiles, slots * (32768 / tile)));
-    s = ceil_div(waves * slots, BH);
+    const int64_t fixed_tiles = std::max<int64_t>(1, 384 / tile);
+    const int64_t lo = std::max<int64_t>(1, ceil_div(tiles, 32768 / tile));
+    const int64_t hi = std::min<int64_t>(tiles, lo + 8 * ceil_div(slots, BH));
+    int64_t best = std::numeric_limits<int64_t>::max();
+    for (int64_t c = lo; c <= hi; ++c) {
+      const int64_t cost = ceil_div(int64_t(BH) * c, slots) * (ceil_div(tiles, c) + fixed_tiles);
+      if (cost < best) {
+        best = cost;
+        s = c;
+      }
+    }
   }
   return static_cast<int>(std::max<int64_t>(1, std::min<int64_t>(s, tiles)));
 }
