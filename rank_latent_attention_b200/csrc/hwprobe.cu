@@ -4,9 +4,10 @@
 //   - MUFU ex2 throughput (fp32, packed f16x2, packed bf16x2) and the FMA
 //     pipe's fp32 and packed f32x2 FMA throughput, in results per clock per SM;
 //   - exp2_poly3 (the kernels' FMA-pipe exponential) in results per clock per SM;
-//   - tcgen05.mma issue rate of back-to-back M=128 N=64 K=16 bf16 MMAs from one
-//     thread of a divergent branch and from a whole warp under elect.sync, in
-//     clocks per MMA (the tensor pipe needs 32);
+//   - tcgen05.mma rate of back-to-back M=128 K=16 bf16 MMAs: N = 64 from one
+//     thread of a divergent branch and from a whole warp under elect.sync;
+//     N = 64, 128, 256 with A in shared memory (SS) and in TMEM (TS), in
+//     clocks per MMA and MACs per clock;
 //   - mbarrier wake-up latency: clocks from one warp's arrive to another
 //     warp's try_wait (with a suspend-time hint) returning.
 // Every wait is bounded; no TMA, no peer memory.
@@ -73,19 +74,22 @@ __global__ void __launch_bounds__(512) pipe_kernel(int reps, float* sink, long l
 }
 
 // ------------------------------------------------------------------ tcgen05.mma issue
-// One CTA; warp 0 allocates 64 TMEM columns.  ELECT = false: thread 0 alone
+// One CTA; warp 0 allocates 512 TMEM columns.  ELECT = false: thread 0 alone
 // (a divergent branch) issues n MMAs; true: warp 1 runs the loop as a whole
-// and issues each MMA under elect.sync.  The operands are zeros in shared
-// memory in the 128-byte-swizzled K-major layout (A 128 x 64, B 64 x 64 bf16).
-template <bool ELECT>
+// and issues each MMA under elect.sync.  M = 128, K = 16, N = NN.  The
+// operands are zeros in shared memory in the 128-byte-swizzled K-major layout
+// (A 128 x 64, B NN x 64 bf16); TS = true reads A from TMEM instead (columns
+// [256, 264), zeroed first), the form the kernels' P.V products take.
+template <bool ELECT, int NN, bool TS>
 __global__ void __launch_bounds__(64) mma_issue_kernel(int n, long long* clk, int* status) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   __shared__ uint64_t bar;
   __shared__ uint32_t taddr;
   using G = TileGeom<64>;
+  static_assert(NN == 64 || NN == 128 || NN == 256, "N");
   const int warp = threadIdx.x >> 5;
-  for (int i = threadIdx.x; i < (128 + 64) * 128 / 16; i += blockDim.x)
+  for (int i = threadIdx.x; i < (128 + NN) * 128 / 16; i += blockDim.x)
     reinterpret_cast<uint4*>(smem)[i] = make_uint4(0, 0, 0, 0);
   ptx::fence_proxy_async_smem();
   if (threadIdx.x == 0) {
@@ -93,21 +97,40 @@ __global__ void __launch_bounds__(64) mma_issue_kernel(int n, long long* clk, in
     ptx::fence_mbar_init();
   }
   if (warp == 0) {
-    ptx::tmem_alloc(&taddr, 64);
+    ptx::tmem_alloc(&taddr, 512);
     ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
   const uint32_t tm = taddr;
+  constexpr uint32_t kColA = 256;
+  if (TS) {
+    // zero the A columns: warp w writes TMEM lanes [32 w, +32) (warps 0-1
+    // reach lanes 0-63; the other lanes hold whatever was there, which only
+    // changes the values, not the timing)
+    const uint32_t z[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    ptx::tmem_st8(tm + (static_cast<uint32_t>(warp * 32) << 16) + kColA, z);
+    ptx::tmem_wait_st();
+  }
+  ptx::tc_fence_before();
+  __syncthreads();
+  ptx::tc_fence_after();
   const uint32_t base = ptx::smem_u32(smem);
   const uint64_t dA = G::kmajor(base, 128, 0);
-  const uint64_t dB = G::kmajor(base + 128 * 128, 64, 0);
-  constexpr uint32_t kIdesc = ptx::idesc_bf16(128, 64, 0, 0);
+  const uint64_t dB = G::kmajor(base + 128 * 128, NN, 0);
+  constexpr uint32_t kIdesc = ptx::idesc_bf16(128, NN, 0, 0);
+  auto issue = [&](int i) {
+    if (TS) {
+      ptx::mma_ts(tm, tm + kColA, dB, kIdesc, i > 0 ? 1u : 0u);
+    } else {
+      ptx::mma_ss(tm, dA, dB, kIdesc, i > 0 ? 1u : 0u);
+    }
+  };
   long long t0 = 0, t1 = 0;
   if (!ELECT && threadIdx.x == 0) {
     t0 = clock64();
-    for (int i = 0; i < n; ++i) ptx::mma_ss(tm, dA, dB, kIdesc, i > 0 ? 1u : 0u);
+    for (int i = 0; i < n; ++i) issue(i);
     ptx::mma_commit(&bar);
     if (!ptx::mbar_wait_drain(&bar, 0)) atomicExch(status, 1);
     t1 = clock64();
@@ -115,7 +138,7 @@ __global__ void __launch_bounds__(64) mma_issue_kernel(int n, long long* clk, in
   if (ELECT && warp == 1) {
     t0 = clock64();
     for (int i = 0; i < n; ++i) {
-      if (ptx::elect_one()) ptx::mma_ss(tm, dA, dB, kIdesc, i > 0 ? 1u : 0u);
+      if (ptx::elect_one()) issue(i);
       __syncwarp();
     }
     if (ptx::elect_one()) ptx::mma_commit(&bar);
@@ -129,8 +152,23 @@ __global__ void __launch_bounds__(64) mma_issue_kernel(int n, long long* clk, in
   __syncthreads();
   if (warp == 0) {
     ptx::tc_fence_after();
-    ptx::tmem_dealloc(tm, 64);
+    ptx::tmem_dealloc(tm, 512);
   }
+}
+
+template <bool ELECT, int NN, bool TS>
+void mma_rate(int n, long long* clk, int* status) {
+  const int smem = (128 + NN) * 128 + 1024;
+  auto k = mma_issue_kernel<ELECT, NN, TS>;
+  if (cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) return;
+  long long c = 0;
+  for (int it = 0; it < 2; ++it) k<<<1, 64, smem>>>(n, clk, status);
+  if (cudaMemcpy(&c, clk, sizeof(c), cudaMemcpyDeviceToHost) != cudaSuccess) c = -1;
+  const double per = static_cast<double>(c) / n;
+  printf("{\"probe\": \"tcgen05.mma M128 N%d K16 bf16 %s, back to back\", \"issuer\": \"%s\", \"mmas\": %d, "
+         "\"clocks_per_mma\": %.1f, \"mac_per_clk\": %.0f}\n",
+         NN, TS ? "TS (A in TMEM)" : "SS", ELECT ? "warp, elect.sync" : "one thread (divergent)", n, per,
+         128.0 * NN * 16 / per);
 }
 
 // ------------------------------------------------------------------ mbarrier wake-up
@@ -209,23 +247,15 @@ int main() {
   // exp2_poly3_x2 plus one fma.rn.f32x2 that keeps its input in range
   pipe_rate<5>("exp2_poly3_x2 (+1 fma.f32x2)", 2, prop.multiProcessorCount, sink, clk);
 
-  const int smem = (128 + 64) * 128 + 1024;
   for (int n : {256, 1024}) {
-    for (int mode = 0; mode < 2; ++mode) {
-      long long c = 0;
-      for (int it = 0; it < 2; ++it) {
-        if (mode == 0) {
-          mma_issue_kernel<false><<<1, 64, smem>>>(n, clk, status);
-        } else {
-          mma_issue_kernel<true><<<1, 64, smem>>>(n, clk, status);
-        }
-      }
-      if (cudaMemcpy(&c, clk, sizeof(c), cudaMemcpyDeviceToHost) != cudaSuccess) c = -1;
-      printf("{\"probe\": \"tcgen05.mma M128 N64 K16 bf16 SS, back to back\", \"issuer\": \"%s\", \"mmas\": %d, "
-             "\"clocks_per_mma\": %.1f}\n",
-             mode ? "warp, elect.sync" : "one thread (divergent)", n, static_cast<double>(c) / n);
-    }
+    mma_rate<false, 64, false>(n, clk, status);
+    mma_rate<true, 64, false>(n, clk, status);
   }
+  mma_rate<true, 128, false>(1024, clk, status);
+  mma_rate<true, 256, false>(1024, clk, status);
+  mma_rate<true, 64, true>(1024, clk, status);
+  mma_rate<true, 128, true>(1024, clk, status);
+  mma_rate<true, 256, true>(1024, clk, status);
 
   const int rounds = 64;
   mbar_wake_kernel<<<1, 64>>>(rounds, clk, status);

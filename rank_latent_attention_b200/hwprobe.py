@@ -5,8 +5,9 @@
 Builds csrc/hwprobe.cu with nvcc into a temporary directory, runs it on the
 current device and prints its JSON lines: MUFU ex2 throughput (fp32 and the
 packed f16x2 / bf16x2 forms), fp32 and packed f32x2 FMA throughput,
-exp2_poly3 throughput, tcgen05.mma issue rate from one divergent thread and
-from a warp under elect.sync, and the mbarrier wake-up latency.
+exp2_poly3 throughput, tcgen05.mma rate (from one divergent thread and from
+a warp under elect.sync; N = 64, 128, 256 with A in shared memory or TMEM),
+and the mbarrier wake-up latency.
 """
 from __future__ import annotations
 
