@@ -15,16 +15,27 @@
 //
 // One CTA per (token range, head); the five [M][D] latent matrices of the
 // head stay in shared memory for the whole range (TMA, loaded once), the
-// token tiles K, dY, V come in by TMA per tile.  Warps 0-7 turn logits into
-// weights, two per TMEM lane quarter (one token row per thread, one half of
-// a chunk's latents per warp); warp 8 issues the TMA loads and the MMAs.
-// Logits are double-buffered: the MMAs of chunk g + 1 run while the rows
-// turn chunk g into weights.
+// token tiles K, dY, V come in by TMA per tile.  Warps 0-15 turn logits into
+// weights, four per TMEM lane quarter (one token row per thread, 8 of a
+// chunk's 32 latents per warp).  Two issuer warps: warp 16 issues the TMA
+// loads and the logit MMAs, warp 17 the accumulation MMAs.  A thread with
+// MMAs in flight stalls on its next mbarrier wait until they complete, so
+// with one issuer every wait (for weights, for a buffer, for the next token
+// tile) also waited for the other kind of MMA; measured on one B200 the
+// single issuer held a chunk to ~2,400 clocks where its MMAs take ~860.
+// Logits run two chunks ahead in two TMEM buffers: the logits of chunk g + 2
+// go into chunk g's buffer as soon as every row has read chunk g, while the
+// rows turn it into weights.  The weights have a TMEM region of their own,
+// single-buffered: the rows store chunk g + 1's once the accumulation of
+// chunk g has read chunk g's.  The token buffer is single: the next tile's
+// K, dY, V are loaded as soon as the logits of this tile's last chunk are
+// done, and only the logits issuer waits for them to land.
 //
-// TMEM columns, logit buffer b at 160 b: S3 [0,32) S1 [32,64) dA2 [64,96)
-// dA1 [96,128) dP3 [128,160) (S3 | S1 and dA2 | dA1 are one MMA each); the
-// weights (bf16 pairs) go over S3 and S1 once read (BtcCfg::w_col);
-// dK [320, 320+D), dV [320+D, 320+2D).
+// TMEM columns: logit buffer b at 160 b: S3 [0,32) S1 [32,64) dA2 [64,96)
+// dA1 [96,128) dP3 [128,160) (S3 | S1 and dA2 | dA1 are one MMA each);
+// weights (bf16 pairs) at 320: wQ, wS, wZ, wD 16 columns each, K step kk of
+// the accumulation (latents [16 kk, +16) of the chunk) at 8 kk of each;
+// dK [384, 384+D), dV [384+D, 384+2D).
 #pragma once
 
 #include <cuda.h>
@@ -55,8 +66,10 @@ struct BwdTcArgs {
 template <int D>
 struct BtcCfg {
   using G = TileGeom<D>;
-  static constexpr int kThreads = 288;
-  static constexpr int kIssuerWarp = 8;  // warps 0-7: two per TMEM lane quarter
+  static constexpr int kRowWarps = 16;  // four per TMEM lane quarter
+  static constexpr int kIssuerWarp = 16;  // logits and loads; warp 17: accumulation
+  static constexpr int kThreads = 32 * 18;
+  static constexpr int kLatPerWarp = kBtcChunk / 4;  // latents of a chunk per row warp
   static constexpr int kMPad = 256;  // latent rows reserved per matrix (M <= 256)
   static constexpr int kLatBytes = G::bytes(kMPad);
   // Latent rows in shared memory, chunk by chunk: block c holds the 32 rows
@@ -71,21 +84,16 @@ struct BtcCfg {
   static constexpr int kOffTok = 5 * kLatBytes;            // K, dY, V
   static constexpr int kOffStats = kOffTok + 3 * kTokBytes;  // float4 {L1, L2, c1, c2} [kMPad]
   static constexpr int kOffBars = kOffStats + 4 * kMPad * 4;
-  static constexpr int kNumBars = 10;
+  static constexpr int kNumBars = 12;
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static_assert(kSmemBytes <= 227 * 1024, "shared memory budget");
-  // logit buffer b at kBufCols * b: S3 [0,32) S1 [32,64) dA2 [64,96)
-  // dA1 [96,128) dP3 [128,160).  The weights of latents [16 hh, 16 hh + 16)
-  // (K step hh of the accumulation) overwrite columns [16 hh, 16 hh + 16) of
-  // S3 (wQ, then wS) and of S1 (wZ, then wD): the columns that the warp
-  // handling those latents has itself just read.
   static constexpr uint32_t kBufCols = 160;
-  __host__ __device__ static constexpr uint32_t w_col(int which, int hh) {
-    return (which >> 1) * 32 + hh * 16 + (which & 1) * 8;  // which: 0 wQ, 1 wS, 2 wZ, 3 wD
-  }
-  static constexpr uint32_t kColDK = 2 * kBufCols;
-  static constexpr uint32_t kColDV = 2 * kBufCols + D;
+  static constexpr uint32_t kColW = 2 * kBufCols;
+  // which: 0 wQ, 1 wS, 2 wZ, 3 wD; K step kk covers latents [16 kk, +16) of the chunk
+  __host__ __device__ static constexpr uint32_t w_col(int which, int kk) { return kColW + which * 16 + kk * 8; }
+  static constexpr uint32_t kColDK = kColW + 64;
+  static constexpr uint32_t kColDV = kColDK + D;
   static_assert(kColDV + D <= 512, "TMEM budget");
   static constexpr uint32_t kIdescLogit = ptx::idesc_bf16(kBtcTile, kBtcChunk, 0, 0);
   static constexpr uint32_t kIdescLogit2 = ptx::idesc_bf16(kBtcTile, 2 * kBtcChunk, 0, 0);
@@ -107,12 +115,14 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* bar_lat = bars + 0;   // latent matrices landed
-  uint64_t* bar_tok = bars + 1;   // token tile landed
+  uint64_t* bar_tok = bars + 1;   // a token tile landed (once per tile)
   uint64_t* bar_S = bars + 2;     // [2] logits of a chunk computed, per buffer
-  uint64_t* bar_W = bars + 4;     // [2] weights of a chunk stored (4 warps), per buffer
-  uint64_t* bar_acc = bars + 6;   // last accumulation of a tile done
-  uint64_t* bar_free = bars + 7;  // dK, dV of a tile read out (4 warps)
-  uint64_t* drain = bars + 8;
+  uint64_t* bar_R = bars + 4;     // [2] logits of a chunk read by every row warp (16), per buffer
+  uint64_t* bar_W = bars + 6;     // weights of a chunk stored (16)
+  uint64_t* bar_accd = bars + 7;  // accumulation of a chunk done (its weights read)
+  uint64_t* bar_acc = bars + 8;   // last accumulation of a tile done
+  uint64_t* bar_free = bars + 9;  // dK, dV of a tile read out (16)
+  uint64_t* drain = bars + 10;
   float4* sStat = reinterpret_cast<float4*>(smem + C::kOffStats);  // per latent {L1, L2, c1, c2}
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -130,11 +140,13 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
     ptx::mbar_init(bar_tok, 1);
     for (int b = 0; b < 2; ++b) {
       ptx::mbar_init(&bar_S[b], 1);
-      ptx::mbar_init(&bar_W[b], 8);
+      ptx::mbar_init(&bar_R[b], C::kRowWarps);
     }
+    ptx::mbar_init(bar_W, C::kRowWarps);
+    ptx::mbar_init(bar_accd, 1);
     ptx::mbar_init(bar_acc, 1);
-    ptx::mbar_init(bar_free, 8);
-    ptx::mbar_init(drain, 32);
+    ptx::mbar_init(bar_free, C::kRowWarps);
+    ptx::mbar_init(drain, 64);  // one commit per lane of the two issuer warps
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
@@ -157,100 +169,100 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
   const uint32_t tmem = *s_tmem;
   const uint32_t sbase = ptx::smem_u32(smem);
 
-  if (warp == C::kIssuerWarp) {
+  if (warp >= C::kIssuerWarp) {
     // ---------------------------------------------------------------- loads + MMAs
+    // Each issuer warp runs its loop as a whole (waits are warp-wide); one
+    // elected lane issues each batch of MMAs, loads and commits.
     const uint32_t aLat = sbase + C::kOffLat;  // matrix j at aLat + j * kLatBytes
     const uint32_t aTok = sbase + C::kOffTok;  // K, dY, V
+    const int nG = T * nC;  // chunks of the CTA, in order; chunk g uses logit buffer g & 1
     bool ok = true;
     int tok_issued = -1;
-    if (ptx::elect_one()) {
-      ptx::mbar_arrive_expect_tx(bar_lat, 5 * nC * kBtcChunk * D * 2);
-      const CUtensorMap* maps[5] = {&tmQd, &tmS, &tmdZ, &tmdQ, &tmZ};  // block order
-      for (int c = 0; c < nC; ++c)
-        for (int j = 0; j < 5; ++j)
-          ptx::tma_load_3d(smem + C::kOffLat + C::lat_row(c, j) * G::kRowBytes, maps[j], bar_lat, 0, c * kBtcChunk,
-                           j == 1 ? h : bh);
-    }
-    __syncwarp();
-    const int nG = T * nC;  // chunks of the CTA, in order; chunk g uses logit buffer g & 1
-    auto load_tokens = [&](int i) {
+    auto wait = [&](uint64_t* bar, int parity) -> bool {
+      return __all_sync(0xffffffffu, ptx::mbar_wait(bar, parity, s_abort, args.wait_ns));
+    };
+    if (warp == C::kIssuerWarp) {
+      // ------------------------------------------------ logits and loads
       if (ptx::elect_one()) {
-        const int tok = (tile0 + i) * kBtcTile;
-        ptx::mbar_arrive_expect_tx(bar_tok, 3 * C::kTokBytes);
-        ptx::tma_load_3d(smem + C::kOffTok, &tmK, bar_tok, 0, tok, bh);
-        ptx::tma_load_3d(smem + C::kOffTok + C::kTokBytes, &tmdY, bar_tok, 0, tok, bh);
-        ptx::tma_load_3d(smem + C::kOffTok + 2 * C::kTokBytes, &tmV, bar_tok, 0, tok, bh);
+        ptx::mbar_arrive_expect_tx(bar_lat, 5 * nC * kBtcChunk * D * 2);
+        const CUtensorMap* maps[5] = {&tmQd, &tmS, &tmdZ, &tmdQ, &tmZ};  // block order
+        for (int c = 0; c < nC; ++c)
+          for (int j = 0; j < 5; ++j)
+            ptx::tma_load_3d(smem + C::kOffLat + C::lat_row(c, j) * G::kRowBytes, maps[j], bar_lat, 0,
+                             c * kBtcChunk, j == 1 ? h : bh);
       }
       __syncwarp();
-      tok_issued = i;
-    };
-    auto issue_logits = [&](int g) {
-      ptx::tc_fence_after();
-      if (ptx::elect_one()) {
-        const uint32_t buf = tmem + C::kBufCols * (g & 1);
-        const int c = g % nC;
-        auto lat = [&](int pos) { return aLat + C::lat_row(c, pos) * G::kRowBytes; };
+      auto load_tokens = [&](int i) {
+        if (ptx::elect_one()) {
+          const int tok = (tile0 + i) * kBtcTile;
+          ptx::mbar_arrive_expect_tx(bar_tok, 3 * C::kTokBytes);
+          ptx::tma_load_3d(smem + C::kOffTok, &tmK, bar_tok, 0, tok, bh);
+          ptx::tma_load_3d(smem + C::kOffTok + C::kTokBytes, &tmdY, bar_tok, 0, tok, bh);
+          ptx::tma_load_3d(smem + C::kOffTok + 2 * C::kTokBytes, &tmV, bar_tok, 0, tok, bh);
+        }
+        __syncwarp();
+        tok_issued = i;
+      };
+      if (nG > 0) {
+        load_tokens(0);
+        ok = wait(bar_tok, 0) && wait(bar_lat, 0);
+      }
+      for (int g = 0; ok && g < nG; ++g) {
+        // a tile's first chunk: its tokens were loaded once the logits of the
+        // tile before were done
+        if (g % nC == 0 && g > 0 && !(ok = wait(bar_tok, (g / nC) & 1))) break;
+        // the buffer of chunk g - 2 has been read by every row warp
+        if (g >= 2 && !(ok = wait(&bar_R[g & 1], ((g - 2) >> 1) & 1))) break;
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
+          const uint32_t buf = tmem + C::kBufCols * (g & 1);
+          const int c = g % nC;
+          auto lat = [&](int pos) { return aLat + C::lat_row(c, pos) * G::kRowBytes; };
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint64_t dKt = G::kmajor(aTok, kBtcTile, k);
-          const uint64_t ddY = G::kmajor(aTok + C::kTokBytes, kBtcTile, k);
-          const uint64_t dVt = G::kmajor(aTok + 2 * C::kTokBytes, kBtcTile, k);
-          const uint32_t acc = k > 0 ? 1u : 0u;
-          ptx::mma_ss(buf + 0, dKt, G::kmajor(lat(0), 2 * kBtcChunk, k), C::kIdescLogit2, acc);   // S3 | S1
-          ptx::mma_ss(buf + 64, dVt, G::kmajor(lat(2), 2 * kBtcChunk, k), C::kIdescLogit2, acc);  // dA2 | dA1
-          ptx::mma_ss(buf + 128, ddY, G::kmajor(lat(4), kBtcChunk, k), C::kIdescLogit, acc);      // dP3
+          for (int k = 0; k < D / 16; ++k) {
+            const uint64_t dKt = G::kmajor(aTok, kBtcTile, k);
+            const uint64_t ddY = G::kmajor(aTok + C::kTokBytes, kBtcTile, k);
+            const uint64_t dVt = G::kmajor(aTok + 2 * C::kTokBytes, kBtcTile, k);
+            const uint32_t acc = k > 0 ? 1u : 0u;
+            ptx::mma_ss(buf + 0, dKt, G::kmajor(lat(0), 2 * kBtcChunk, k), C::kIdescLogit2, acc);   // S3 | S1
+            ptx::mma_ss(buf + 64, dVt, G::kmajor(lat(2), 2 * kBtcChunk, k), C::kIdescLogit2, acc);  // dA2 | dA1
+            ptx::mma_ss(buf + 128, ddY, G::kmajor(lat(4), kBtcChunk, k), C::kIdescLogit, acc);      // dP3
+          }
+          ptx::mma_commit(&bar_S[g & 1]);
         }
-        ptx::mma_commit(&bar_S[g & 1]);
+        __syncwarp();
+        // the last chunk of a tile: once its logits are done, the token
+        // buffer takes the next tile
+        if (g + 1 < nG && (g + 1) % nC == 0) {
+          if (!(ok = wait(&bar_S[g & 1], (g >> 1) & 1))) break;
+          load_tokens((g + 1) / nC);
+        }
       }
-      __syncwarp();
-    };
-    // accumulation of chunk g; false on a timed-out wait
-    auto issue_acc = [&](int g) -> bool {
-      const int i = g / nC, c = g % nC;
-      bool w = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_W[g & 1], (g >> 1) & 1, s_abort, args.wait_ns) &&
-                                           (c > 0 || i == 0 || ptx::mbar_wait(bar_free, (i - 1) & 1, s_abort, args.wait_ns)));
-      if (!w) return false;
-      ptx::tc_fence_after();
-      if (ptx::elect_one()) {
-        const uint32_t buf = tmem + C::kBufCols * (g & 1);
+    } else {
+      // ------------------------------------------------ accumulation
+      for (int g = 0; ok && g < nG; ++g) {
+        const int i = g / nC, c = g % nC;
+        // the first chunk of a tile also waits for the previous tile's dK, dV
+        // to be read out
+        ok = wait(bar_W, g & 1) && (c > 0 || i == 0 || wait(bar_free, (i - 1) & 1));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < kBtcChunk / 16; ++kk) {
-          const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
-          auto mn = [&](int pos) {
-            return G::mnmajor(aLat + C::lat_row(c, pos) * G::kRowBytes, C::kChunkRows, kk);
-          };
-          ptx::mma_ts(tmem + C::kColDK, buf + C::w_col(0, kk), mn(0), C::kIdescAcc, first);  // wQ Q_dyn
-          ptx::mma_ts(tmem + C::kColDK, buf + C::w_col(1, kk), mn(1), C::kIdescAcc, 1u);     // wS Q~
-          ptx::mma_ts(tmem + C::kColDV, buf + C::w_col(2, kk), mn(2), C::kIdescAcc, first);  // wZ dZ
-          ptx::mma_ts(tmem + C::kColDV, buf + C::w_col(3, kk), mn(3), C::kIdescAcc, 1u);     // wD dQ_dyn
+          for (int kk = 0; kk < kBtcChunk / 16; ++kk) {
+            const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
+            auto mn = [&](int pos) {
+              return G::mnmajor(aLat + C::lat_row(c, pos) * G::kRowBytes, C::kChunkRows, kk);
+            };
+            ptx::mma_ts(tmem + C::kColDK, tmem + C::w_col(0, kk), mn(0), C::kIdescAcc, first);  // wQ Q_dyn
+            ptx::mma_ts(tmem + C::kColDK, tmem + C::w_col(1, kk), mn(1), C::kIdescAcc, 1u);     // wS Q~
+            ptx::mma_ts(tmem + C::kColDV, tmem + C::w_col(2, kk), mn(2), C::kIdescAcc, first);  // wZ dZ
+            ptx::mma_ts(tmem + C::kColDV, tmem + C::w_col(3, kk), mn(3), C::kIdescAcc, 1u);     // wD dQ_dyn
+          }
+          ptx::mma_commit(bar_accd);
+          if (c == nC - 1) ptx::mma_commit(bar_acc);
         }
-        if (c == nC - 1) ptx::mma_commit(bar_acc);
-      }
-      __syncwarp();
-      return true;
-    };
-    if (nG > 0) {
-      load_tokens(0);
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_tok, 0, s_abort, args.wait_ns) &&
-                                       ptx::mbar_wait(bar_lat, 0, s_abort, args.wait_ns));
-      if (ok) issue_logits(0);
-    }
-    for (int g = 0; ok && g < nG; ++g) {
-      const bool more = g + 1 < nG;
-      const bool new_tile = more && (g + 1) % nC == 0;
-      // the next chunk's logits go into the other buffer while this chunk's
-      // weights are computed (its rows read that buffer two chunks ago)
-      if (more && !new_tile) issue_logits(g + 1);
-      ok = issue_acc(g);
-      if (ok && new_tile) {
-        const int i = g / nC;
-        // every MMA of tile i done: the token tiles may be overwritten
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, i & 1, s_abort, args.wait_ns));
-        if (ok) {
-          load_tokens(i + 1);
-          ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_tok, (i + 1) & 1, s_abort, args.wait_ns));
-        }
-        if (ok) issue_logits(g + 1);
+        __syncwarp();
       }
     }
     if (!ok) {
@@ -258,90 +270,125 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       *s_abort = 1;
     }
     // every MMA and every load issued completes before the CTA releases TMEM
+    // (each lane of both issuer warps commits)
     ptx::mma_commit(drain);
     ptx::mbar_wait_drain(drain, 0);
     if (tok_issued >= 0) ptx::mbar_wait_drain(bar_tok, tok_issued & 1);
-    ptx::mbar_wait_drain(bar_lat, 0);
+    if (warp == C::kIssuerWarp) ptx::mbar_wait_drain(bar_lat, 0);
   } else {
     // ---------------------------------------------------------------- weights
-    const int quarter = warp & 3, hh = warp >> 2;  // TMEM lanes 32 quarter.., latents 16 hh.. of a chunk
+    const int quarter = warp & 3, hq = warp >> 2;  // TMEM lanes 32 quarter.., latents 8 hq.. of a chunk
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t trow = tmem + lane_off;
     const size_t tok_base = static_cast<size_t>(bh) * args.N;
+    // this warp's weights: 4 columns (8 latents as bf16 pairs) of K step hq / 2
+    const uint32_t wcol = (hq >> 1) * 8 + (hq & 1) * 4;
+    // Read-out of dK (warps hq 0-1) or dV (hq 2-3): columns [d_lo, d_lo + D / 2)
+    // of this lane's row.  Each lane writes its own row, so a store touches 32
+    // lines: 32-byte stores (when both outputs are 32-byte aligned; 16-column
+    // groups of a row half then are too) halve the requests of 16-byte ones.
+    constexpr int kHalfD = D / 2;
+    constexpr int kGroupCols = kHalfD < 16 ? kHalfD : 16;
+    const int which = hq >> 1, d_lo = (hq & 1) * kHalfD;
+    const uint32_t col_out = (which == 0 ? C::kColDK : C::kColDV) + d_lo;
+    __nv_bfloat16* const out = which == 0 ? args.dK : args.dV;
+    const bool wide = kGroupCols == 16 &&
+                      ((reinterpret_cast<uintptr_t>(args.dK) | reinterpret_cast<uintptr_t>(args.dV)) & 31u) == 0;
+    auto row_of = [&](int i) { return static_cast<long long>(tile0 + i) * kBtcTile + quarter * 32 + lane; };
+    // a tile's row statistics are loaded while the tile before is read out
+    auto row_stats = [&](int i, float& L3, float& dl) {
+      const long long n = row_of(i);
+      const bool live = n < args.N;
+      L3 = live ? args.lse3[tok_base + n] * kL2e : 0.f;
+      dl = live ? args.delta[tok_base + n] : 0.f;
+    };
+    float L3n = 0.f, dln = 0.f;  // the next tile's row statistics, loaded a tile ahead
+    if (T > 0) row_stats(0, L3n, dln);
     bool ok = true;
     int kc = 0;
     for (int i = 0; ok && i < T; ++i) {
-      const long long n = static_cast<long long>(tile0 + i) * kBtcTile + quarter * 32 + lane;
+      const long long n = row_of(i);
       const bool live_tok = n < args.N;
-      const float L3 = live_tok ? args.lse3[tok_base + n] * kL2e : 0.f;
-      const float dl = live_tok ? args.delta[tok_base + n] : 0.f;
+      const float L3 = L3n, dl = dln;
       for (int c = 0; c < nC; ++c, ++kc) {
         const int b = kc & 1;
-        const uint32_t buf = trow + C::kBufCols * b;
+        const uint32_t buf = trow + C::kBufCols * b + hq * C::kLatPerWarp;
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&bar_S[b], (kc >> 1) & 1, s_abort, args.wait_ns));
         if (!ok) break;
         ptx::tc_fence_after();
-        {
-          float s3[16], dp[16], da2[16], s1[16], da1[16];
-          ptx::tmem_ld16(buf + 0 + hh * 16, s3);
-          ptx::tmem_ld16(buf + 32 + hh * 16, s1);
-          ptx::tmem_ld16(buf + 64 + hh * 16, da2);
-          ptx::tmem_ld16(buf + 96 + hh * 16, da1);
-          ptx::tmem_ld16(buf + 128 + hh * 16, dp);
-          ptx::tmem_wait_ld();
-          uint32_t wq[8], ws[8], wz[8], wd[8];
+        float s3[8], dp[8], da2[8], s1[8], da1[8];
+        ptx::tmem_ld8(buf + 0, s3);
+        ptx::tmem_ld8(buf + 32, s1);
+        ptx::tmem_ld8(buf + 64, da2);
+        ptx::tmem_ld8(buf + 96, da1);
+        ptx::tmem_ld8(buf + 128, dp);
+        ptx::tmem_wait_ld();
+        // the buffer may take the logits of chunk kc + 2
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&bar_R[b]);
+        uint32_t wq[4], ws[4], wz[4], wd[4];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) {
-            float q[2], sd[2], z[2], dq[2];
+        for (int u = 0; u < 4; ++u) {
+          float q[2], sd[2], z[2], dq[2];
 #pragma unroll
-            for (int e = 0; e < 2; ++e) {
-              const int j = 2 * u + e;
-              const int m = c * kBtcChunk + hh * 16 + j;
-              const float4 st = sStat[m];
-              const float p3 = m < args.M ? ptx::ex2(fmaf(s3[j], kL2e, -L3)) : 0.f;
-              const float a2 = ptx::ex2(fmaf(s3[j], kL2e, -st.y));
-              const float a1 = ptx::ex2(fmaf(s1[j], kL2e, -st.x));
-              q[e] = fmaf(p3, dp[j] - dl, a2 * (da2[j] - st.w));
-              sd[e] = a1 * (da1[j] - st.z);
-              z[e] = a2;
-              dq[e] = a1;
-            }
-            wq[u] = ptx::pack_bf16(q[0], q[1]);
-            ws[u] = ptx::pack_bf16(sd[0], sd[1]);
-            wz[u] = ptx::pack_bf16(z[0], z[1]);
-            wd[u] = ptx::pack_bf16(dq[0], dq[1]);
+          for (int e = 0; e < 2; ++e) {
+            const int j = 2 * u + e;
+            const int m = c * kBtcChunk + hq * C::kLatPerWarp + j;
+            const float4 st = sStat[m];
+            const float p3 = m < args.M ? ptx::ex2(fmaf(s3[j], kL2e, -L3)) : 0.f;
+            const float a2 = ptx::ex2(fmaf(s3[j], kL2e, -st.y));
+            const float a1 = ptx::ex2(fmaf(s1[j], kL2e, -st.x));
+            q[e] = fmaf(p3, dp[j] - dl, a2 * (da2[j] - st.w));
+            sd[e] = a1 * (da1[j] - st.z);
+            z[e] = a2;
+            dq[e] = a1;
           }
-          ptx::tmem_st8(buf + C::w_col(0, hh), wq);
-          ptx::tmem_st8(buf + C::w_col(1, hh), ws);
-          ptx::tmem_st8(buf + C::w_col(2, hh), wz);
-          ptx::tmem_st8(buf + C::w_col(3, hh), wd);
+          wq[u] = ptx::pack_bf16(q[0], q[1]);
+          ws[u] = ptx::pack_bf16(sd[0], sd[1]);
+          wz[u] = ptx::pack_bf16(z[0], z[1]);
+          wd[u] = ptx::pack_bf16(dq[0], dq[1]);
         }
+        // the weights region is free once the accumulation of chunk kc - 1 has read it
+        if (kc > 0) {
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_accd, (kc - 1) & 1, s_abort, args.wait_ns));
+          if (!ok) break;
+          ptx::tc_fence_after();
+        }
+        ptx::tmem_st4(trow + C::w_col(0, 0) + wcol, wq);
+        ptx::tmem_st4(trow + C::w_col(1, 0) + wcol, ws);
+        ptx::tmem_st4(trow + C::w_col(2, 0) + wcol, wz);
+        ptx::tmem_st4(trow + C::w_col(3, 0) + wcol, wd);
         ptx::tmem_wait_st();
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&bar_W[b]);
+        if (lane == 0) ptx::mbar_arrive(bar_W);
       }
       if (!ok) break;
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_acc, i & 1, s_abort, args.wait_ns));
       if (!ok) break;
+      // the next tile's row statistics: their loads overlap the read-out
+      if (i + 1 < T) row_stats(i + 1, L3n, dln);
       ptx::tc_fence_after();
-      {
-        const int which = hh;  // warps 0-3 store dK, warps 4-7 dV
-        __nv_bfloat16* dst = (which == 0 ? args.dK : args.dV) + (tok_base + (live_tok ? n : 0)) * D;
-        const uint32_t col = which == 0 ? C::kColDK : C::kColDV;
+      __nv_bfloat16* dst = out + (tok_base + (live_tok ? n : 0)) * D + d_lo;
 #pragma unroll
-        for (int d0 = 0; d0 < D; d0 += 16) {
-          float v[16];
-          ptx::tmem_ld16(trow + col + d0, v);
-          ptx::tmem_wait_ld();
-          uint32_t pk[8];
+      for (int d0 = 0; d0 < kHalfD; d0 += kGroupCols) {
+        float v[kGroupCols];
+        if constexpr (kGroupCols == 16) ptx::tmem_ld16(trow + col_out + d0, v); else ptx::tmem_ld8(trow + col_out + d0, v);
+        ptx::tmem_wait_ld();
+        uint32_t pk[kGroupCols / 2];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) pk[u] = ptx::pack_bf16(v[2 * u], v[2 * u + 1]);
-          if (live_tok) {
-            uint4* o = reinterpret_cast<uint4*>(dst + d0);
-            o[0] = make_uint4(pk[0], pk[1], pk[2], pk[3]);
-            o[1] = make_uint4(pk[4], pk[5], pk[6], pk[7]);
+        for (int u = 0; u < kGroupCols / 2; ++u) pk[u] = ptx::pack_bf16(v[2 * u], v[2 * u + 1]);
+        if (live_tok) {
+          if constexpr (kGroupCols == 16) {
+            if (wide) {
+              ptx::st_global_v8(dst + d0, pk);
+              continue;
+            }
           }
+          uint4* o = reinterpret_cast<uint4*>(dst + d0);
+#pragma unroll
+          for (int z = 0; z < kGroupCols / 8; ++z) o[z] = make_uint4(pk[4 * z], pk[4 * z + 1], pk[4 * z + 2], pk[4 * z + 3]);
         }
       }
       ptx::tc_fence_before();
