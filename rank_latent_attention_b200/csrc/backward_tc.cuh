@@ -207,6 +207,13 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
         load_tokens(0);
         ok = wait(bar_tok, 0) && wait(bar_lat, 0);
       }
+      // Operand descriptors built once: only the start-address field moves
+      // between K steps, chunks and tensors, so each MMA adds a constant (the
+      // issuer shares its SMSP with busy row warps; rebuilding 64-bit
+      // descriptors per MMA made each batch several hundred clocks long).
+      const uint64_t dTok = G::kmajor(aTok, kBtcTile, 0);  // K; dY and V kTokStep and 2 kTokStep on
+      constexpr uint32_t kTokStep = static_cast<uint32_t>(C::kTokBytes) >> 4;
+      const uint64_t dLat = G::kmajor(aLat, 2 * kBtcChunk, 0);
       for (int g = 0; ok && g < nG; ++g) {
         // a tile's first chunk: its tokens were loaded once the logits of the
         // tile before were done
@@ -217,16 +224,16 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
         if (ptx::elect_one()) {
           const uint32_t buf = tmem + C::kBufCols * (g & 1);
           const int c = g % nC;
-          auto lat = [&](int pos) { return aLat + C::lat_row(c, pos) * G::kRowBytes; };
+          auto lat = [&](int pos) { return dLat + ((C::lat_row(c, pos) * G::kRowBytes) >> 4); };
 #pragma unroll
           for (int k = 0; k < D / 16; ++k) {
-            const uint64_t dKt = G::kmajor(aTok, kBtcTile, k);
-            const uint64_t ddY = G::kmajor(aTok + C::kTokBytes, kBtcTile, k);
-            const uint64_t dVt = G::kmajor(aTok + 2 * C::kTokBytes, kBtcTile, k);
+            const uint32_t sk = G::kmajor_step(kBtcTile, k);
             const uint32_t acc = k > 0 ? 1u : 0u;
-            ptx::mma_ss(buf + 0, dKt, G::kmajor(lat(0), 2 * kBtcChunk, k), C::kIdescLogit2, acc);   // S3 | S1
-            ptx::mma_ss(buf + 64, dVt, G::kmajor(lat(2), 2 * kBtcChunk, k), C::kIdescLogit2, acc);  // dA2 | dA1
-            ptx::mma_ss(buf + 128, ddY, G::kmajor(lat(4), kBtcChunk, k), C::kIdescLogit, acc);      // dP3
+            ptx::mma_ss(buf + 0, dTok + sk, lat(0) + G::kmajor_step(2 * kBtcChunk, k), C::kIdescLogit2, acc);  // S3 | S1
+            ptx::mma_ss(buf + 64, dTok + 2 * kTokStep + sk, lat(2) + G::kmajor_step(2 * kBtcChunk, k), C::kIdescLogit2,
+                        acc);                                                                                 // dA2 | dA1
+            ptx::mma_ss(buf + 128, dTok + kTokStep + sk, lat(4) + G::kmajor_step(kBtcChunk, k), C::kIdescLogit,
+                        acc);                                                                                 // dP3
           }
           ptx::mma_commit(&bar_S[g & 1]);
         }
@@ -240,6 +247,7 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
       }
     } else {
       // ------------------------------------------------ accumulation
+      const uint64_t dLatMN = G::mnmajor(aLat, C::kChunkRows, 0);  // built once, as the logits' descriptors
       for (int g = 0; ok && g < nG; ++g) {
         const int i = g / nC, c = g % nC;
         // the first chunk of a tile also waits for the previous tile's dK, dV
@@ -252,7 +260,7 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
           for (int kk = 0; kk < kBtcChunk / 16; ++kk) {
             const uint32_t first = (c == 0 && kk == 0) ? 0u : 1u;
             auto mn = [&](int pos) {
-              return G::mnmajor(aLat + C::lat_row(c, pos) * G::kRowBytes, C::kChunkRows, kk);
+              return dLatMN + ((C::lat_row(c, pos) * G::kRowBytes) >> 4) + G::mnmajor_step(kk);
             };
             ptx::mma_ts(tmem + C::kColDK, tmem + C::w_col(0, kk), mn(0), C::kIdescAcc, first);  // wQ Q_dyn
             ptx::mma_ts(tmem + C::kColDK, tmem + C::w_col(1, kk), mn(1), C::kIdescAcc, 1u);     // wS Q~
@@ -531,10 +539,18 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
     __syncwarp();
     loaded = T < 2 ? T : 2;
     bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_lat, 0, s_abort, args.wait_ns));
-    const uint32_t aA = sbase + C::kOffLat, aB = aA + C::kLatBytes;
+    // Operand descriptors built once: only the start-address field moves
+    // between K steps and stages, so each MMA adds a constant (the issuer
+    // shares its SMSP with busy row warps, and rebuilding 64-bit descriptors
+    // per MMA made each batch of MMAs several hundred clocks long).
+    const uint64_t dA = G::kmajor(sbase + C::kOffLat, 128, 0);
+    const uint64_t dB = G::kmajor(sbase + C::kOffLat + C::kLatBytes, 128, 0);
+    const uint64_t dK0 = G::kmajor(sbase + C::kOffTok, kBltcTok, 0);
+    const uint64_t dKmn0 = G::mnmajor(sbase + C::kOffTok, kBltcTok, 0);
+    constexpr uint32_t kStageStep = static_cast<uint32_t>(2 * C::kTokBytes) >> 4;
+    constexpr uint32_t kXStep = static_cast<uint32_t>(C::kTokBytes) >> 4;
     for (int i = 0; ok && i < T; ++i) {
       const int st = i & 1;
-      const uint32_t aK = sbase + C::kOffTok + st * 2 * C::kTokBytes, aX = aK + C::kTokBytes;
       ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[st], (i >> 1) & 1, s_abort, args.wait_ns));
       if (!ok) break;
       ptx::tc_fence_after();
@@ -542,8 +558,9 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
 #pragma unroll
         for (int k = 0; k < D / 16; ++k) {
           const uint32_t acc = k > 0 ? 1u : 0u;
-          ptx::mma_ss(tmem + 0, G::kmajor(aA, 128, k), G::kmajor(aK, kBltcTok, k), C::kIdescLogit, acc);
-          ptx::mma_ss(tmem + 64, G::kmajor(aB, 128, k), G::kmajor(aX, kBltcTok, k), C::kIdescLogit, acc);
+          const uint32_t sa = G::kmajor_step(128, k), sk = st * kStageStep + G::kmajor_step(kBltcTok, k);
+          ptx::mma_ss(tmem + 0, dA + sa, dK0 + sk, C::kIdescLogit, acc);
+          ptx::mma_ss(tmem + 64, dB + sa, dK0 + kXStep + sk, C::kIdescLogit, acc);
         }
         ptx::mma_commit(bar_S);
       }
@@ -555,9 +572,10 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kBltcTok / 16; ++kk) {
           const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+          const uint32_t sm = st * kStageStep + G::mnmajor_step(kk);
           if constexpr (kDec)
-            ptx::mma_ts(tmem + C::kColOut0, tmem + 0 + kk * 8, G::mnmajor(aX, kBltcTok, kk), C::kIdescAcc, acc);
-          ptx::mma_ts(tmem + C::kColOut1, tmem + 64 + kk * 8, G::mnmajor(aK, kBltcTok, kk), C::kIdescAcc, acc);
+            ptx::mma_ts(tmem + C::kColOut0, tmem + 0 + kk * 8, dKmn0 + kXStep + sm, C::kIdescAcc, acc);
+          ptx::mma_ts(tmem + C::kColOut1, tmem + 64 + kk * 8, dKmn0 + sm, C::kIdescAcc, acc);
         }
         ptx::mma_commit(&empty[st]);
         if (i == T - 1) ptx::mma_commit(bar_fin);
@@ -592,18 +610,27 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
       cm = live_m ? args.c_row[lat_row] : 0.f;
     }
     const size_t tok_base = static_cast<size_t>(bh) * args.N;
+    // DEC: threads 0-63 hold the {lse3 (log2 domain), delta} of token j of
+    // the next tile, loaded a tile ahead: their latency overlaps a tile's
+    // exponentials instead of stalling every row warp at the barrier
+    auto tok_stat = [&](int i) -> float2 {
+      const long long t = static_cast<long long>(tile0 + i) * kBltcTok + threadIdx.x;
+      return t < args.N ? make_float2(args.lse3[tok_base + t] * kL2e, args.delta[tok_base + t]) : make_float2(0.f, 0.f);
+    };
+    float2 next_stat = make_float2(0.f, 0.f);
+    if (kDec && threadIdx.x < kBltcTok && T > 0) next_stat = tok_stat(0);
     bool ok = true;
     for (int i = 0; ok && i < T; ++i) {
       const long long t0 = static_cast<long long>(tile0 + i) * kBltcTok;
       const int live_cols = static_cast<int>(args.N - t0 < kBltcTok ? args.N - t0 : kBltcTok);
       float2* stat = reinterpret_cast<float2*>(sTok) + (i & 1) * kBltcTok;  // {lse3 log2 domain, delta}
       if constexpr (kDec) {
-        // the tile's token statistics, shared by the 128 rows
+        // the tile's token statistics, shared by the 128 rows (buffers
+        // alternate by tile parity; every row warp has finished tile i - 2
+        // once all of them have passed tile i - 1's barrier)
         if (threadIdx.x < kBltcTok) {
-          const int j = threadIdx.x;
-          const bool live = j < live_cols;
-          stat[j] = live ? make_float2(args.lse3[tok_base + t0 + j] * kL2e, args.delta[tok_base + t0 + j])
-                         : make_float2(0.f, 0.f);
+          stat[threadIdx.x] = next_stat;
+          if (i + 1 < T) next_stat = tok_stat(i + 1);
         }
         asm volatile("bar.sync 1, 128;" ::: "memory");
       }
