@@ -92,10 +92,11 @@ def dist_env():
 
 
 # DRAM bytes (read + write) per full-size launch of the encode, from one
-# ncu --set full capture of the same workload cut to 2 of its 16 heads and
-# scaled by tokens (traffic grows in proportion); it holds for the kernel
-# sources with this digest and is reported as null once they change.
-ENCODE_TRAFFIC = {"bytes_per_launch": 4.3236e9, "sources_sha256": "9b6cadef71f599079120ddd8b0b2cc69f259ccd6f54f80e5a4677c1ab196ea1a"}
+# ncu capture (dram__bytes_read.sum + dram__bytes_write.sum) of the same
+# workload cut to 2 of its 16 heads, scaled by heads (traffic grows in
+# proportion); it holds for the kernel sources with this digest and is
+# reported as null once they change.
+ENCODE_TRAFFIC = {"bytes_per_launch": 4.3221e9, "sources_sha256": "3e7a05fd97760ba2eaac1d20f65b98505034ec4227f46795eb2a0186176aa7a3"}
 ENCODE_SOURCES = ("encode_tc.cuh", "common.cuh", "ptx_sm100.cuh")
 
 

@@ -549,10 +549,9 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
     const uint64_t dKmn0 = G::mnmajor(sbase + C::kOffTok, kBltcTok, 0);
     constexpr uint32_t kStageStep = static_cast<uint32_t>(2 * C::kTokBytes) >> 4;
     constexpr uint32_t kXStep = static_cast<uint32_t>(C::kTokBytes) >> 4;
-    for (int i = 0; ok && i < T; ++i) {
+    // logits of tile i into S/G (stage i & 1 holds its tokens)
+    auto issue_logits = [&](int i) {
       const int st = i & 1;
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[st], (i >> 1) & 1, s_abort, args.wait_ns));
-      if (!ok) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
@@ -565,7 +564,18 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
         ptx::mma_commit(bar_S);
       }
       __syncwarp();
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_W, i & 1, s_abort, args.wait_ns));
+    };
+    if (ok && T > 0) {
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[0], 0, s_abort, args.wait_ns));
+      if (ok) issue_logits(0);
+    }
+    for (int i = 0; ok && i < T; ++i) {
+      const int st = i & 1;
+      // Every wait before the MMAs (a wait after them stalls until they
+      // complete): the rows' weights of tile i, and the tokens of tile i + 1.
+      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_W, i & 1, s_abort, args.wait_ns) &&
+                                       (i + 1 >= T || ptx::mbar_wait(&full[st ^ 1], ((i + 1) >> 1) & 1, s_abort,
+                                                                     args.wait_ns)));
       if (!ok) break;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
@@ -581,6 +591,11 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
         if (i == T - 1) ptx::mma_commit(bar_fin);
       }
       __syncwarp();
+      // The next tile's logits overwrite S/G, whose e and w the accumulation
+      // just issued reads: the tensor pipe runs MMAs in issue order, so they
+      // are issued right behind it instead of after it completes and after
+      // the stage refill below (which took ~430 clocks off every tile).
+      if (i + 1 < T) issue_logits(i + 1);
       if (i + 2 < T) {
         ok = __all_sync(0xffffffffu, ptx::mbar_wait(&empty[st], (i >> 1) & 1, s_abort, args.wait_ns));
         if (!ok) break;
