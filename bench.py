@@ -46,7 +46,8 @@ the data path.  Rank 0 prints one JSON line:
   warm-ups, L2-warm and L2-cold (a 256 MB scrub write before each call,
   outside the timed events), each call queued behind a short device-side
   spin so the events time the device's work; with tokens/s, TFLOP/s and the
-  fraction of their single-pass HBM / tensor roofline.
+  fraction of their roofline: the largest of the single-pass HBM time, the
+  tensor time and the exponentials' time on MUFU (the bound for D <= 32).
 
 --impl reference times the oracle (the reference arm of this comparison) on
 the host cores, rank 0 only, and prints the same line with "impl": "reference".
@@ -98,6 +99,7 @@ def dist_env():
 # reported as null once they change.
 ENCODE_TRAFFIC = {"bytes_per_launch": 4.3221e9, "sources_sha256": "3e7a05fd97760ba2eaac1d20f65b98505034ec4227f46795eb2a0186176aa7a3"}
 ENCODE_SOURCES = ("encode_tc.cuh", "common.cuh", "ptx_sm100.cuh")
+MAX_SM_MHZ = 1965.0  # the B200's clocks.max.sm, for MUFU floors when no clock record is at hand
 
 
 def encode_sources_digest():
@@ -701,7 +703,7 @@ def run_native(args):
     # Peak at the maximum SM clock; frac_at_clock uses the median SM clock
     # sampled under load (the kernels run power-capped).
     exps = float(w.N) * w.M * w.H
-    alu_peak = 16.0 * 148 * (clk["sm_max_mhz"] or 1965.0) * 1e6  # 1965 MHz: the B200's clocks.max.sm
+    alu_peak = 16.0 * 148 * (clk["sm_max_mhz"] or MAX_SM_MHZ) * 1e6
     alu_at_clock = 16.0 * 148 * clk["sm_mhz"] * 1e6 if clk.get("sm_mhz") else None
     alu_roof = {"bound": "alu", "kernel": "encode_tc", "unit": "exp/s", "achieved": exps / (enc_ms * 1e-3),
                 "peak": alu_peak, "frac": exps / (enc_ms * 1e-3) / alu_peak,
@@ -776,11 +778,14 @@ L2_SCRUB_BYTES = 256 << 20  # written before each L2-cold call: twice the 126 MB
 
 def small_configs(torch, flare, inputs, dev, peaks):
     """One flarepp_mix call per small workload: median of 20 event-timed calls
-    after 3 warm-ups, L2-warm and L2-cold.  Roofline per call: the larger of
+    after 3 warm-ups, L2-warm and L2-cold.  Roofline per call: the largest of
     12 N M D B H FLOP at the burst bf16 GEMM peak (bf16 workloads; each call
-    is a short region timed alone) and the single-pass bytes (K and V read
-    once, Y written once) at the measured copy bandwidth; these heads fit in
-    L2, so one pass is the minimum."""
+    is a short region timed alone), the single-pass bytes (K and V read once,
+    Y written once) at the measured copy bandwidth (these heads fit in L2,
+    so one pass is the minimum), and 3 N M B H exponentials (one per score of
+    each of the three steps) at MUFU's 16 per clock per SM on 148 SMs at the
+    maximum SM clock: with D <= 32 the exponentials, not the MMAs, bound a
+    call."""
     scrub = torch.empty(L2_SCRUB_BYTES, dtype=torch.uint8, device=dev)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     tensor_peak = peaks["bf16_tflops"]
@@ -829,11 +834,15 @@ def small_configs(torch, flare, inputs, dev, peaks):
         nbytes = 3.0 * w.N * w.D * w.B * w.H * esz
         t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3
         t_tensor = flops / (tensor_peak * 1e12) * 1e3 if w.dtype != "f32" else 0.0
-        t_roof = max(t_hbm, t_tensor)
+        exps = 3.0 * w.N * w.M * w.B * w.H
+        t_mufu = exps / (16.0 * 148 * MAX_SM_MHZ * 1e6) * 1e3
+        t_roof = max(t_hbm, t_tensor, t_mufu)
+        bound = "alu" if t_mufu >= max(t_hbm, t_tensor) else ("tensor" if t_tensor > t_hbm else "hbm")
         out[tag] = {"workload": name, "B": w.B, "H": w.H, "N": w.N, "M": w.M, "D": w.D, "dtype": w.dtype,
                     "ms_warm": ms_w, "ms_cold": ms_c, "tokens_per_s_cold": w.B * w.N / (ms_c * 1e-3),
                     "tflops_cold": flops / (ms_c * 1e-3) / 1e12, "roofline_ms": t_roof,
-                    "bound": "tensor" if t_tensor > t_hbm else "hbm", "frac_cold": t_roof / ms_c,
+                    "roofline_parts_ms": {"tensor": t_tensor, "hbm": t_hbm, "mufu": t_mufu},
+                    "bound": bound, "frac_cold": t_roof / ms_c,
                     "calls": 20,
                     "launch_us": [[k, t] for (k, _), t in zip(recs[-len(per_launch):], per_launch)]}
         del s_d, K_d, V_d, Y_d, ws
