@@ -288,18 +288,29 @@ class ClockSampler:
         self.stop = threading.Event()
 
     def _nvml_handle(self):
+        """(pynvml, handle, how matched): the NVML device of CUDA device self.gpu,
+        by UUID, else by PCI bus id, else (CUDA_VISIBLE_DEVICES unset) by index."""
         import pynvml
         import torch
         pynvml.nvmlInit()
+        props = torch.cuda.get_device_properties(self.gpu)
         try:
-            uuid = str(torch.cuda.get_device_properties(self.gpu).uuid)
-            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid)
+            uuid = str(props.uuid)
+            return pynvml, pynvml.nvmlDeviceGetHandleByUUID(uuid if uuid.startswith("GPU-") else "GPU-" + uuid), "uuid"
         except Exception:
-            return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu)
+            pass
+        try:
+            bus = f"{props.pci_domain_id:08x}:{props.pci_bus_id:02x}:{props.pci_device_id:02x}.0"
+            return pynvml, pynvml.nvmlDeviceGetHandleByPciBusId(bus), "pci bus id"
+        except Exception:
+            pass
+        if os.environ.get("CUDA_VISIBLE_DEVICES"):
+            raise RuntimeError("cannot match the CUDA device to an NVML device")
+        return pynvml, pynvml.nvmlDeviceGetHandleByIndex(self.gpu), "index"
 
     def __enter__(self):
         try:
-            nv, h = self._nvml_handle()
+            nv, h, how = self._nvml_handle()
             bits = {"hw_slowdown": nv.nvmlClocksEventReasonHwSlowdown,
                     "hw_thermal_slowdown": nv.nvmlClocksEventReasonHwThermalSlowdown,
                     "sw_thermal_slowdown": nv.nvmlClocksEventReasonSwThermalSlowdown,
@@ -316,7 +327,7 @@ class ClockSampler:
                         pass
                     self.stop.wait(self.PERIOD_S)
 
-            self.source = "nvml, 10 ms"
+            self.source = f"nvml ({how}), 10 ms"
             self.thread = threading.Thread(target=poll, daemon=True)
             self.thread.start()
             return self
