@@ -318,8 +318,9 @@ const char* flare_cuda_error_string(void);
  *     every token-split kernel, each clamped to that kernel's number of token
  *     tiles (64 tokens for the encode and the backward's latent-side kernel,
  *     128 for the decode, the statistics and the token-gradient kernels); 0
- *     restores the built-in choice (whole waves of the SMs' resident CTA
- *     slots, at most ~32k tokens per CTA).
+ *     restores the built-in choice: the count that minimises (waves of the
+ *     SMs' resident CTA slots) x (tiles per CTA + a fixed per-CTA cost of
+ *     384 tokens), among counts that keep a CTA at most ~32k tokens.
  *   flare_set_wait_limit_ms(ms): how long a tensor-core kernel waits on one
  *     barrier before recording FLARE_ERR_TIMEOUT and returning (default 2000).
  *   flare_set_launch_overlap(mode): whether the mixer's merges, routing
