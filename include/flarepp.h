@@ -94,7 +94,9 @@ size_t flarepp_workspace_size(int B, int H, int64_t N, int M, int D, int dtype);
  *   K, V       [B][H][N][D]
  *   Z          [B][H][M][D] output
  * The token axis is split across CTAs; the per-split softmax statistics are
- * merged exactly (log-sum-exp) in a second kernel.
+ * merged exactly (log-sum-exp) in a second kernel.  With one CTA per head
+ * (flare_encode_splits() == 1, tensor-core modes) the encode writes the
+ * normalised result itself and no second kernel runs.
  */
 int flare_encode(const void* Q, int q_batched, const void* K, const void* V, void* Z, int B, int H, int64_t N,
                  int M, int D, int dtype, void* workspace, size_t workspace_bytes, void* stream);
@@ -334,6 +336,14 @@ const char* flare_cuda_error_string(void);
  * All return the previous value.
  */
 int flare_set_split_override(int splits);
+/*
+ * The number of CTAs per head along the tokens that the tensor-core encode
+ * uses for B x H heads of N tokens (the built-in choice, or the override):
+ * with 1, the encode writes its normalised result and log-sum-exp itself
+ * and no lse_merge_kernel follows it.  0 for B, H or N below 1.  Reads
+ * only host state; no device work.
+ */
+int flare_encode_splits(int B, int H, int64_t N);
 int flare_set_wait_limit_ms(int ms);
 int flare_set_launch_overlap(int mode);
 

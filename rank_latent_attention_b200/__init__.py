@@ -44,6 +44,7 @@ __all__ = [
     "flare_last_launch_count",
     "flare_cuda_error_string",
     "flare_set_split_override",
+    "flare_encode_splits",
     "flare_set_launch_overlap",
     "flare_set_wait_limit_ms",
     "flare_profile_begin",
@@ -90,6 +91,7 @@ _SIGNATURES = {
     "flare_communication_workspace_size": (_c_size, _SIZES),
     "flare_communication_matrix": (_c_int, [_vp, _c_int, _vp, _vp, *_SIZES, _vp, _c_size, _vp]),
     "flare_set_split_override": (_c_int, [_c_int]),
+    "flare_encode_splits": (_c_int, [_c_int, _c_int, ctypes.c_int64]),
     "flare_set_launch_overlap": (_c_int, [_c_int]),
     "flare_selftest_wait_timeout": (_c_int, [_c_int, _vp]),
     "flare_set_wait_limit_ms": (_c_int, [_c_int]),
@@ -465,6 +467,11 @@ def flare_last_launch_count() -> int:
 
 def flare_set_split_override(splits: int) -> int:
     return lib().flare_set_split_override(splits)
+
+
+def flare_encode_splits(B: int, H: int, N: int) -> int:
+    """CTAs per head of the tensor-core encode for B x H heads of N tokens (1: no merge follows)."""
+    return lib().flare_encode_splits(B, H, N)
 
 
 def flare_set_launch_overlap(mode: int) -> int:

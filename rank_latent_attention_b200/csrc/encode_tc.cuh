@@ -77,6 +77,8 @@
 // polynomial's 7.5e-5 relative error would be the largest term left).
 #pragma once
 
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 
 namespace flare {
@@ -98,7 +100,53 @@ struct EncodeArgs {
   float* l_part;  // [BH][P][M]
   int* status;    // device status word {code, site}
   unsigned long long wait_ns;
+  // One split per head (splits == 1, P == 1): the CTA writes the normalised
+  // result and the log-sum-exp itself, with the merge's own operations on
+  // the same fp32 values (out = O / l, lse = (mref + log2 l) ln 2), instead
+  // of a partial for lse_merge_kernel.
+  int direct;
+  void* out;                // [BH][M][D]: bf16, or fp32 when out_f32
+  int out_f32;
+  float* lse_out;           // [BH][M] natural log, or null
+  __nv_bfloat16* out_hi;    // fp32 out only: the result as a bf16 pair hi + lo, or null
+  __nv_bfloat16* out_lo;
 };
+
+// Stores n consecutive elements of one row of a direct encode's result:
+// v = acc / l (0 when the row saw no token), as the merge forms it.
+template <int n>
+__device__ __forceinline__ void encode_store_direct(const EncodeArgs& a, size_t e0, const float* acc, float l) {
+  float v[n];
+#pragma unroll
+  for (int z = 0; z < n; ++z) v[z] = l > 0.f ? acc[z] / l : 0.f;
+  if (a.out_f32) {
+    float4* o = reinterpret_cast<float4*>(static_cast<float*>(a.out) + e0);
+#pragma unroll
+    for (int z = 0; z < n / 4; ++z) o[z] = make_float4(v[4 * z], v[4 * z + 1], v[4 * z + 2], v[4 * z + 3]);
+    if (a.out_hi) {
+      uint32_t hi[n / 2], lo[n / 2];
+#pragma unroll
+      for (int z = 0; z < n / 2; ++z) {
+        hi[z] = ptx::pack_bf16(v[2 * z], v[2 * z + 1]);
+        lo[z] = ptx::pack_bf16(v[2 * z] - __uint_as_float(hi[z] << 16), v[2 * z + 1] - __uint_as_float(hi[z] & 0xffff0000u));
+      }
+      uint4* oh = reinterpret_cast<uint4*>(a.out_hi + e0);
+      uint4* ol = reinterpret_cast<uint4*>(a.out_lo + e0);
+#pragma unroll
+      for (int z = 0; z < n / 8; ++z) {
+        oh[z] = make_uint4(hi[4 * z], hi[4 * z + 1], hi[4 * z + 2], hi[4 * z + 3]);
+        ol[z] = make_uint4(lo[4 * z], lo[4 * z + 1], lo[4 * z + 2], lo[4 * z + 3]);
+      }
+    }
+  } else {
+    uint32_t b[n / 2];
+#pragma unroll
+    for (int z = 0; z < n / 2; ++z) b[z] = ptx::pack_bf16(v[2 * z], v[2 * z + 1]);
+    uint4* o = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a.out) + e0);
+#pragma unroll
+    for (int z = 0; z < n / 8; ++z) o[z] = make_uint4(b[4 * z], b[4 * z + 1], b[4 * z + 2], b[4 * z + 3]);
+  }
+}
 
 // Partials per (head, split) written by encode_tc_kernel.
 __host__ __device__ constexpr int encode_partials_per_split(int /*D*/, int /*nhalf*/) { return 1; }
@@ -673,14 +721,23 @@ __global__ void __launch_bounds__(EncodeCfg<D, NHALF, NS, PREC>::kThreads, 1)
             for (int z = 0; z < kChunk; ++z) acc[z] = fmaf(w[a], o[z], acc[z]);
           }
           if (m < args.M) {
+            if (args.direct) {
+              encode_store_direct<kChunk>(args, row * D + c * kHalfD + z0, acc, lsum);
+            } else {
 #pragma unroll
-            for (int z = 0; z < kChunk / 4; ++z)
-              dst[z0 / 4 + z] = make_float4(acc[4 * z], acc[4 * z + 1], acc[4 * z + 2], acc[4 * z + 3]);
+              for (int z = 0; z < kChunk / 4; ++z)
+                dst[z0 / 4 + z] = make_float4(acc[4 * z], acc[4 * z + 1], acc[4 * z + 2], acc[4 * z + 3]);
+            }
           }
         }
         if (m < args.M && c == 0) {
-          args.m_part[row] = ms;
-          args.l_part[row] = lsum;
+          if (args.direct) {
+            constexpr float kLn2 = 0.6931471805599453f;
+            if (args.lse_out) args.lse_out[row] = lsum > 0.f ? (ms + log2f(lsum)) * kLn2 : -INFINITY;
+          } else {
+            args.m_part[row] = ms;
+            args.l_part[row] = lsum;
+          }
         }
       } else {
         record_error(args.status, kErrTimeout, kSiteEncSoftmax);

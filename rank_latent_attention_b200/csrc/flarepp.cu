@@ -425,11 +425,22 @@ int run_encode(const void* Q, int q_batched, const void* K, const void* V, void*
     a.l_part = w.l;
     a.status = status;
     a.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
+    // one split per head: the encode writes the result itself, no merge
+    a.direct = P == 1 ? 1 : 0;
+    a.out = out;
+    a.out_f32 = (f32_out || prec > 0) ? 1 : 0;
+    a.lse_out = lse_out;
+    a.out_hi = split.hi;
+    a.out_lo = split.lo;
     {
       ProfScope prof(FLARE_KERNEL_ENCODE_TC, st);
       e = launch_encode_tc(D, M, prec, maps, a, BH, st, pdl);
     }
     if (e != cudaSuccess) return FLARE_ERR_CUDA;
+    if (a.direct) {
+      *launches += 1;
+      return FLARE_OK;
+    }
     ProfScope prof(FLARE_KERNEL_MERGE, st);
     e = (f32_out || prec > 0) ? launch_merge<float>(w, out, lse_out, BH, P, M, D, st, pdl_merge, split)
                               : launch_merge<__nv_bfloat16>(w, out, lse_out, BH, P, M, D, st, pdl_merge);
@@ -1619,6 +1630,11 @@ int flare_last_launch_count(void) { return t_last_launches; }
 const char* flare_cuda_error_string(void) { return cudaGetErrorString(cudaPeekAtLastError()); }
 
 int flare_set_split_override(int splits) { return g_split_override.exchange(splits < 0 ? 0 : splits); }
+
+int flare_encode_splits(int B, int H, int64_t N) {
+  if (B < 1 || H < 1 || N < 1) return 0;
+  return choose_splits(B * H, N, kEncTile);
+}
 
 int flare_set_wait_limit_ms(int ms) { return g_wait_ms.exchange(ms < 1 ? 1 : ms); }
 

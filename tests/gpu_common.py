@@ -36,6 +36,22 @@ def to_dev(arr: np.ndarray, dtype: str):
     return t.to(torch.bfloat16) if dtype == "bf16" else t
 
 
+def encode_kernels(B: int, H: int, N: int, tensor_cores: bool = True) -> list:
+    """The kernels of one encode: the tensor-core encode is followed by a
+    log-sum-exp merge unless it runs one CTA per head (then it writes its
+    result itself); the CUDA-core encode always merges."""
+    if not tensor_cores:
+        return ["encode_f32", "lse_merge"]
+    import rank_latent_attention_b200 as flare
+    return ["encode_tc"] + (["lse_merge"] if flare.flare_encode_splits(B, H, N) > 1 else [])
+
+
+def mix_kernels(B: int, H: int, N: int, tensor_cores: bool = True) -> list:
+    """The kernels of one flarepp_mix call: two encodes and the decode."""
+    enc = encode_kernels(B, H, N, tensor_cores)
+    return enc + enc + ["decode_tc" if tensor_cores else "decode_f32"]
+
+
 def to_host(t) -> np.ndarray:
     return t.float().cpu().numpy().astype(np.float64)
 
