@@ -32,6 +32,15 @@ def _encode_splits(B, H, N, M, D):
 ])
 def test_encode_split_count(shape, splits):
     assert _encode_splits(*shape) == splits
+    # the host query reports the same count (1: the encode writes its result, no merge)
+    B, H, N = shape[:3]
+    assert flare.flare_encode_splits(B, H, N) == splits
+
+
+def test_split_query_rejects_empty_shapes():
+    assert flare.flare_encode_splits(0, 1, 10) == 0
+    assert flare.flare_encode_splits(1, 0, 10) == 0
+    assert flare.flare_encode_splits(1, 1, 0) == 0
 
 
 def test_override_wins_and_is_clamped():
@@ -39,5 +48,7 @@ def test_override_wins_and_is_clamped():
     try:
         assert _encode_splits(4, 8, 11271, 128, 32) == 3
         assert _encode_splits(1, 1, 100, 16, 16) == 2  # 2 tiles of 64 tokens
+        assert flare.flare_encode_splits(4, 8, 11271) == 3
+        assert flare.flare_encode_splits(1, 1, 100) == 2
     finally:
         flare.flare_set_split_override(old)
