@@ -427,10 +427,14 @@ __global__ void __launch_bounds__(BtcCfg<D>::kThreads, 1)
 // The partial sums of the CTA's token range go to the same [BH][S][M][D] fp32
 // blocks as latent_grad_kernel's, summed by grad_reduce_kernel.
 //
-// Warps 0-3: one latent row per thread.  Warp 4: TMA (two token stages) and
-// MMAs.  TMEM: S [0,64), G [64,128); e and w (bf16 pairs) are written over
-// the first half of S and of G once read; out0 [128, 128+D) (dZ, DEC only),
-// out1 [128+D, 128+2D).
+// Warps 0-3: one latent row per thread.  Warp 4: TMA (a ring of token
+// stages) and MMAs.  TMEM: S [0,64), G [64,128); out0 [128, 128+D) (dZ, DEC
+// only), out1 [128+D, 128+2D).  DEC writes e and w (bf16 pairs) over the first
+// half of S and of G once read, so the next tile's logits wait for the
+// accumulation.  ENC has no out0 and needs no e: w gets 32 columns of its own
+// and the next tile's logits are issued as soon as the rows have read S and
+// G, ahead of this tile's accumulation (a ring of four stages keeps the token
+// loads ahead of the shorter period).
 constexpr int kBltcTok = 64;
 
 struct BltcArgs {
@@ -445,23 +449,28 @@ struct BltcArgs {
   unsigned long long wait_ns;
 };
 
-template <int D>
+template <int D, int MODE>
 struct BltcCfg {
   using G = TileGeom<D>;
   static constexpr int kThreads = 160;
   static constexpr int kIssuerWarp = 4;
+  static constexpr int kStages = MODE == 0 ? 2 : 4;
   static constexpr int kLatBytes = G::bytes(128);
   static constexpr int kTokBytes = G::bytes(kBltcTok);
-  static constexpr int kOffLat = 0;                              // A, B [128][D]
-  static constexpr int kOffTok = 2 * kLatBytes;                  // stage s: K, X
-  static constexpr int kOffStat = kOffTok + 4 * kTokBytes;       // [2 buffers][2][64] floats
+  static constexpr int kOffLat = 0;                                  // A, B [128][D]
+  static constexpr int kOffTok = 2 * kLatBytes;                      // stage s: K, X
+  static constexpr int kOffStat = kOffTok + kStages * 2 * kTokBytes;  // [2 buffers][2][64] floats
   static constexpr int kOffBars = kOffStat + 2 * 2 * kBltcTok * 4;
-  static constexpr int kNumBars = 10;
+  static constexpr int kNumBars = 16;
   static constexpr int kOffMisc = kOffBars + 8 * kNumBars;
   static constexpr int kSmemBytes = kOffMisc + 16 + 1024;
   static constexpr uint32_t kColOut0 = 128;
   static constexpr uint32_t kColOut1 = 128 + D;
   static_assert(kColOut1 + D <= 256, "TMEM budget (256 columns per CTA)");
+  // ENC: w (64 tokens as bf16 pairs) in the first 32 free columns
+  static constexpr uint32_t kColW = kColOut1 + D + kBltcTok / 2 <= 256 ? kColOut1 + D : kColOut0;
+  static_assert(kColW + kBltcTok / 2 <= 256 && (kColW >= kColOut1 + D || kColW + kBltcTok / 2 <= kColOut1),
+                "ENC weight columns");
   static constexpr uint32_t kIdescLogit = ptx::idesc_bf16(128, kBltcTok, 0, 0);
   static constexpr uint32_t kIdescAcc = ptx::idesc_bf16(128, D, 0, 1);
 };
@@ -469,23 +478,27 @@ struct BltcCfg {
 enum { kSiteBwdLatIssuer = 9, kSiteBwdLatWeights = 10 };
 
 template <int D, int MODE>
-__global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
+__global__ void __launch_bounds__(BltcCfg<D, MODE>::kThreads, 1)
     latent_grad_tc_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                           const __grid_constant__ CUtensorMap tmK, const __grid_constant__ CUtensorMap tmX,
                           const BltcArgs args, int a_per_batch_head, int H) {
-  using C = BltcCfg<D>;
+  using C = BltcCfg<D, MODE>;
   using G = typename C::G;
   constexpr bool kDec = MODE == 0;
+  constexpr int NS = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::kOffBars);
   uint64_t* bar_lat = bars + 0;
-  uint64_t* full = bars + 1;   // [2] token stage landed
-  uint64_t* empty = bars + 3;  // [2] token stage consumed by the accumulation MMAs
-  uint64_t* bar_S = bars + 5;
-  uint64_t* bar_W = bars + 6;
-  uint64_t* bar_fin = bars + 7;
-  uint64_t* drain = bars + 8;
+  uint64_t* full = bars + 1;        // [NS] token stage landed
+  uint64_t* empty = bars + 1 + NS;  // [NS] token stage consumed by the accumulation MMAs
+  uint64_t* bar_S = bars + 1 + 2 * NS;
+  uint64_t* bar_W = bar_S + 1;
+  uint64_t* bar_fin = bar_S + 2;
+  uint64_t* drain = bar_S + 3;
+  uint64_t* bar_R = bar_S + 4;     // ENC: the rows have read S and G
+  uint64_t* bar_accd = bar_S + 5;  // ENC: the accumulation has read w
+  static_assert(1 + 2 * NS + 6 <= C::kNumBars, "barrier slots");
   float* sTok = reinterpret_cast<float*>(smem + C::kOffStat);
   uint32_t* s_tmem = reinterpret_cast<uint32_t*>(smem + C::kOffMisc);
   volatile int* s_abort = reinterpret_cast<volatile int*>(smem + C::kOffMisc + 4);
@@ -498,7 +511,7 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
 
   if (threadIdx.x == 0) {
     ptx::mbar_init(bar_lat, 1);
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < NS; ++i) {
       ptx::mbar_init(&full[i], 1);
       ptx::mbar_init(&empty[i], 1);
     }
@@ -506,6 +519,8 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
     ptx::mbar_init(bar_W, 4);
     ptx::mbar_init(bar_fin, 1);
     ptx::mbar_init(drain, 32);
+    ptx::mbar_init(bar_R, 4);
+    ptx::mbar_init(bar_accd, 1);
     *s_abort = 0;
     ptx::fence_mbar_init();
   }
@@ -523,7 +538,7 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
     // ---------------------------------------------------------------- loads + MMAs
     const int planeA = a_per_batch_head ? bh : bh % H;
     auto load_tile = [&](int i) {
-      const int st = i & 1;
+      const int st = i % NS;
       const int tok = (tile0 + i) * kBltcTok;
       ptx::mbar_arrive_expect_tx(&full[st], 2 * C::kTokBytes);
       ptx::tma_load_3d(smem + C::kOffTok + st * 2 * C::kTokBytes, &tmK, &full[st], 0, tok, bh);
@@ -534,10 +549,10 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
       ptx::mbar_arrive_expect_tx(bar_lat, 2 * C::kLatBytes);
       ptx::tma_load_3d(smem + C::kOffLat, &tmA, bar_lat, 0, m0, planeA);
       ptx::tma_load_3d(smem + C::kOffLat + C::kLatBytes, &tmB, bar_lat, 0, m0, bh);
-      for (int i = 0; i < 2 && i < T; ++i) load_tile(i);
+      for (int i = 0; i < NS && i < T; ++i) load_tile(i);
     }
     __syncwarp();
-    loaded = T < 2 ? T : 2;
+    loaded = T < NS ? T : NS;
     bool ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_lat, 0, s_abort, args.wait_ns));
     // Operand descriptors built once: only the start-address field moves
     // between K steps and stages, so each MMA adds a constant (the issuer
@@ -549,9 +564,9 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
     const uint64_t dKmn0 = G::mnmajor(sbase + C::kOffTok, kBltcTok, 0);
     constexpr uint32_t kStageStep = static_cast<uint32_t>(2 * C::kTokBytes) >> 4;
     constexpr uint32_t kXStep = static_cast<uint32_t>(C::kTokBytes) >> 4;
-    // logits of tile i into S/G (stage i & 1 holds its tokens)
+    // logits of tile i into S/G (stage i % NS holds its tokens)
     auto issue_logits = [&](int i) {
-      const int st = i & 1;
+      const int st = i % NS;
       ptx::tc_fence_after();
       if (ptx::elect_one()) {
 #pragma unroll
@@ -565,43 +580,84 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
       }
       __syncwarp();
     };
-    if (ok && T > 0) {
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[0], 0, s_abort, args.wait_ns));
-      if (ok) issue_logits(0);
-    }
-    for (int i = 0; ok && i < T; ++i) {
-      const int st = i & 1;
-      // Every wait before the MMAs (a wait after them stalls until they
-      // complete): the rows' weights of tile i, and the tokens of tile i + 1.
-      ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_W, i & 1, s_abort, args.wait_ns) &&
-                                       (i + 1 >= T || ptx::mbar_wait(&full[st ^ 1], ((i + 1) >> 1) & 1, s_abort,
-                                                                     args.wait_ns)));
-      if (!ok) break;
-      ptx::tc_fence_after();
-      if (ptx::elect_one()) {
-#pragma unroll
-        for (int kk = 0; kk < kBltcTok / 16; ++kk) {
-          const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
-          const uint32_t sm = st * kStageStep + G::mnmajor_step(kk);
-          if constexpr (kDec)
-            ptx::mma_ts(tmem + C::kColOut0, tmem + 0 + kk * 8, dKmn0 + kXStep + sm, C::kIdescAcc, acc);
-          ptx::mma_ts(tmem + C::kColOut1, tmem + 64 + kk * 8, dKmn0 + sm, C::kIdescAcc, acc);
-        }
-        ptx::mma_commit(&empty[st]);
-        if (i == T - 1) ptx::mma_commit(bar_fin);
+    if constexpr (kDec) {
+      if (ok && T > 0) {
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[0], 0, s_abort, args.wait_ns));
+        if (ok) issue_logits(0);
       }
-      __syncwarp();
-      // The next tile's logits overwrite S/G, whose e and w the accumulation
-      // just issued reads: the tensor pipe runs MMAs in issue order, so they
-      // are issued right behind it instead of after it completes and after
-      // the stage refill below (which took ~430 clocks off every tile).
-      if (i + 1 < T) issue_logits(i + 1);
-      if (i + 2 < T) {
-        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&empty[st], (i >> 1) & 1, s_abort, args.wait_ns));
+      for (int i = 0; ok && i < T; ++i) {
+        const int st = i & 1;
+        // Every wait before the MMAs (a wait after them stalls until they
+        // complete): the rows' weights of tile i, and the tokens of tile i + 1.
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_W, i & 1, s_abort, args.wait_ns) &&
+                                         (i + 1 >= T || ptx::mbar_wait(&full[st ^ 1], ((i + 1) >> 1) & 1, s_abort,
+                                                                       args.wait_ns)));
         if (!ok) break;
-        if (ptx::elect_one()) load_tile(i + 2);
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kBltcTok / 16; ++kk) {
+            const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+            const uint32_t sm = st * kStageStep + G::mnmajor_step(kk);
+            ptx::mma_ts(tmem + C::kColOut0, tmem + 0 + kk * 8, dKmn0 + kXStep + sm, C::kIdescAcc, acc);
+            ptx::mma_ts(tmem + C::kColOut1, tmem + 64 + kk * 8, dKmn0 + sm, C::kIdescAcc, acc);
+          }
+          ptx::mma_commit(&empty[st]);
+          if (i == T - 1) ptx::mma_commit(bar_fin);
+        }
         __syncwarp();
-        loaded = i + 3;
+        // The next tile's logits overwrite S/G, whose e and w the accumulation
+        // just issued reads: the tensor pipe runs MMAs in issue order, so they
+        // are issued right behind it instead of after it completes and after
+        // the stage refill below (which took ~430 clocks off every tile).
+        if (i + 1 < T) issue_logits(i + 1);
+        if (i + 2 < T) {
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&empty[st], (i >> 1) & 1, s_abort, args.wait_ns));
+          if (!ok) break;
+          if (ptx::elect_one()) load_tile(i + 2);
+          __syncwarp();
+          loaded = i + 3;
+        }
+      }
+    } else {
+      // Tile i + 1's logits go out once the rows have read S and G of tile i
+      // (and its tokens have landed), ahead of tile i's accumulation: the
+      // rows then find the next logits done when they finish a tile.
+      if (ok && T > 0) {
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(&full[0], 0, s_abort, args.wait_ns));
+        if (ok) issue_logits(0);
+      }
+      for (int i = 0; ok && i < T; ++i) {
+        const int st = i % NS;
+        if (i + 1 < T) {
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_R, i & 1, s_abort, args.wait_ns) &&
+                                           ptx::mbar_wait(&full[(i + 1) % NS], ((i + 1) / NS) & 1, s_abort,
+                                                          args.wait_ns));
+          if (!ok) break;
+          issue_logits(i + 1);
+        }
+        ok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_W, i & 1, s_abort, args.wait_ns));
+        if (!ok) break;
+        ptx::tc_fence_after();
+        if (ptx::elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < kBltcTok / 16; ++kk) {
+            const uint32_t acc = (i > 0 || kk > 0) ? 1u : 0u;
+            ptx::mma_ts(tmem + C::kColOut1, tmem + C::kColW + kk * 8, dKmn0 + st * kStageStep + G::mnmajor_step(kk),
+                        C::kIdescAcc, acc);
+          }
+          ptx::mma_commit(&empty[st]);
+          ptx::mma_commit(bar_accd);
+          if (i == T - 1) ptx::mma_commit(bar_fin);
+        }
+        __syncwarp();
+        if (i + NS < T) {
+          ok = __all_sync(0xffffffffu, ptx::mbar_wait(&empty[st], (i / NS) & 1, s_abort, args.wait_ns));
+          if (!ok) break;
+          if (ptx::elect_one()) load_tile(i + NS);
+          __syncwarp();
+          loaded = i + NS + 1;
+        }
       }
     }
     if (!ok) {
@@ -610,7 +666,7 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
     }
     ptx::mma_commit(drain);
     ptx::mbar_wait_drain(drain, 0);
-    for (int t = (loaded > 2 ? loaded - 2 : 0); t < loaded; ++t) ptx::mbar_wait_drain(&full[t & 1], (t >> 1) & 1);
+    for (int t = (loaded > NS ? loaded - NS : 0); t < loaded; ++t) ptx::mbar_wait_drain(&full[t % NS], (t / NS) & 1);
     ptx::mbar_wait_drain(bar_lat, 0);
   } else {
     // ---------------------------------------------------------------- weights
@@ -660,44 +716,85 @@ __global__ void __launch_bounds__(BltcCfg<D>::kThreads, 1)
       const float4* stat4 = reinterpret_cast<const float4*>(stat);
       const uint64_t kL2e2 = ptx::f2(kL2e, kL2e);
       const uint64_t nL = ptx::f2(-Lm, -Lm), nc = ptx::f2(-cm, -cm);
+      if constexpr (!kDec) {
+        // All of S and G read at once (128 registers a thread): the rows
+        // release S/G to the next tile's logits (bar_R) before computing, and
+        // before the first store of w wait for the accumulation of tile i - 1,
+        // which reads the same columns.
+        float sv[4][16], gv[4][16];
 #pragma unroll
-      for (int p = 0; p < 4; ++p) {
-        float sv[16], gv[16];
-        ptx::tmem_ld16(trow + 0 + 16 * p, sv);
-        ptx::tmem_ld16(trow + 64 + 16 * p, gv);
-        ptx::tmem_wait_ld();
-        uint32_t pe[8], pw[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int j = 16 * p + 2 * u;  // tokens j, j + 1
-          uint64_t a, b;
-          if constexpr (kDec) {
-            const float4 tj = stat4[j / 2];  // {lse3, delta} of tokens j and j + 1
-            a = ptx::fma2(ptx::f2(sv[2 * u], sv[2 * u + 1]), kL2e2, ptx::f2(-tj.x, -tj.z));
-            b = ptx::add2(ptx::f2(gv[2 * u], gv[2 * u + 1]), ptx::f2(-tj.y, -tj.w));
-          } else {
-            a = ptx::fma2(ptx::f2(sv[2 * u], sv[2 * u + 1]), kL2e2, nL);
-            b = ptx::add2(ptx::f2(gv[2 * u], gv[2 * u + 1]), nc);
-          }
-          float a0, a1;
-          ptx::f2_split(a, a0, a1);
-          const uint64_t e = ptx::f2(ptx::ex2(a0), ptx::ex2(a1));
-          const uint64_t w = ptx::mul2(e, b);
-          float e0, e1, w0, w1;
-          ptx::f2_split(e, e0, e1);
-          ptx::f2_split(w, w0, w1);
-          if (ragged) {
-            e0 = j < live_cols ? e0 : 0.f;
-            w0 = j < live_cols ? w0 : 0.f;
-            e1 = j + 1 < live_cols ? e1 : 0.f;
-            w1 = j + 1 < live_cols ? w1 : 0.f;
-          }
-          pe[u] = ptx::pack_bf16(e0, e1);
-          pw[u] = ptx::pack_bf16(w0, w1);
+        for (int p = 0; p < 4; ++p) {
+          ptx::tmem_ld16(trow + 0 + 16 * p, sv[p]);
+          ptx::tmem_ld16(trow + 64 + 16 * p, gv[p]);
         }
-        // over columns of S and G this thread has already read
-        ptx::tmem_st8(trow + 0 + 8 * p, pe);
-        ptx::tmem_st8(trow + 64 + 8 * p, pw);
+        ptx::tmem_wait_ld();
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(bar_R);
+        bool wok = true;
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          uint32_t pw[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = 16 * p + 2 * u;  // tokens j, j + 1
+            const uint64_t a = ptx::fma2(ptx::f2(sv[p][2 * u], sv[p][2 * u + 1]), kL2e2, nL);
+            const uint64_t b = ptx::add2(ptx::f2(gv[p][2 * u], gv[p][2 * u + 1]), nc);
+            float a0, a1;
+            ptx::f2_split(a, a0, a1);
+            const uint64_t w = ptx::mul2(ptx::f2(ptx::ex2(a0), ptx::ex2(a1)), b);
+            float w0, w1;
+            ptx::f2_split(w, w0, w1);
+            if (ragged) {
+              w0 = j < live_cols ? w0 : 0.f;
+              w1 = j + 1 < live_cols ? w1 : 0.f;
+            }
+            pw[u] = ptx::pack_bf16(w0, w1);
+          }
+          if (p == 0 && i > 0) {
+            wok = __all_sync(0xffffffffu, ptx::mbar_wait(bar_accd, (i - 1) & 1, s_abort, args.wait_ns));
+            ptx::tc_fence_after();
+          }
+          ptx::tmem_st8(trow + C::kColW + 8 * p, pw);
+        }
+        if (!wok) {
+          ok = false;
+          break;
+        }
+      } else {
+#pragma unroll
+        for (int p = 0; p < 4; ++p) {
+          float sv[16], gv[16];
+          ptx::tmem_ld16(trow + 0 + 16 * p, sv);
+          ptx::tmem_ld16(trow + 64 + 16 * p, gv);
+          ptx::tmem_wait_ld();
+          uint32_t pe[8], pw[8];
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int j = 16 * p + 2 * u;  // tokens j, j + 1
+            const float4 tj = stat4[j / 2];  // {lse3, delta} of tokens j and j + 1
+            const uint64_t a = ptx::fma2(ptx::f2(sv[2 * u], sv[2 * u + 1]), kL2e2, ptx::f2(-tj.x, -tj.z));
+            const uint64_t b = ptx::add2(ptx::f2(gv[2 * u], gv[2 * u + 1]), ptx::f2(-tj.y, -tj.w));
+            float a0, a1;
+            ptx::f2_split(a, a0, a1);
+            const uint64_t e = ptx::f2(ptx::ex2(a0), ptx::ex2(a1));
+            const uint64_t w = ptx::mul2(e, b);
+            float e0, e1, w0, w1;
+            ptx::f2_split(e, e0, e1);
+            ptx::f2_split(w, w0, w1);
+            if (ragged) {
+              e0 = j < live_cols ? e0 : 0.f;
+              w0 = j < live_cols ? w0 : 0.f;
+              e1 = j + 1 < live_cols ? e1 : 0.f;
+              w1 = j + 1 < live_cols ? w1 : 0.f;
+            }
+            pe[u] = ptx::pack_bf16(e0, e1);
+            pw[u] = ptx::pack_bf16(w0, w1);
+          }
+          // over columns of S and G this thread has already read
+          ptx::tmem_st8(trow + 0 + 8 * p, pe);
+          ptx::tmem_st8(trow + 64 + 8 * p, pw);
+        }
       }
       ptx::tmem_wait_st();
       ptx::tc_fence_before();

@@ -938,7 +938,8 @@ cudaError_t launch_dyn(K kernel, dim3 grid, int smem, cudaStream_t st, const Bwd
 
 template <int D, int MODE>
 cudaError_t launch_latent_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH, cudaStream_t st) {
-  using C = BltcCfg<D>;
+  constexpr int kMode = MODE == kBwdDec ? 0 : 1;
+  using C = BltcCfg<D, kMode>;
   CUtensorMap mA, mB, mK, mX;
   const int64_t N = a.N;
   const void* A = MODE == kBwdEncSeed ? a.seeds : w.Qd;
@@ -962,7 +963,6 @@ cudaError_t launch_latent_grad_tc(const BwdArgs& a, const BackwardWs& w, int BH,
   t.wait_ns = static_cast<unsigned long long>(g_wait_ms.load()) * 1000000ull;
   // at least 80 KB of shared memory: at most two CTAs per SM, each with 256 TMEM columns
   const int smem = C::kSmemBytes > 80 * 1024 ? C::kSmemBytes : 80 * 1024;
-  constexpr int kMode = MODE == kBwdDec ? 0 : 1;
   auto kern = latent_grad_tc_kernel<D, kMode>;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
