@@ -90,6 +90,36 @@ def test_backward_matches_oracle(name, spec):
             assert_backward_bar(f"{w.name}.{n}.exact", g, r, w.dtype, True)
 
 
+@pytest.mark.parametrize("spec", [(1, 2, 64 * 13 + 5, 256, 64), (1, 2, 64 * 9 + 33, 144, 32),
+                                  (2, 1, 64 * 7 + 1, 48, 16)], ids=str)
+def test_backward_many_tiles_per_cta(spec):
+    """One and three token splits per head: every backward kernel runs several
+    token tiles per CTA (14, 10 and 8 of the latent kernel's 64 tokens at one
+    split), so its stage rings wrap -- four stages in the encode part, two in
+    the decode part -- and the ragged last tile comes after full ones.  The
+    default split rule gives these sizes one tile per CTA."""
+    require_cuda()
+    B, H, N, M, D = spec
+    w = inputs.custom(B, H, N, M, D, dtype="bf16", seed_index=90 + N % 13)
+    exact = None
+    for splits in (1, 3):
+        old = flare.flare_set_split_override(splits)
+        try:
+            (seeds, K, V, dY), got, Qd, Z, _ = _run(w)
+        finally:
+            flare.flare_set_split_override(old)
+        args = [x.astype(np.float64) for x in (seeds, K, V, dY)]
+        stored = oracle.flarepp_backward(*args, Q_dyn=Qd, Z=Z)
+        if exact is None:
+            exact = oracle.flarepp_backward(*args)
+        print(f"{spec} splits={splits}: stored {_excess(got, stored, 2.0 ** -8)} exact {_excess(got, exact, 2.0 ** -8)}")
+        for n, g, r in zip(NAMES, got, stored):
+            assert np.all(np.isfinite(g))
+            assert_backward_bar(f"{spec}/{splits}.{n}.stored", g, r, "bf16", True)
+        for n, g, r in zip(NAMES, got, exact):
+            assert_backward_bar(f"{spec}/{splits}.{n}.exact", g, r, "bf16", True)
+
+
 def test_workspace_and_stream():
     import torch
 
