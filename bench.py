@@ -854,7 +854,7 @@ def small_configs(torch, flare, inputs, dev, peaks):
                     "tflops_cold": flops / (ms_c * 1e-3) / 1e12, "roofline_ms": t_roof,
                     "roofline_parts_ms": {"tensor": t_tensor, "hbm": t_hbm, "mufu": t_mufu},
                     "bound": bound, "frac_cold": t_roof / ms_c,
-                    "calls": 20,
+                    "calls": 20, "launches_per_call": len(per_launch),
                     "launch_us": [[k, t] for (k, _), t in zip(recs[-len(per_launch):], per_launch)]}
         del s_d, K_d, V_d, Y_d, ws
     del scrub
